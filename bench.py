@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 triangle multiplicative update.
+
+One step = one pass of the whole layer in both directions (outgoing, then
+incoming) over one synthetic pair representation: per direction the prologue,
+contraction and epilogue kernels, called through the C ABI. The default
+workload is the Boltz-2 crop size N = 768 (bf16, c_z = c_h = 128, per-channel
+scale on z). The metric is pair-cells/s (one cell through one direction of the
+layer is one pair-cell); algorithmic TFLOP/s is reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs an independent replica on its
+own GPU (the layer is not sharded); value = cells of all ranks / max time.
+
+Timing: CUDA events on the launching stream; L2 is flushed (512 MB write)
+before every step and the flush is outside the timed events; a barrier and a
+device synchronize bracket the K timed steps on every rank.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "trimul pair-cells/s and TFLOP/s at N=768 bf16 (% of B200 tensor peak)"
+UNIT = "pair-cells/s"
+DEFAULT_WORKLOAD = 3
+FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ("prologue_tc_kernel", "contract_tc_kernel", "epilogue_tc_kernel")
+
+
+def flops_per_cell(N: int) -> int:
+    """Algorithmic FLOP per cell and direction: projections 2*(4*128*128 + 128*128 + 128*128), contraction 2*N*128."""
+    return 196608 + 256 * N
+
+
+def kernel_algorithmic(N: int):
+    """Per launch: (quantity, unit, bound) of each kernel's algorithmic work."""
+    cells = N * N
+    return {
+        "prologue_tc_kernel": (cells * (256 + 2 + 512) + 4 * 128 * 128 * 2, "bytes", "hbm"),
+        "contract_tc_kernel": (2 * N ** 3 * 128, "flop", "tensor"),
+        "epilogue_tc_kernel": (cells * (256 + 256 + 256) + 2 * 128 * 128 * 2, "bytes", "hbm"),
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(kernel: str) -> str:
+    fname = {"prologue_tc_kernel": "prologue_tc.cu", "contract_tc_kernel": "contract_tc.cu",
+             "epilogue_tc_kernel": "epilogue_tc.cu"}[kernel]
+    h = hashlib.sha256()
+    for f in (fname, "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "pair_representation_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, N: int):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None when there is none for this kernel at this N or the kernel's source
+    has changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rows = json.load(f)
+    for r in rows.get("kernels", []):
+        if r.get("kernel") == kernel and r.get("N") == N and r.get("src_sha") == source_sha(kernel):
+            return int(r["dram_bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+
+    BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.nvml = None
+            self.err = str(e)
+        self.period = period_s
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.BITS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nvml:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline)
+
+def oracle_sample(workload, n_idx: int, seed: int = 0, threads=None):
+    """Run the oracle on the sampled grid I x I (|I| = n_idx) in every direction of the
+    workload; returns (cells computed, seconds)."""
+    import numpy as np
+
+    import oracle
+    import pair_inputs as pi
+    rng = np.random.default_rng([workload.seed, 77, seed])
+    I = np.sort(rng.choice(workload.N, size=min(n_idx, workload.N), replace=False)).astype(np.int32)
+    case = pi.make_workload(workload)
+    t0 = time.perf_counter()
+    cells = 0
+    for d in workload.directions:
+        oracle.trimul_grid(case, d, I, threads=threads)
+        cells += len(I) ** 2
+    return cells, time.perf_counter() - t0
+
+
+def calibrated_oracle(workload, budget_s: float, threads=None):
+    """Choose |I| so the oracle sample takes about budget_s seconds, then run it."""
+    cells, t = oracle_sample(workload, 8, seed=1, threads=threads)
+    per_line = t / 8.0  # projection cost is linear in |I| and dominates
+    n_idx = int(max(8, min(workload.N, budget_s / max(per_line, 1e-6))))
+    cells, t = oracle_sample(workload, n_idx, threads=threads)
+    return cells, t, n_idx
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import pair_inputs as pi
+    import pair_representation_b200 as tm
+    from pair_representation_b200 import build as tmbuild
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        tmbuild.build()
+    if dist:
+        dist.barrier()
+    tm.lib()
+
+    w = pi.WORKLOADS[args.workload]
+    N = w.N
+    case = pi.make_workload(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    z_host = torch.from_numpy(case["z"]).to(tdt).pin_memory()
+    m_host = torch.from_numpy(case["mask"]).to(tdt).pin_memory()
+    z = z_host.to(dev)
+    mask = m_host.to(dev)
+    layers = {}
+    for name, cls in (("outgoing", tm.TriangleMultiplicationOutgoing), ("incoming", tm.TriangleMultiplicationIncoming)):
+        sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+        layers[name] = cls(128, 128).load_state_dict(sd).to(dev, tdt)
+    dirs = list(w.directions)
+    code = {"outgoing": tm.OUTGOING, "incoming": tm.INCOMING}
+    params = {d: layers[d].params(N) for d in dirs}
+    outs = {d: torch.empty_like(z) for d in dirs}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    names = ("prologue_tc_kernel", "contract_tc_kernel", "epilogue_tc_kernel") if w.dtype == "bf16" else \
+        ("prologue_f32_kernel", "contract_f32_kernel", "epilogue_f32_kernel")
+
+    def one_step(evs):
+        for d in dirs:
+            p = params[d]
+            evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            tm.trimul_prologue(z, mask, p, sh)
+            evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            tm.trimul_contract(p, code[d], sh)
+            evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            tm.trimul_epilogue(z, p, outs[d], sh)
+        evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step([])
+    torch.cuda.synchronize()
+    for d in dirs:
+        rc, detail = tm.trimul_device_status(params[d], sh)
+        if rc != 0:
+            raise RuntimeError(f"device status {rc} {detail}")
+
+    sampler = ClockSampler(local_rank)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    step_events = []
+    for _ in range(args.steps):
+        flush.zero_()
+        evs = []
+        one_step(evs)
+        step_events.append(evs)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if dist:
+        dist.barrier()
+
+    step_ms = [evs[0].elapsed_time(evs[-1]) for evs in step_events]
+    total_ms = sum(step_ms)
+    kern_ms = {n: 0.0 for n in names}
+    for evs in step_events:
+        for k, d in enumerate(dirs):
+            for s, n in enumerate(names):
+                kern_ms[n] += evs[3 * k + s].elapsed_time(evs[3 * k + s + 1])
+    launches = {n: args.steps * len(dirs) for n in names}
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- end to end through the public layer API, host buffers in and out
+    e2e = None
+    if not args.no_e2e:
+        out_host = {d: torch.empty(z.shape, dtype=tdt, pin_memory=True) for d in dirs}
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            zd = z_host.to(dev, non_blocking=True)
+            md = m_host.to(dev, non_blocking=True)
+            for d in dirs:
+                o = layers[d](zd, md, out=outs[d], stream=stream)
+                out_host[d].copy_(o, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e2e_ms = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0.record(stream)
+            e2e_step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms += ev0.elapsed_time(ev1)
+        if dist:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * args.steps * len(dirs) * N * N / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": z_host.numel() * z_host.element_size() + m_host.numel() * m_host.element_size(),
+               "d2h_bytes_per_step": sum(out_host[d].numel() * out_host[d].element_size() for d in dirs)}
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    alg = kernel_algorithmic(N)
+    dom = max(kern_ms, key=lambda n: kern_ms[n])
+    per_launch_s = kern_ms[dom] / launches[dom] / 1e3
+    breakdown = {}
+    for n in names:
+        avg = kern_ms[n] / launches[n] / 1e3
+        entry = {"avg_us": round(avg * 1e6, 2), "share": round(kern_ms[n] / sum(kern_ms.values()), 4)}
+        if n in alg:
+            q, u, bound = alg[n]
+            if u == "bytes":
+                entry["achieved_gbs"] = round(q / avg / 1e9, 1)
+                entry["frac_hbm"] = round(q / avg / 1e9 / peaks["hbm_gbs"], 4)
+            else:
+                entry["achieved_tflops"] = round(q / avg / 1e12, 1)
+                entry["frac_tensor"] = round(q / avg / 1e12 / peaks["bf16_tflops"], 4)
+        breakdown[n] = entry
+    roofline = None
+    if dom in alg:
+        q, u, bound = alg[dom]
+        if u == "bytes":
+            achieved, peak, unit = q / per_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            achieved, peak, unit = q / per_launch_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        roofline = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                    "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, N),
+                    "peak_source": f"{peak_src} ({'burst' if u != 'bytes' else 'copy'})"}
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 only, N = 1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cells, secs, n_idx = calibrated_oracle(w, args.oracle_seconds)
+        cpu = {"value": cells / secs, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"float64 oracle (grid mode) on {n_idx} x {n_idx} sampled cells of the N={N} "
+                         f"workload, {'+'.join(dirs)}: {cells} pair-cells in {secs:.1f} s"}
+
+    cells_total = world * args.steps * len(dirs) * N * N
+    value = cells_total / (total_ms / 1e3)
+    tflops = world * args.steps * len(dirs) * N * N * flops_per_cell(N) / (total_ms / 1e3) / 1e12
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "c_z": 128, "c_h": 128, "batch": 1, "directions": dirs,
+                   "l2": "flushed (512 MB write) before every step, outside the timed events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "tflops": round(tflops, 2),
+        "tflops_frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+        "roofline": roofline,
+        "kernels": breakdown,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": sum(launches.values()),
+        "clocks": clocks,
+    }
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The float64 oracle as it stands, on the host cores, on bounded samples of the workload."""
+    if rank != 0:
+        return
+    import pair_inputs as pi
+    w = pi.WORKLOADS[args.workload]
+    per_step = max(1.0, args.reference_budget / max(1, args.steps + args.warmup))
+    cells, t = 0, 0.0
+    _, _, n_idx = calibrated_oracle(w, per_step)
+    for k in range(args.warmup):
+        oracle_sample(w, n_idx, seed=100 + k)
+    for k in range(args.steps):
+        c, s = oracle_sample(w, n_idx, seed=k)
+        cells += c
+        t += s
+    value = cells / t
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "N": w.N, "c_z": 128, "c_h": 128, "batch": 1,
+                   "directions": list(w.directions)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"each step: float64 oracle (grid mode) on {n_idx} x {n_idx} sampled cells "
+                                   f"of the N={w.N} workload, {'+'.join(w.directions)}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=(1, 2, 3, 4, 5))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-budget", type=float, default=120.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

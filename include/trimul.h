@@ -1,0 +1,141 @@
+/*
+ * trimul.h - C ABI of the B200 (sm_100a) triangle multiplicative update.
+ *
+ * The layer is the pair-representation update the pages call
+ * TriangleMultiplicationOutgoing, invoked as layer(x, mask) after loading a
+ * state dict ("Scaling biomolecular modeling with context parallelism in
+ * NVIDIA BioNeMo", section "Context-parallel implementation of triangle
+ * multiplication"), together with its incoming counterpart. Per cell (i, j)
+ * of the N x N pair representation z (c_z channels):
+ *
+ *   zh    = LayerNorm_in(z)                                   (over c_z)
+ *   a     = mask * sigmoid(W_ag zh + b_ag) * (W_a zh + b_a)  (c_h channels)
+ *   b     = mask * sigmoid(W_bg zh + b_bg) * (W_b zh + b_b)
+ *   x_ij  = sum_k a_ik * b_jk      (TRIMUL_OUTGOING)
+ *   x_ij  = sum_k a_ki * b_kj      (TRIMUL_INCOMING)
+ *   out   = sigmoid(W_g zh + b_g) * (W_o LayerNorm_out(x) + b_o)
+ *
+ * LayerNorm uses the biased variance over its channels and eps inside the
+ * square root. The mask multiplies a and b at their own cell only.
+ *
+ * Layouts (row-major, contiguous, element type = params.dtype):
+ *   z, out   [N][N][c_z]   channel-last pair representation
+ *   mask     [N][N]        or NULL (all ones)
+ *   W_a, W_ag, W_b, W_bg  [c_h][c_z];  W_g [c_z][c_z];  W_o [c_z][c_h]
+ *            PyTorch Linear layout [out][in], y = W x + b
+ *   biases, LayerNorm weight/bias: vectors, or NULL (bias 0, gamma 1, beta 0)
+ *
+ * Ownership and threading: the caller owns every buffer, including the
+ * workspace. The library allocates nothing, frees nothing and does not
+ * synchronise in trimul_forward or the stage calls: work is enqueued on
+ * `stream` and the call returns. Its only global state is per-device launch
+ * configuration (maximum shared memory attribute, SM count, cached driver
+ * entry point), set up once and guarded for concurrent callers.
+ *
+ * Errors: every call returns TRIMUL_OK (0) or a negative code; no exception
+ * crosses this boundary. Argument errors are detected on the host before any
+ * work is enqueued. Errors found by a kernel (a bounded wait that ran out) are
+ * written to a status word in the workspace and read with trimul_device_status.
+ *
+ * Version 1 supports c_z == c_h == 128, batch 1, dtype F32 (CUDA-core fp32
+ * kernels) or BF16 (tcgen05 tensor-core kernels with fp32 accumulation).
+ */
+#ifndef TRIMUL_B200_H
+#define TRIMUL_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st *trimul_stream_t;
+
+enum trimul_direction { TRIMUL_OUTGOING = 0, TRIMUL_INCOMING = 1 };
+enum trimul_dtype { TRIMUL_DTYPE_F32 = 0, TRIMUL_DTYPE_BF16 = 1 };
+
+enum trimul_status {
+    TRIMUL_OK = 0,
+    TRIMUL_ERR_INVALID_ARG = -1,  /* NULL required pointer, N < 1 or too large, bad direction */
+    TRIMUL_ERR_UNSUPPORTED = -2,  /* c_z or c_h != 128, unknown dtype, no sm_100 device */
+    TRIMUL_ERR_MISALIGNED = -3,   /* a pointer the kernels read with TMA is not 16-byte aligned */
+    TRIMUL_ERR_ALIAS = -4,        /* out overlaps z, the mask or the workspace */
+    TRIMUL_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than trimul_workspace_size_dtype */
+    TRIMUL_ERR_CUDA = -6,         /* a CUDA runtime / driver call failed (launch, tensor map) */
+    TRIMUL_ERR_TIMEOUT = -7,      /* device: a bounded in-kernel wait ran out; results invalid */
+    TRIMUL_ERR_DEVICE = -8        /* device: another kernel-detected fault; results invalid */
+};
+
+/* Debug flags (0 in production). */
+#define TRIMUL_DEBUG_STALL_CONTRACT 0x1u /* contraction's MMA issuer waits on a barrier nothing
+                                            signals, so its bounded wait runs out (failure test) */
+
+typedef struct trimul_params {
+    int N;              /* residues; 1 <= N <= 16384 */
+    int c_z, c_h;       /* channels; both must be 128 in version 1 */
+    int dtype;          /* enum trimul_dtype: element type of z, mask, weights, out */
+    float ln_eps;       /* LayerNorm epsilon for both LayerNorms (1e-5 = torch default) */
+    const void *ln_in_w, *ln_in_b;     /* [c_z] or NULL */
+    const void *w_a, *w_ag, *w_b, *w_bg; /* [c_h][c_z], required */
+    const void *b_a, *b_ag, *b_b, *b_bg; /* [c_h] or NULL */
+    const void *w_g, *b_g;             /* [c_z][c_z] required; [c_z] or NULL */
+    const void *ln_out_w, *ln_out_b;   /* [c_h] or NULL */
+    const void *w_o, *b_o;             /* [c_z][c_h] required; [c_z] or NULL */
+    void *workspace;                   /* device memory, 256-byte aligned */
+    size_t workspace_bytes;
+    uint32_t timeout_ms;               /* bound on any in-kernel wait; 0 = 2000 ms */
+    uint32_t debug_flags;              /* TRIMUL_DEBUG_*; 0 in production */
+} trimul_params;
+
+/* Bytes of workspace that trimul_forward needs for any dtype (sized for the
+ * fp32 element). Returns 0 for invalid sizes. The workspace holds a 256-byte
+ * status header and a, b, x as [c_h][N][ld] with ld = N rounded up to 8. */
+size_t trimul_workspace_size(int N, int c_z, int c_h);
+
+/* Exact bytes of workspace for one dtype (<= trimul_workspace_size). */
+size_t trimul_workspace_size_dtype(int N, int c_z, int c_h, int dtype);
+
+/* The whole layer: out = TriMul_direction(z, mask). Enqueues three kernels
+ * (prologue, contraction, epilogue) on `stream` after clearing the workspace
+ * status word. z, out, weights and the workspace must be 16-byte aligned;
+ * out must not overlap z, mask or the workspace. Asynchronous. */
+int trimul_forward(const void *z, const void *mask, const trimul_params *p, int direction,
+                   void *out, trimul_stream_t stream);
+
+/* The three stages of trimul_forward, for callers that time or check them one
+ * at a time. Each is asynchronous and needs the same params.
+ *  prologue: z, mask -> a, b in the workspace (channel-major [c_h][N][ld])
+ *  contract: a, b -> x in the workspace, x_c = a_c b_c^T (outgoing) or a_c^T b_c
+ *  epilogue: x, z -> out
+ * trimul_prologue also clears the status word. */
+int trimul_prologue(const void *z, const void *mask, const trimul_params *p, trimul_stream_t stream);
+int trimul_contract(const trimul_params *p, int direction, trimul_stream_t stream);
+int trimul_epilogue(const void *z, const trimul_params *p, void *out, trimul_stream_t stream);
+
+/* Device pointers of a, b and x inside p->workspace and their leading
+ * dimension in elements (each is [c_h][N][ld] of p->dtype). Host-only. */
+int trimul_workspace_views(const trimul_params *p, void **a, void **b, void **x, size_t *ld);
+
+/* Synchronises `stream`, then returns the status word the kernels wrote
+ * since it was last cleared: TRIMUL_OK, TRIMUL_ERR_TIMEOUT or
+ * TRIMUL_ERR_DEVICE (or TRIMUL_ERR_CUDA if reading it failed). If `detail` is
+ * not NULL it receives 4 ints: code, site, block index, auxiliary value. */
+int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *detail);
+
+/* Static description of a status code. */
+const char *trimul_error_string(int code);
+
+/* Human-readable detail of the last error this thread saw (the failing CUDA
+ * call and its message), or "" if none. Valid until the next call. */
+const char *trimul_last_error_detail(void);
+
+/* Library version (major * 100 + minor). */
+int trimul_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRIMUL_B200_H */

@@ -1,0 +1,505 @@
+// api.cu - the C ABI declared in include/trimul.h: argument checks, workspace
+// carve-up, TMA descriptors and the launch sequence of the three stages.
+//
+// Nothing here allocates device memory or synchronises, except
+// trimul_device_status, whose contract is to synchronise.
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+#include "trimul.h"
+
+using namespace trimul;
+
+namespace {
+
+constexpr int kMaxN = 16384;
+constexpr size_t kHeader = 256;  // DeviceStatus lives at the start of the workspace
+constexpr int kMaxDevices = 64;
+
+thread_local char g_detail[512];
+
+void set_detail(const char *what, cudaError_t e) {
+    snprintf(g_detail, sizeof g_detail, "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+size_t ld_of(int N) { return ((size_t)N + 7) & ~(size_t)7; }
+size_t elem_size(int dtype) { return dtype == TRIMUL_DTYPE_F32 ? 4 : 2; }
+size_t section_bytes(int N, int dtype) { return round_up((size_t)kC * (size_t)N * ld_of(N) * elem_size(dtype), 256); }
+
+bool valid_dtype(int d) { return d == TRIMUL_DTYPE_F32 || d == TRIMUL_DTYPE_BF16; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool overlap(const void *p, size_t pn, const void *q, size_t qn) {
+    if (!p || !q || !pn || !qn) return false;
+    const uintptr_t a = (uintptr_t)p, b = (uintptr_t)q;
+    return a < b + qn && b < a + pn;
+}
+
+// ---- per-device state ------------------------------------------------------
+
+struct DevState {
+    bool init = false;
+    int sms = 0;
+    int cc_major = 0, cc_minor = 0;
+    cudaError_t tc_setup = cudaSuccess;
+};
+
+std::mutex g_mu;
+DevState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_state(const DevState **out, bool need_tc) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_detail("cudaGetDevice", e);
+        return TRIMUL_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return TRIMUL_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevState &d = g_dev[dev];
+    if (!d.init) {
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) {
+            set_detail("cudaDeviceGetAttribute", e);
+            return TRIMUL_ERR_CUDA;
+        }
+        if (d.cc_major == 10 && d.cc_minor == 0) {
+            if ((e = prologue_tc_setup()) == cudaSuccess && (e = contract_tc_setup()) == cudaSuccess)
+                e = epilogue_tc_setup();
+            d.tc_setup = e;
+        } else {
+            d.tc_setup = cudaErrorNoKernelImageForDevice;
+        }
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e == cudaSuccess && q == cudaDriverEntryPointSuccess && fn)
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        d.init = true;
+    }
+    if (need_tc) {
+        if (d.cc_major != 10 || d.cc_minor != 0) {
+            snprintf(g_detail, sizeof g_detail, "bf16 path needs sm_100 (found sm_%d%d)", d.cc_major, d.cc_minor);
+            return TRIMUL_ERR_UNSUPPORTED;
+        }
+        if (d.tc_setup != cudaSuccess) {
+            set_detail("kernel attribute setup", d.tc_setup);
+            return TRIMUL_ERR_CUDA;
+        }
+        if (!g_encode) {
+            snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled entry point unavailable");
+            return TRIMUL_ERR_CUDA;
+        }
+    }
+    *out = &d;
+    return TRIMUL_OK;
+}
+
+// A pointer the kernels dereference must be device (or managed) memory.
+int check_device_ptr(const void *p, const char *name) {
+    if (!p) return TRIMUL_OK;
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        set_detail(name, e);
+        return TRIMUL_ERR_INVALID_ARG;
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) {
+        snprintf(g_detail, sizeof g_detail, "%s is not device memory", name);
+        return TRIMUL_ERR_INVALID_ARG;
+    }
+    return TRIMUL_OK;
+}
+
+// ---- argument checks (pure host logic, no CUDA calls) ------------------------
+
+int check_params(const trimul_params *p) {
+    if (!p) return TRIMUL_ERR_INVALID_ARG;
+    if (p->N < 1 || p->N > kMaxN || p->c_z < 1 || p->c_h < 1) return TRIMUL_ERR_INVALID_ARG;
+    if (p->c_z != kC || p->c_h != kC || !valid_dtype(p->dtype)) return TRIMUL_ERR_UNSUPPORTED;
+    if (!(p->ln_eps > 0.f) || p->ln_eps > 1.f) return TRIMUL_ERR_INVALID_ARG;
+    const void *req[] = {p->w_a, p->w_ag, p->w_b, p->w_bg, p->w_g, p->w_o};
+    for (const void *w : req) {
+        if (!w) return TRIMUL_ERR_INVALID_ARG;
+        if (!aligned(w, 16)) return TRIMUL_ERR_MISALIGNED;
+    }
+    const size_t es = elem_size(p->dtype);
+    const void *vec[] = {p->ln_in_w, p->ln_in_b, p->b_a, p->b_ag, p->b_b, p->b_bg,
+                         p->b_g, p->ln_out_w, p->ln_out_b, p->b_o};
+    for (const void *v : vec)
+        if (v && !aligned(v, es)) return TRIMUL_ERR_MISALIGNED;
+    if (!p->workspace || p->workspace_bytes < trimul_workspace_size_dtype(p->N, p->c_z, p->c_h, p->dtype))
+        return TRIMUL_ERR_WORKSPACE;
+    if (!aligned(p->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
+    return TRIMUL_OK;
+}
+
+size_t pair_bytes(const trimul_params *p) { return (size_t)p->N * p->N * kC * elem_size(p->dtype); }
+size_t mask_bytes(const trimul_params *p) { return (size_t)p->N * p->N * elem_size(p->dtype); }
+
+int check_z(const trimul_params *p, const void *z) {
+    if (!z) return TRIMUL_ERR_INVALID_ARG;
+    if (!aligned(z, 16)) return TRIMUL_ERR_MISALIGNED;
+    if (overlap(z, pair_bytes(p), p->workspace, p->workspace_bytes)) return TRIMUL_ERR_ALIAS;
+    return TRIMUL_OK;
+}
+
+int check_mask(const trimul_params *p, const void *mask) {
+    if (!mask) return TRIMUL_OK;
+    if (!aligned(mask, elem_size(p->dtype))) return TRIMUL_ERR_MISALIGNED;
+    if (overlap(mask, mask_bytes(p), p->workspace, p->workspace_bytes)) return TRIMUL_ERR_ALIAS;
+    return TRIMUL_OK;
+}
+
+int check_out(const trimul_params *p, const void *out, const void *z, const void *mask) {
+    if (!out) return TRIMUL_ERR_INVALID_ARG;
+    if (!aligned(out, 16)) return TRIMUL_ERR_MISALIGNED;
+    const size_t n = pair_bytes(p);
+    if (overlap(out, n, z, n) || overlap(out, n, mask, mask_bytes(p)) ||
+        overlap(out, n, p->workspace, p->workspace_bytes))
+        return TRIMUL_ERR_ALIAS;
+    return TRIMUL_OK;
+}
+
+int check_direction(int d) { return (d == TRIMUL_OUTGOING || d == TRIMUL_INCOMING) ? TRIMUL_OK : TRIMUL_ERR_INVALID_ARG; }
+
+int check_weights_on_device(const trimul_params *p) {
+    const void *all[] = {p->w_a, p->w_ag, p->w_b, p->w_bg, p->w_g, p->w_o, p->ln_in_w, p->ln_in_b,
+                         p->b_a, p->b_ag, p->b_b, p->b_bg, p->b_g, p->ln_out_w, p->ln_out_b, p->b_o,
+                         p->workspace};
+    for (const void *v : all) {
+        int rc = check_device_ptr(v, "weight/workspace pointer");
+        if (rc) return rc;
+    }
+    return TRIMUL_OK;
+}
+
+// ---- workspace views ----------------------------------------------------------
+
+struct Views {
+    DeviceStatus *status;
+    uint8_t *a, *b, *x;
+    size_t ld;
+};
+
+Views views_of(const trimul_params *p) {
+    Views v;
+    uint8_t *base = static_cast<uint8_t *>(p->workspace);
+    const size_t sec = section_bytes(p->N, p->dtype);
+    v.status = reinterpret_cast<DeviceStatus *>(base);
+    v.a = base + kHeader;
+    v.b = v.a + sec;
+    v.x = v.b + sec;
+    v.ld = ld_of(p->N);
+    return v;
+}
+
+KernelCtl ctl_of(const trimul_params *p, const Views &v) {
+    KernelCtl c;
+    c.status = v.status;
+    c.timeout_ns = (unsigned long long)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
+    c.debug_flags = p->debug_flags;
+    return c;
+}
+
+// ---- tensor maps ----------------------------------------------------------------
+
+int encode(CUtensorMap *m, int rank, const void *base, const uint64_t *dims, const uint64_t *strides,
+           const uint32_t *box, CUtensorMapSwizzle sw) {
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bd[5], es[5];
+    for (int r = 0; r < rank; ++r) {
+        gd[r] = dims[r];
+        bd[r] = box[r];
+        es[r] = 1;
+        if (r < rank - 1) gs[r] = strides[r];
+    }
+    CUresult res = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gd, gs,
+                            bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (res != CUDA_SUCCESS) {
+        snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled failed (%d), rank %d", (int)res, rank);
+        return TRIMUL_ERR_CUDA;
+    }
+    return TRIMUL_OK;
+}
+
+// 128 x 128 weight [out][in], loaded as two 64-column halves with 128-byte swizzle.
+int map_weight(CUtensorMap *m, const void *w) {
+    const uint64_t dims[2] = {128, 128}, strides[1] = {128 * 2};
+    const uint32_t box[2] = {64, 128};
+    return encode(m, 2, w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// z or out [N][N][128] as (c, j, i): 64 channels x 128 cells of one row.
+int map_pair(CUtensorMap *m, const void *t, int N) {
+    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)N};
+    const uint64_t strides[2] = {128 * 2, (uint64_t)N * 128 * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    return encode(m, 3, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// a, b or x [128][N][ld] as (col, row, c) with the given box and swizzle.
+int map_cm(CUtensorMap *m, const void *t, int N, size_t ld, uint32_t b0, uint32_t b1, uint32_t b2,
+           CUtensorMapSwizzle sw) {
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, 128};
+    const uint64_t strides[2] = {ld * 2, (uint64_t)N * ld * 2};
+    const uint32_t box[3] = {b0, b1, b2};
+    return encode(m, 3, t, dims, strides, box, sw);
+}
+
+F32Layer f32_layer(const trimul_params *p, const void *mask, const Views &v) {
+    F32Layer L;
+    L.N = p->N;
+    L.ld = v.ld;
+    L.eps = p->ln_eps;
+    L.mask = static_cast<const float *>(mask);
+    L.ln_in_w = static_cast<const float *>(p->ln_in_w);
+    L.ln_in_b = static_cast<const float *>(p->ln_in_b);
+    L.ln_out_w = static_cast<const float *>(p->ln_out_w);
+    L.ln_out_b = static_cast<const float *>(p->ln_out_b);
+    L.w_a = static_cast<const float *>(p->w_a);
+    L.w_ag = static_cast<const float *>(p->w_ag);
+    L.w_b = static_cast<const float *>(p->w_b);
+    L.w_bg = static_cast<const float *>(p->w_bg);
+    L.w_g = static_cast<const float *>(p->w_g);
+    L.w_o = static_cast<const float *>(p->w_o);
+    L.b_a = static_cast<const float *>(p->b_a);
+    L.b_ag = static_cast<const float *>(p->b_ag);
+    L.b_b = static_cast<const float *>(p->b_b);
+    L.b_bg = static_cast<const float *>(p->b_bg);
+    L.b_g = static_cast<const float *>(p->b_g);
+    L.b_o = static_cast<const float *>(p->b_o);
+    L.a = reinterpret_cast<float *>(v.a);
+    L.b = reinterpret_cast<float *>(v.b);
+    L.x = reinterpret_cast<float *>(v.x);
+    return L;
+}
+
+int cuda_rc(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return TRIMUL_OK;
+    set_detail(what, e);
+    return TRIMUL_ERR_CUDA;
+}
+
+// ---- stages ------------------------------------------------------------------------
+
+int run_prologue(const void *z, const void *mask, const trimul_params *p, const DevState &d, cudaStream_t s) {
+    const Views v = views_of(p);
+    if (p->dtype == TRIMUL_DTYPE_F32) {
+        const long tiles = (long)p->N * ((p->N + 31) / 32);
+        const int grid = (int)(tiles < (long)d.sms * 8 ? tiles : (long)d.sms * 8);
+        return cuda_rc(launch_prologue_f32(static_cast<const float *>(z), f32_layer(p, mask, v), grid, s),
+                       "prologue_f32 launch");
+    }
+    PrologueMaps m;
+    const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
+    for (int k = 0; k < 4; ++k)
+        if (int rc = map_weight(&m.w[k], w[k])) return rc;
+    if (int rc = map_pair(&m.z, z, p->N)) return rc;
+    if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 128, 1, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 128, 1, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    PrologueArgs a;
+    a.N = p->N;
+    a.jt_tiles = (p->N + 127) / 128;
+    a.total_tiles = p->N * a.jt_tiles;
+    a.eps = p->ln_eps;
+    a.mask = static_cast<const __nv_bfloat16 *>(mask);
+    a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
+    a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
+    a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
+    a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
+    a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
+    a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
+    a.ctl = ctl_of(p, v);
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_prologue_tc(m, a, grid, s), "prologue_tc launch");
+}
+
+int run_contract(const trimul_params *p, int direction, const DevState &d, cudaStream_t s) {
+    const Views v = views_of(p);
+    if (p->dtype == TRIMUL_DTYPE_F32)
+        return cuda_rc(launch_contract_f32(f32_layer(p, nullptr, v), direction, s), "contract_f32 launch");
+    ContractMaps m;
+    if (direction == TRIMUL_OUTGOING) {
+        if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 256, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    } else {
+        if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    }
+    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    ContractArgs a;
+    a.N = p->N;
+    a.incoming = direction == TRIMUL_INCOMING;
+    a.ti_tiles = (p->N + 127) / 128;
+    a.tj_tiles = (p->N + 255) / 256;
+    a.total_tiles = kC * a.ti_tiles * a.tj_tiles;
+    a.kblocks = (p->N + 63) / 64;
+    a.ctl = ctl_of(p, v);
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_contract_tc(m, a, grid, s), "contract_tc launch");
+}
+
+int run_epilogue(const void *z, const trimul_params *p, void *out, const DevState &d, cudaStream_t s) {
+    const Views v = views_of(p);
+    if (p->dtype == TRIMUL_DTYPE_F32) {
+        const long tiles = (long)p->N * ((p->N + 31) / 32);
+        const int grid = (int)(tiles < (long)d.sms * 8 ? tiles : (long)d.sms * 8);
+        return cuda_rc(launch_epilogue_f32(static_cast<const float *>(z), static_cast<float *>(out),
+                                           f32_layer(p, nullptr, v), grid, s),
+                       "epilogue_f32 launch");
+    }
+    EpilogueMaps m;
+    if (int rc = map_weight(&m.wg, p->w_g)) return rc;
+    if (int rc = map_weight(&m.wo, p->w_o)) return rc;
+    if (int rc = map_pair(&m.z, z, p->N)) return rc;
+    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 128, 1, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    if (int rc = map_pair(&m.out, out, p->N)) return rc;
+    EpilogueArgs a;
+    a.N = p->N;
+    a.jt_tiles = (p->N + 127) / 128;
+    a.total_tiles = p->N * a.jt_tiles;
+    a.eps = p->ln_eps;
+    a.ln_in_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
+    a.ln_in_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
+    a.ln_out_w = static_cast<const __nv_bfloat16 *>(p->ln_out_w);
+    a.ln_out_b = static_cast<const __nv_bfloat16 *>(p->ln_out_b);
+    a.b_g = static_cast<const __nv_bfloat16 *>(p->b_g);
+    a.b_o = static_cast<const __nv_bfloat16 *>(p->b_o);
+    a.ctl = ctl_of(p, v);
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_epilogue_tc(m, a, grid, s), "epilogue_tc launch");
+}
+
+int clear_status(const trimul_params *p, cudaStream_t s) {
+    return cuda_rc(cudaMemsetAsync(p->workspace, 0, sizeof(DeviceStatus), s), "status clear");
+}
+
+}  // namespace
+
+// ---- exported symbols -------------------------------------------------------------
+
+extern "C" {
+
+size_t trimul_workspace_size_dtype(int N, int c_z, int c_h, int dtype) {
+    if (N < 1 || N > kMaxN || c_z != kC || c_h != kC || !valid_dtype(dtype)) return 0;
+    return kHeader + 3 * section_bytes(N, dtype);
+}
+
+size_t trimul_workspace_size(int N, int c_z, int c_h) {
+    return trimul_workspace_size_dtype(N, c_z, c_h, TRIMUL_DTYPE_F32);
+}
+
+int trimul_prologue(const void *z, const void *mask, const trimul_params *p, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_z(p, z)) || (rc = check_mask(p, mask))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, p->dtype == TRIMUL_DTYPE_BF16))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
+        (rc = check_device_ptr(mask, "mask")))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(p, s))) return rc;
+    return run_prologue(z, mask, p, *d, s);
+}
+
+int trimul_contract(const trimul_params *p, int direction, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, p->dtype == TRIMUL_DTYPE_BF16))) return rc;
+    if ((rc = check_device_ptr(p->workspace, "workspace"))) return rc;
+    return run_contract(p, direction, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int trimul_epilogue(const void *z, const trimul_params *p, void *out, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_z(p, z)) || (rc = check_out(p, out, z, nullptr))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, p->dtype == TRIMUL_DTYPE_BF16))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) || (rc = check_device_ptr(out, "out")))
+        return rc;
+    return run_epilogue(z, p, out, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int trimul_forward(const void *z, const void *mask, const trimul_params *p, int direction, void *out,
+                   trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction)) || (rc = check_z(p, z)) ||
+        (rc = check_mask(p, mask)) || (rc = check_out(p, out, z, mask)))
+        return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, p->dtype == TRIMUL_DTYPE_BF16))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
+        (rc = check_device_ptr(mask, "mask")) || (rc = check_device_ptr(out, "out")))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(p, s))) return rc;
+    if ((rc = run_prologue(z, mask, p, *d, s))) return rc;
+    if ((rc = run_contract(p, direction, *d, s))) return rc;
+    return run_epilogue(z, p, out, *d, s);
+}
+
+int trimul_workspace_views(const trimul_params *p, void **a, void **b, void **x, size_t *ld) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    const Views v = views_of(p);
+    if (a) *a = v.a;
+    if (b) *b = v.b;
+    if (x) *x = v.x;
+    if (ld) *ld = v.ld;
+    return TRIMUL_OK;
+}
+
+int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *detail) {
+    if (!p || !p->workspace) return TRIMUL_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceStatus st;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(&st, p->workspace, sizeof st, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        set_detail("status read", e);
+        return TRIMUL_ERR_CUDA;
+    }
+    if (detail) {
+        detail[0] = st.code;
+        detail[1] = st.site;
+        detail[2] = st.block;
+        detail[3] = st.aux;
+    }
+    if (st.code == DEV_OK) return TRIMUL_OK;
+    return st.code == DEV_TIMEOUT ? TRIMUL_ERR_TIMEOUT : TRIMUL_ERR_DEVICE;
+}
+
+const char *trimul_error_string(int code) {
+    switch (code) {
+        case TRIMUL_OK: return "ok";
+        case TRIMUL_ERR_INVALID_ARG: return "invalid argument";
+        case TRIMUL_ERR_UNSUPPORTED: return "unsupported configuration";
+        case TRIMUL_ERR_MISALIGNED: return "pointer not aligned";
+        case TRIMUL_ERR_ALIAS: return "output overlaps an input or the workspace";
+        case TRIMUL_ERR_WORKSPACE: return "workspace missing or too small";
+        case TRIMUL_ERR_CUDA: return "CUDA runtime or driver error";
+        case TRIMUL_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
+        case TRIMUL_ERR_DEVICE: return "kernel-detected fault";
+        default: return "unknown status";
+    }
+}
+
+const char *trimul_last_error_detail(void) { return g_detail; }
+
+int trimul_version(void) { return 100; }
+
+}  // extern "C"
