@@ -90,6 +90,23 @@ def ncu_traffic(kernel: str, N: int):
     return None
 
 
+# ---------------------------------------------------------------- multi-rank host logic
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest value over all ranks (timing is the slowest replica's)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def pair_cells_per_s(world: int, steps: int, n_dirs: int, N: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank processes steps * n_dirs * N^2 pair-cells."""
+    return world * steps * n_dirs * N * N / (total_ms / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -260,10 +277,7 @@ def run_ours(args, rank, world, local_rank):
             for s, n in enumerate(names):
                 kern_ms[n] += evs[3 * k + s].elapsed_time(evs[3 * k + s + 1])
     launches = {n: args.steps * len(dirs) for n in names}
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # ---- end to end through the public layer API, host buffers in and out
     e2e = None
@@ -291,11 +305,8 @@ def run_ours(args, rank, world, local_rank):
             ev1.record(stream)
             torch.cuda.synchronize()
             e2e_ms += ev0.elapsed_time(ev1)
-        if dist:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * args.steps * len(dirs) * N * N / (e2e_ms / 1e3), "unit": UNIT,
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+        e2e = {"value": pair_cells_per_s(world, args.steps, len(dirs), N, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": z_host.numel() * z_host.element_size() + m_host.numel() * m_host.element_size(),
                "d2h_bytes_per_step": sum(out_host[d].numel() * out_host[d].element_size() for d in dirs)}
 
@@ -336,8 +347,7 @@ def run_ours(args, rank, world, local_rank):
                "sample": f"float64 oracle (grid mode) on {n_idx} x {n_idx} sampled cells of the N={N} "
                          f"workload, {'+'.join(dirs)}: {cells} pair-cells in {secs:.1f} s"}
 
-    cells_total = world * args.steps * len(dirs) * N * N
-    value = cells_total / (total_ms / 1e3)
+    value = pair_cells_per_s(world, args.steps, len(dirs), N, total_ms)
     tflops = world * args.steps * len(dirs) * N * N * flops_per_cell(N) / (total_ms / 1e3) / 1e12
     clocks = sampler.summary()
     line = {
