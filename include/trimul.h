@@ -131,6 +131,32 @@ const char *trimul_error_string(int code);
  * call and its message), or "" if none. Valid until the next call. */
 const char *trimul_last_error_detail(void);
 
+/* Bytes of the library's static scratch array used by trimul_forward_noalloc:
+ * room for the bf16 layer at N <= 128 and the fp32 layer at N <= 88. */
+#define TRIMUL_NOALLOC_SCRATCH_BYTES (256u + 3u * 4194304u)
+
+/* trimul_forward for callers that cannot allocate device memory. The pages
+ * have no counterpart of this entry point; it exists for callers such as a
+ * plugin whose host application owns all device memory and forbids other
+ * allocations, or a latency-critical loop that must not risk an allocation.
+ *
+ * Same arguments and results as trimul_forward, except that p->workspace and
+ * p->workspace_bytes are ignored: the scratch lives in a file-scope device
+ * array of TRIMUL_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library keeps until the process exits. Sizes that do not fit
+ * it (bf16 N > 128, fp32 N > 88) return TRIMUL_ERR_WORKSPACE before any work
+ * is enqueued. Nothing is allocated or freed.
+ *
+ * All calls share the one array and a call leaves its contents behind (the
+ * status word is cleared at the start of each call): calls whose GPU work
+ * overlaps, on different streams or from different host threads, race and
+ * give wrong results. The first call with a given device current looks up
+ * the array's device address for that device; make that first call before
+ * any stream capture. trimul_device_status cannot read this scratch's status
+ * word; an in-kernel timeout still leaves the output invalid. */
+int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params *p, int direction,
+                           void *out, trimul_stream_t stream);
+
 /* Library version (major * 100 + minor). */
 int trimul_version(void);
 

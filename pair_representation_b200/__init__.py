@@ -37,7 +37,7 @@ ERR = {v: k for k, v in STATUS.items()}
 # Every symbol include/trimul.h declares.
 EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forward", "trimul_prologue",
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
-           "trimul_error_string", "trimul_last_error_detail", "trimul_version")
+           "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc")
 
 
 class TrimulError(RuntimeError):
@@ -85,6 +85,7 @@ def lib():
         L.trimul_workspace_size_dtype.argtypes = [I, I, I, I]
         L.trimul_workspace_size_dtype.restype = S
         L.trimul_forward.argtypes = [P, P, PP, I, P, P]
+        L.trimul_forward_noalloc.argtypes = [P, P, PP, I, P, P]
         L.trimul_prologue.argtypes = [P, P, PP, P]
         L.trimul_contract.argtypes = [PP, I, P]
         L.trimul_epilogue.argtypes = [P, PP, P, P]
@@ -96,7 +97,7 @@ def lib():
         L.trimul_last_error_detail.argtypes = []
         L.trimul_last_error_detail.restype = ctypes.c_char_p
         L.trimul_version.argtypes = []
-        for f in ("trimul_forward", "trimul_prologue", "trimul_contract", "trimul_epilogue",
+        for f in ("trimul_forward", "trimul_forward_noalloc", "trimul_prologue", "trimul_contract", "trimul_epilogue",
                   "trimul_workspace_views", "trimul_device_status", "trimul_version"):
             getattr(L, f).restype = I
         _lib = L
@@ -140,6 +141,19 @@ def trimul_forward(z, mask, params: TrimulParams, direction: int, out, stream=No
     rc = lib().trimul_forward(_ptr(z), _ptr(mask), ctypes.byref(params), direction, _ptr(out), _stream(stream))
     if check:
         _check(rc, "trimul_forward")
+    return rc
+
+
+def trimul_forward_noalloc(z, mask, params: TrimulParams, direction: int, out, stream=None, check=True) -> int:
+    """trimul_forward with the library's static scratch instead of params.workspace.
+
+    For callers that cannot allocate device memory; limited to bf16 N <= 128
+    and fp32 N <= 88. Overlapping calls share the scratch and race.
+    """
+    rc = lib().trimul_forward_noalloc(_ptr(z), _ptr(mask), ctypes.byref(params), direction, _ptr(out),
+                                      _stream(stream))
+    if check:
+        _check(rc, "trimul_forward_noalloc")
     return rc
 
 

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtrimul_b200.so")
-SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu"]
+SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 
