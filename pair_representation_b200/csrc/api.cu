@@ -242,12 +242,12 @@ int map_weight(CUtensorMap *m, const void *w) {
     return encode(m, 2, w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// z or out [N][N][128] as (c, j, i): 64 channels x 128 cells of one row.
-int map_pair(CUtensorMap *m, const void *t, int N) {
+// z or out [N][N][128] as (c, j, i): box of b0 channels x b1 cells of one row.
+int map_pair(CUtensorMap *m, const void *t, int N, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
     const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)N};
     const uint64_t strides[2] = {128 * 2, (uint64_t)N * 128 * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    return encode(m, 3, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    const uint32_t box[3] = {b0, b1, 1};
+    return encode(m, 3, t, dims, strides, box, sw);
 }
 
 // a, b or x [128][N][ld] as (col, row, c) with the given box and swizzle.
@@ -307,9 +307,10 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
     const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
     for (int k = 0; k < 4; ++k)
         if (int rc = map_weight(&m.w[k], w[k])) return rc;
-    if (int rc = map_pair(&m.z, z, p->N)) return rc;
-    if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 128, 1, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
-    if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 128, 1, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    // Each worker warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
+    if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
+    if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     PrologueArgs a;
     a.N = p->N;
     a.jt_tiles = (p->N + 127) / 128;
@@ -331,10 +332,12 @@ int run_contract(const trimul_params *p, int direction, const DevState &d, cudaS
     const Views v = views_of(p);
     if (p->dtype == TRIMUL_DTYPE_F32)
         return cuda_rc(launch_contract_f32(f32_layer(p, nullptr, v), direction, s), "contract_f32 launch");
+    // CTA pairs share each 256 x 256 output tile: CTA r loads rows [128 r, 128 r + 128)
+    // of the A and B panels (boxes of 128 rows, or 2 x 64-wide blocks when MN-major).
     ContractMaps m;
     if (direction == TRIMUL_OUTGOING) {
         if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 256, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     } else {
         if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
         if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
@@ -343,13 +346,13 @@ int run_contract(const trimul_params *p, int direction, const DevState &d, cudaS
     ContractArgs a;
     a.N = p->N;
     a.incoming = direction == TRIMUL_INCOMING;
-    a.ti_tiles = (p->N + 127) / 128;
+    a.ti_tiles = (p->N + 255) / 256;
     a.tj_tiles = (p->N + 255) / 256;
     a.total_tiles = kC * a.ti_tiles * a.tj_tiles;
     a.kblocks = (p->N + 63) / 64;
     a.ctl = ctl_of(p, v);
-    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
-    return cuda_rc(launch_contract_tc(m, a, grid, s), "contract_tc launch");
+    const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
+    return cuda_rc(launch_contract_tc(m, a, 2 * pairs, s), "contract_tc launch");
 }
 
 int run_epilogue(const void *z, const trimul_params *p, void *out, const DevState &d, cudaStream_t s) {
@@ -364,9 +367,10 @@ int run_epilogue(const void *z, const trimul_params *p, void *out, const DevStat
     EpilogueMaps m;
     if (int rc = map_weight(&m.wg, p->w_g)) return rc;
     if (int rc = map_weight(&m.wo, p->w_o)) return rc;
-    if (int rc = map_pair(&m.z, z, p->N)) return rc;
+    if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 128, 1, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
-    if (int rc = map_pair(&m.out, out, p->N)) return rc;
+    // Each worker warp stores 32 channels x 32 cells (64-byte rows, 64-byte swizzle).
+    if (int rc = map_pair(&m.out, out, p->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     EpilogueArgs a;
     a.N = p->N;
     a.jt_tiles = (p->N + 127) / 128;

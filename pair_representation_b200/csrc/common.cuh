@@ -223,6 +223,51 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 16 lanes x 256 bits, 4 repetitions along columns (32 columns): thread t gets, for
+// repetition k, r[4k], r[4k+1] = lane (base + t/4), columns 8k + 2(t%4) + {0,1} and
+// r[4k+2], r[4k+3] = lane (base + 8 + t/4), the same columns.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Four 8x8 bf16 matrices from registers to shared memory, transposed: thread t
+// holds in q[i] the pair (row t/4, columns 2(t%4), 2(t%4)+1) of matrix i; thread
+// 8i + j supplies the address of stored row j of matrix i, which receives
+// column j of matrix i (16 bytes).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(q0), "r"(q1),
+                 "r"(q2), "r"(q3)
+                 : "memory");
+}
+
+// Named barrier `id` over `n` threads that also returns the AND of `pred`
+// across them, so all participants take the same branch afterwards.
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+// Bounded wait by lane 0 of a warp, result broadcast to the warp.
+static __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                 const KernelCtl &ctl, int site, int aux) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, abort_flag, ctl, site, aux) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle.
 //   K-major operand  (rows of 64 bf16 = 128 B along K): lbo unused (16), sbo =
 //     byte distance between groups of 8 rows (1024 for densely packed rows).

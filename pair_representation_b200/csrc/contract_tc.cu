@@ -1,37 +1,43 @@
-// contract_tc.cu - the triangle contraction on tcgen05 tensor cores.
+// contract_tc.cu - the triangle contraction on tcgen05 tensor cores, CTA pairs.
 //
-// For every channel c of the hidden pair features, outgoing computes
-// X_c = A_c B_c^T (x_ij = sum_k a_ik b_jk) and incoming X_c = A_c^T B_c
-// (x_ij = sum_k a_ki b_kj): 128 independent N x N x N products, the step the
-// layer's name refers to (TriangleMultiplicationOutgoing, "Scaling
+// For every channel c of the hidden pair features (outgoing X_c = A_c B_c^T,
+// incoming X_c = A_c^T B_c; TriangleMultiplicationOutgoing, "Scaling
 // biomolecular modeling with context parallelism in NVIDIA BioNeMo", section
-// "Context-parallel implementation of triangle multiplication").
+// "Context-parallel implementation of triangle multiplication"), computed by
+// pairs of CTAs on neighbouring SMs (a cluster of 2) that share one
+// 256 x 256 output tile through tcgen05.mma.cta_group::2:
+//   * CTA r of the pair loads rows [128 r, 128 r + 128) of the tile's A panel
+//     and rows [128 r, 128 r + 128) of its B panel (its half of N) into its own
+//     shared memory, 16 KB + 16 KB per 64-deep K block, 6 stages;
+//   * one thread of CTA 0 issues M = 256, N = 256 MMAs that read both CTAs'
+//     operands; CTA r's tensor memory receives rows [128 r, 128 r + 128) of
+//     the fp32 accumulator (double-buffered, 2 x 256 columns);
+//   * each CTA's epilogue warps drain their own half and TMA-store it.
+// Per SM this moves 32 KB of operands per K block for the same MMA work that
+// a single CTA with a 128 x 256 tile needs 48 KB for.
 //
-// a, b and x are channel-major [128][N][ld] bf16 arrays in the workspace.
-// Both directions read the same arrays: outgoing feeds the tensor core
-// K-major tiles (k contiguous), incoming feeds the transposed operands as
-// MN-major tiles (i or j contiguous) selected by the instruction descriptor,
-// so nothing is transposed in memory.
-//
-// Kernel shape: persistent, one CTA per SM, 128 x 256 output tiles, 64-deep
-// K blocks in a 4-stage TMA ring, fp32 accumulators double-buffered in tensor
-// memory (2 x 256 columns), and warp roles:
-//   warp 0      TMA producer (one thread)
-//   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2..5  epilogue: TMEM -> registers -> bf16 -> swizzled smem -> TMA store
-// Tiles are ordered channel-major so CTAs resident together share one
-// channel's panels in L2. Out-of-range rows / k are zero-filled by TMA on load
-// and clipped on store, so ragged N needs no masking.
+// Synchronisation (every wait bounded):
+//   full[s]    CTA 0: armed by CTA 0's producer for the pair's 64 KB; CTA 0's
+//              loads and CTA 1's loads (cta_group::2 TMA addressed to CTA 0's
+//              barrier) both complete bytes on it; the MMA issuer waits on it
+//   empty[s]   both CTAs, arrived by the MMA commit multicast to the pair
+//   tfull[a]   both CTAs, MMA commit multicast -> epilogue warps
+//   tempty[a]  CTA 0, arrivals of the 4 + 4 epilogue warps of both CTAs
+// On the way out CTA 1 publishes how many phases of each stage it loaded and
+// CTA 0 reconciles full[s] (arming phases only CTA 1 loaded, completing the
+// bytes of phases only CTA 0 loaded), then waits for every stage to land, so
+// no copy is in flight when the pair passes its final cluster barrier.
 #include "kernels.h"
 
 namespace trimul {
 namespace con {
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;            // 16 KB
-constexpr int B_BYTES = BN * BK * 2;            // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int BN = 256, BK = 64, STAGES = 6;
+constexpr int HALF = 128;                         // rows per CTA of A and of B
+constexpr int A_BYTES = HALF * BK * 2;            // 16 KB
+constexpr int B_BYTES = HALF * BK * 2;            // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
 constexpr int OUT_COLS = 64;
-constexpr int OUT_BYTES = BM * OUT_COLS * 2;    // 16 KB
+constexpr int OUT_BYTES = HALF * OUT_COLS * 2;    // 16 KB
 constexpr int NUM_OUT = 2;
 constexpr int TMEM_COLS = 512;
 constexpr int THREADS = 192;
@@ -40,37 +46,101 @@ constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_OUT * OUT_BYTE
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace con
 
-__global__ void __launch_bounds__(con::THREADS, 1)
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_remote_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose bytes complete on a barrier of
+// the leader CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on `bar` (same offset) in both CTAs of the pair once this thread's MMAs have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_local2(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
     contract_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmX, const ContractArgs args) {
+                        const __grid_constant__ CUtensorMap tmX, const ContractArgs args) {
     using namespace con;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;
     uint8_t *outbuf = smem + STAGES * STAGE_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + NUM_OUT * OUT_BYTES);
-    uint64_t *full = bars;                 // [STAGES] TMA -> MMA
-    uint64_t *empty = bars + STAGES;       // [STAGES] MMA -> TMA
-    uint64_t *tfull = bars + 2 * STAGES;   // [2] MMA -> epilogue
-    uint64_t *tempty = tfull + 2;          // [2] epilogue -> MMA
+    uint64_t *full = bars;                 // [STAGES] (CTA 0) operands of both CTAs landed
+    uint64_t *empty = bars + STAGES;       // [STAGES] MMA done reading the stage (both CTAs)
+    uint64_t *tfull = bars + 2 * STAGES;   // [2]
+    uint64_t *tempty = tfull + 2;          // [2] (CTA 0)
     uint64_t *dead = tempty + 2;           // never signalled (failure-path test)
-    uint64_t *drain = dead + 1;            // MMA completion before teardown
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *drain = dead + 1;
+    uint64_t *peer_done = drain + 1;       // (CTA 0) CTA 1's producer has published its phase counts
+    uint32_t *peer_phases = reinterpret_cast<uint32_t *>(peer_done + 1);  // [STAGES] (CTA 0) written by CTA 1
+    uint32_t *tmem_slot = peer_phases + STAGES;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_go = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
     const KernelCtl &ctl = args.ctl;
     const int tiles_per_c = args.ti_tiles * args.tj_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1);  // CTA 0's producer arms it (arrive + expect_tx)
             mbar_init(&empty[s], 1);
+            peer_phases[s] = 0;
         }
+        mbar_init(peer_done, 1);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+            mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA
         }
         mbar_init(dead, 1);
         mbar_init(drain, 1);
@@ -82,25 +152,40 @@ __global__ void __launch_bounds__(con::THREADS, 1)
         tma_prefetch_desc(&tmX);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const uint32_t peer_abort = map_to_rank((const void *)abort_flag, rank ^ 1u);
+    // Raise the abort in this CTA and in its peer.
+    auto raise_abort = [&]() {
+        *abort_flag = 1;
+        st_remote_u32(peer_abort, 1u);
+    };
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer ----------------
+            // ---------------- TMA producer (both CTAs) ----------------
+            const uint32_t full0 = map_to_rank(full, 0);  // CTA 0's full[0] in the cluster window
             int stage = 0;
-            uint32_t phase = 0, ever = 0, par = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0;  // K blocks this CTA has loaded; stages are used round-robin
+            auto phases_of = [&](int s) -> uint32_t {
+                return issued / STAGES + ((uint32_t)s < issued % STAGES ? 1u : 0u);
+            };
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x) {
+            for (int tile = pair; ok && tile < args.total_tiles; tile += npairs) {
                 const int c = tile / tiles_per_c;
                 const int r = tile - c * tiles_per_c;
                 const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
-                const int i0 = ti * BM, j0 = tj * BN;
+                const int i0 = ti * 256 + (int)rank * HALF, j0 = tj * BN + (int)rank * HALF;
                 for (int kb = 0; kb < args.kblocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, ctl, SITE_CON | 1, tile)) {
                         ok = false;
@@ -108,40 +193,57 @@ __global__ void __launch_bounds__(con::THREADS, 1)
                     }
                     uint8_t *sa = stages + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    const uint32_t bar = full0 + (uint32_t)(stage * 8);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const int k0 = kb * BK;
                     if (!args.incoming) {
-                        tma_load_3d(sa, &tmA, &full[stage], k0, i0, c);
-                        tma_load_3d(sb, &tmB, &full[stage], k0, j0, c);
+                        tma_load_3d_pair(sa, &tmA, bar, k0, i0, c);
+                        tma_load_3d_pair(sb, &tmB, bar, k0, j0, c);
                     } else {
-                        // MN-major: 64-wide row blocks, each BK k-rows of 128 B.
-                        tma_load_3d(sa, &tmA, &full[stage], i0, k0, c);
-                        tma_load_3d(sa + BK * 128, &tmA, &full[stage], i0 + 64, k0, c);
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) tma_load_3d(sb + h * BK * 128, &tmB, &full[stage], j0 + 64 * h, k0, c);
+                        tma_load_3d_pair(sa, &tmA, bar, i0, k0, c);
+                        tma_load_3d_pair(sa + BK * 128, &tmA, bar, i0 + 64, k0, c);
+                        tma_load_3d_pair(sb, &tmB, bar, j0, k0, c);
+                        tma_load_3d_pair(sb + BK * 128, &tmB, bar, j0 + 64, k0, c);
                     }
-                    ever |= 1u << stage;
-                    par = (par & ~(1u << stage)) | (phase << stage);
+                    ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            // Let every load already issued land before shared memory is released.
-            for (int s = 0; s < STAGES; ++s)
-                if ((ever >> s) & 1u) wait_drain(&full[s], (par >> s) & 1u, ctl.timeout_ns);
+            if (!ok) raise_abort();
+            if (rank == 1) {
+                // Publish the phase counts to CTA 0, then signal it.
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s) st_remote_u32(map_to_rank(&peer_phases[s], 0), phases_of(s));
+                fence_acq_rel_cluster();
+                mbar_arrive_remote(map_to_rank(peer_done, 0));
+            } else {
+                // Reconcile every stage with CTA 1's loads, then let all of them land.
+                const bool peer_ok = wait_drain(peer_done, 0, ctl.timeout_ns);
+                fence_acq_rel_cluster();  // CTA 1's counts, released before its arrival, are visible
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s) {
+                    const uint32_t n0 = phases_of(s);
+                    const uint32_t n1 = peer_ok ? peer_phases[s] : n0;
+                    if (n1 > n0) mbar_arrive_expect_tx(&full[s], STAGE_BYTES);  // a phase only CTA 1 loaded
+                    if (n0 > n1) mbar_complete_tx(&full[s], STAGE_BYTES);       // a phase only CTA 0 loaded
+                    const uint32_t n = n0 > n1 ? n0 : n1;
+                    if (n > 0) wait_drain(&full[s], (n - 1) & 1u, ctl.timeout_ns);
+                }
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            const uint32_t idesc = idesc_bf16(BM, BN, args.incoming, args.incoming);
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (CTA 0) ----------------
+            const uint32_t idesc = idesc_bf16(256, BN, args.incoming, args.incoming);
             const bool stall = (ctl.debug_flags & 0x1u) != 0;
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             int lt = 0;
-            for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x, ++lt) {
+            for (int tile = pair; ok && tile < args.total_tiles; tile += npairs, ++lt) {
                 const int acc = lt & 1;
                 const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
                 if (!wait_bounded(&tempty[acc], acc_par ^ 1u, abort_flag, ctl, SITE_CON | 2, tile)) {
@@ -172,40 +274,51 @@ __global__ void __launch_bounds__(con::THREADS, 1)
                             ad = sdesc_sw128(sa + kk * 2048, BK * 128, 1024);
                             bd = sdesc_sw128(sb + kk * 2048, BK * 128, 1024);
                         }
-                        mma_bf16(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    mma_commit(&empty[stage]);  // frees the smem stage once these MMAs have read it
+                    mma_commit_pair(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&tfull[acc]);
+                mma_commit_pair(&tfull[acc]);
             }
-            // No MMA may still be writing tensor memory at teardown.
-            mma_commit(drain);
+            if (!ok) raise_abort();
+            mma_commit_local2(drain);
             wait_drain(drain, 0, ctl.timeout_ns);
         }
     } else {
-        // ---------------- epilogue warps 2..5 ----------------
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+        const int q = warp & 3;
         const int row = q * 32 + lane;
         const bool leader = (threadIdx.x == 64);
+        const uint32_t tempty0 = map_to_rank(&tempty[0], 0);
+        const uint32_t tempty1 = map_to_rank(&tempty[1], 0);
         int lt = 0;
-        for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++lt) {
+        for (int tile = pair; tile < args.total_tiles; tile += npairs, ++lt) {
             const int c = tile / tiles_per_c;
             const int r = tile - c * tiles_per_c;
             const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
-            const int i0 = ti * BM, j0 = tj * BN;
+            const int i0 = ti * 256 + (int)rank * HALF, j0 = tj * BN;
             const int acc = lt & 1;
             const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
-            if (leader) *epi_go = wait_bounded(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile) ? 1 : 0;
+            if (leader) {
+                const bool got = wait_bounded(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile);
+                if (!got) raise_abort();
+                *epi_go = got ? 1 : 0;
+            }
             named_bar_sync(1, 128);
             if (!*epi_go) break;
             tc_fence_after();
-            // Chunks whose first column is past N are neither read nor stored.
-            const int nch = min(BN / OUT_COLS, (args.N - j0 + OUT_COLS - 1) / OUT_COLS);
+            // Chunks whose first column is past N, and whole halves whose first row is past N,
+            // are neither read nor stored.
+            const int nch = (i0 < args.N) ? min(BN / OUT_COLS, (args.N - j0 + OUT_COLS - 1) / OUT_COLS) : 0;
+            if (nch == 0) {
+                tc_fence_before();
+                if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
+            }
 #pragma unroll 1
             for (int ch = 0; ch < nch; ++ch) {
                 uint32_t v[64];
@@ -215,13 +328,13 @@ __global__ void __launch_bounds__(con::THREADS, 1)
                 tmem_ld_wait();
                 if (ch == nch - 1) {
                     tc_fence_before();
-                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                    if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
                 }
                 uint32_t p[32];
 #pragma unroll
                 for (int k = 0; k < 32; ++k) p[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
                 uint8_t *ob = outbuf + (ch & 1) * OUT_BYTES;
-                if (leader) tma_store_wait_read<1>();  // the store that last used `ob` has read it
+                if (leader) tma_store_wait_read<1>();
                 named_bar_sync(1, 128);
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
@@ -241,8 +354,11 @@ __global__ void __launch_bounds__(con::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still touch its shared or tensor memory
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
 }
 
 size_t contract_tc_smem() { return con::SMEM; }

@@ -27,13 +27,13 @@ struct PrologueArgs {
 struct PrologueMaps {
     CUtensorMap w[4];  // W_a, W_ag, W_b, W_bg: 2-D [128 out][128 in], box 64 x 128, swizzle 128B
     CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 128, 1), swizzle 128B
-    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (128, 1, 64), no swizzle
+    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (32, 1, 32), swizzle 64B
 };
 
 struct ContractArgs {
     int N;
     int incoming;
-    int ti_tiles;     // ceil(N / 128)
+    int ti_tiles;     // ceil(N / 256)
     int tj_tiles;     // ceil(N / 256)
     int total_tiles;  // 128 * ti_tiles * tj_tiles
     int kblocks;      // ceil(N / 64)
@@ -41,7 +41,7 @@ struct ContractArgs {
 };
 
 struct ContractMaps {
-    CUtensorMap a, b;  // outgoing: box (64 k, 128|256 rows, 1); incoming: box (64 rows, 64 k, 1); swizzle 128B
+    CUtensorMap a, b;  // outgoing: box (64 k, 128 rows, 1); incoming: box (64 rows, 64 k, 1); swizzle 128B
     CUtensorMap x;     // 3-D (j, i, c) over x, box (64, 128, 1), swizzle 128B
 };
 
@@ -60,16 +60,17 @@ struct EpilogueMaps {
     CUtensorMap wg, wo;  // 2-D [128][128], box 64 x 128, swizzle 128B
     CUtensorMap z;       // as in the prologue
     CUtensorMap x;       // 3-D (j, i, c) over x, box (128, 1, 128), no swizzle
-    CUtensorMap out;     // 3-D (c, j, i) over out, box (64, 128, 1), swizzle 128B
+    CUtensorMap out;     // 3-D (c, j, i) over out, box (32, 32, 1), swizzle 64B
 };
 
 size_t prologue_tc_smem();
-size_t contract_tc_smem();
 size_t epilogue_tc_smem();
 cudaError_t prologue_tc_setup();
-cudaError_t contract_tc_setup();
 cudaError_t epilogue_tc_setup();
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s);
+size_t contract_tc_smem();
+cudaError_t contract_tc_setup();
+// Clusters of 2 CTAs, one 256 x 256 output tile per pair; grid = 2 x pairs.
 cudaError_t launch_contract_tc(const ContractMaps &m, const ContractArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_epilogue_tc(const EpilogueMaps &m, const EpilogueArgs &a, int grid, cudaStream_t s);
 

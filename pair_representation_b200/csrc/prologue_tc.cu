@@ -11,81 +11,46 @@
 // [128][N][ld] bf16 layout the contraction's TMA reads.
 //
 // Tiles are 128 consecutive cells of one residue row (z[i][j0 .. j0+127][:],
-// one contiguous 32 KB block). Per tile:
-//   TMA  z tile -> smem (128-byte swizzle, two 64-channel halves)
-//   LN   in place, fp32 statistics, bf16 result (the MMA's A operand)
-//   MMA  D[128 cells][512] = zh * [W_a; W_ag; W_b; W_bg]^T as two N = 256
-//        halves (a-half, b-half) into all 512 TMEM columns
-//   gate TMEM -> registers -> sigmoid, mask -> [64 ch][128 cells] smem
-//   TMA  store of each 64-channel slab to a or b (4 slabs per tile)
-// The four weight matrices (128 KB bf16) stay resident in shared memory for
-// the whole persistent CTA. The loop is software-pipelined so that the MMA of
-// the next tile runs while this tile is gated and stored, and the z load of
-// tile t+2 is in flight for a whole iteration.
+// one contiguous 32 KB block). The four weight matrices (128 KB bf16) stay in
+// shared memory for the whole persistent CTA. Roles (288 threads):
+//   warp 8 (control): TMA loads of z, the two projection MMAs per tile
+//     (a-half D[:, 0:256] = zh [W_a; W_ag]^T, b-half D[:, 256:512] = zh [W_b; W_bg]^T,
+//     M = 128 cells, N = 256, K = 128, all 512 TMEM columns), gated by
+//     mbarriers the workers arrive on.
+//   warps 0-7 (workers), each on its own, with no CTA-wide barrier:
+//     * LayerNorm of 16 cells of the next tile in place (fp32 statistics);
+//     * gating of 32 cells x 32 channels of a and of b: TMEM is read in the
+//       16-lane fragment layout, the gate m * sigmoid(g) * v is formed in
+//       packed fp32x2, the bf16 results are written channel-major with
+//       stmatrix.trans into a 64-byte-swizzled 2 KB buffer of the warp and
+//       stored by that warp's own TMA store.
+// Per tile the workers arrive on ln_done (next tile normalised), a_free (a-half
+// TMEM columns read) and b_free; the control warp issues the next tile's MMAs
+// into columns as soon as they are free, so tensor work, gating and the z loads
+// of two tiles ahead overlap.
 #include "kernels.h"
+#include "tile_ops.cuh"
 
 namespace trimul {
 namespace pro {
 constexpr int TILE = 128;
-constexpr int THREADS = 256;
-constexpr int W_HALF = 512 * 128;     // one 64-channel K half of the 4 stacked weights: 64 KB
-constexpr int W_BYTES = 2 * W_HALF;   // 128 KB
-constexpr int Z_HALF = TILE * 128;    // 16 KB
-constexpr int Z_BYTES = 2 * Z_HALF;   // 32 KB
-constexpr int ST_BYTES = 64 * TILE * 2;  // 16 KB staging slab [64 ch][128 cells]
-constexpr int NUM_ST = 2;
+constexpr int WORKERS = 8;
+constexpr int THREADS = 32 * (WORKERS + 1);
+constexpr int W_HALF = 512 * 128;       // one 64-channel K half of the 4 stacked weights: 64 KB
+constexpr int W_BYTES = 2 * W_HALF;     // 128 KB
+constexpr int Z_HALF = TILE * 128;      // 16 KB
+constexpr int Z_BYTES = 2 * Z_HALF;     // 32 KB
+constexpr int ST_BYTES = 32 * 32 * 2;   // 2 KB per warp buffer: [32 ch][32 cells], 64-byte swizzle
+constexpr int ST_PER_WARP = 2;
 constexpr int BAR_BYTES = 128;
-constexpr size_t SMEM = 1024 + (size_t)W_BYTES + 2 * Z_BYTES + NUM_ST * ST_BYTES + BAR_BYTES;
+constexpr size_t SMEM =
+    1024 + (size_t)W_BYTES + 2 * Z_BYTES + (size_t)WORKERS * ST_PER_WARP * ST_BYTES + BAR_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pro
 
-// In-place LayerNorm of one swizzled z tile: 2 threads per cell (one per
-// 64-channel half), statistics in fp32, partner exchange by shuffle.
-__device__ __forceinline__ void layer_norm_tile_sw128(uint8_t *zt, const __nv_bfloat16 *gw, const __nv_bfloat16 *gb,
-                                                      float eps) {
-    const int t = threadIdx.x;
-    const int r = t >> 1, h = t & 1;
-    uint8_t *rowp = zt + h * pro::Z_HALF + r * 128;
-    float v[64];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const int kc = (q + 4 * h) & 7;  // staggered so the two halves hit different banks
-        uint4 u = *reinterpret_cast<const uint4 *>(rowp + ((kc ^ (r & 7)) << 4));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            v[kc * 8 + 2 * e] = __uint_as_float(w[e] << 16);
-            v[kc * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 64; ++k) s += v[k];
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    const float mean = s * (1.f / 128.f);
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < 64; ++k) {
-        const float d = v[k] - mean;
-        ss = fmaf(d, d, ss);
-    }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    const float rstd = rsqrtf(ss * (1.f / 128.f) + eps);
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int c0 = h * 64 + kc * 8 + 2 * e;
-            const float g0 = gw ? __bfloat162float(gw[c0]) : 1.f, g1 = gw ? __bfloat162float(gw[c0 + 1]) : 1.f;
-            const float b0 = gb ? __bfloat162float(gb[c0]) : 0.f, b1 = gb ? __bfloat162float(gb[c0 + 1]) : 0.f;
-            w[e] = pack_bf16x2(fmaf((v[kc * 8 + 2 * e] - mean) * rstd, g0, b0),
-                               fmaf((v[kc * 8 + 2 * e + 1] - mean) * rstd, g1, b1));
-        }
-        *reinterpret_cast<uint4 *>(rowp + ((kc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
+// kVec: some LayerNorm affine or projection bias is present (general path);
+// without them the kernel skips every per-channel vector access.
+template <bool kVec>
 __global__ void __launch_bounds__(pro::THREADS, 1)
     prologue_tc_kernel(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWag,
                        const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmWbg,
@@ -95,15 +60,18 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *wsm = smem;
-    uint8_t *zsm = smem + W_BYTES;               // [2] z tiles
-    uint8_t *stsm = zsm + 2 * Z_BYTES;           // [2] staging slabs
-    uint64_t *bars = reinterpret_cast<uint64_t *>(stsm + NUM_ST * ST_BYTES);
-    uint64_t *wbar = bars;       // weights landed
-    uint64_t *zfull = bars + 1;  // [2] z tile landed
-    uint64_t *mma_a = bars + 3;  // a-half projections done
-    uint64_t *mma_b = bars + 4;  // b-half projections done
-    uint64_t *drain = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint8_t *zsm = smem + W_BYTES;                 // [2] z tiles
+    uint8_t *stsm = zsm + 2 * Z_BYTES;             // [8 warps][2] staging buffers
+    uint64_t *bars = reinterpret_cast<uint64_t *>(stsm + WORKERS * ST_PER_WARP * ST_BYTES);
+    uint64_t *wbar = bars;        // weights landed
+    uint64_t *zfull = bars + 1;   // [2] z tile landed
+    uint64_t *mma_a = bars + 3;   // a-half projections done
+    uint64_t *mma_b = bars + 4;   // b-half projections done
+    uint64_t *ln_done = bars + 5; // workers: next tile normalised (8 arrivals)
+    uint64_t *a_free = bars + 6;  // workers: a-half TMEM columns read (8 arrivals)
+    uint64_t *b_free = bars + 7;  // workers: b-half TMEM columns read (8 arrivals)
+    uint64_t *drain = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,12 +86,14 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         mbar_init(&zfull[1], 1);
         mbar_init(mma_a, 1);
         mbar_init(mma_b, 1);
+        mbar_init(ln_done, WORKERS);
+        mbar_init(a_free, WORKERS);
+        mbar_init(b_free, WORKERS);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {
-        __syncwarp();  // thread 0 ran the set-up above alone; the allocation is warp-wide
+    if (warp == WORKERS) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -137,166 +107,220 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         i = tile / args.jt_tiles;
         j0 = (tile - i * args.jt_tiles) * TILE;
     };
-    int last_load[2] = {-1, -1};  // thread 0: last tile loaded into each z buffer
-    auto load_z = [&](int lt) {
-        int i, j0;
-        tile_coords(lt, i, j0);
-        last_load[lt & 1] = lt;
-        uint8_t *dst = zsm + (lt & 1) * Z_BYTES;
-        mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES);
-        tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
-        tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
-    };
-    // One projection half: D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T (K = 128).
-    auto issue_half = [&](int half, int buf) {
-        const uint32_t idesc = idesc_bf16(128, 256, 0, 0);
-        const uint32_t za = smem_u32(zsm + buf * Z_BYTES);
-        const uint32_t wb = smem_u32(wsm) + (uint32_t)(half * 256 * 128);
-        const uint32_t d = tmem_base + (uint32_t)(half * 256);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (uint32_t)((kk >> 2) * Z_HALF + (kk & 3) * 32);
-            const uint32_t woff = (uint32_t)((kk >> 2) * W_HALF + (kk & 3) * 32);
-            mma_bf16(d, sdesc_sw128(za + koff, 16, 1024), sdesc_sw128(wb + woff, 16, 1024), idesc, kk ? 1u : 0u);
-        }
-    };
 
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(wbar, W_BYTES);
-        const CUtensorMap *wm[4] = {&tmWa, &tmWag, &tmWb, &tmWbg};
+    if (warp == WORKERS) {
+        // ------------------------------ control warp ------------------------------
+        if (lane == 0) {
+            int last_load0 = -1, last_load1 = -1;
+            auto load_z = [&](int lt) {
+                int i, j0;
+                tile_coords(lt, i, j0);
+                if (lt & 1) last_load1 = lt; else last_load0 = lt;
+                uint8_t *dst = zsm + (lt & 1) * Z_BYTES;
+                mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES);
+                tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
+                tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
+            };
+            // D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T over K = 128.
+            auto issue_half = [&](int half, int buf) {
+                const uint32_t idesc = idesc_bf16(128, 256, 0, 0);
+                const uint32_t za = smem_u32(zsm + buf * Z_BYTES);
+                const uint32_t wb = smem_u32(wsm) + (uint32_t)(half * 256 * 128);
+                const uint32_t d = tmem_base + (uint32_t)(half * 256);
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (uint32_t)((kk >> 2) * Z_HALF + (kk & 3) * 32);
+                    const uint32_t woff = (uint32_t)((kk >> 2) * W_HALF + (kk & 3) * 32);
+                    mma_bf16(d, sdesc_sw128(za + koff, 16, 1024), sdesc_sw128(wb + woff, 16, 1024), idesc,
+                             kk ? 1u : 0u);
+                }
+            };
+            mbar_arrive_expect_tx(wbar, W_BYTES);
+            const CUtensorMap *wm[4] = {&tmWa, &tmWag, &tmWb, &tmWbg};
 #pragma unroll
-            for (int kh = 0; kh < 2; ++kh) tma_load_2d(wsm + kh * W_HALF + w * 128 * 128, wm[w], wbar, kh * 64, 0);
-        if (n_local > 0) load_z(0);
-        if (n_local > 1) load_z(1);
-    }
-
-    int st_round = 0;  // staging slabs used so far (alternating buffers)
-    // Gate, mask and store one 64-channel slab of a (which = 0) or b (which = 1).
-    auto slab = [&](int which, int hh, float m, int i, int j0) {
-        const int q = warp & 3, sub = warp >> 2;
-        const int r = q * 32 + lane;
-        const int ch0 = hh * 64 + sub * 32;
-        uint32_t V[32], G[32];
-        __syncwarp();  // tcgen05.ld is warp-wide; thread 0 may have just issued a store alone
-        const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-        tmem_ld32(lane_base + (uint32_t)(which * 256 + ch0), V);
-        tmem_ld32(lane_base + (uint32_t)(which * 256 + 128 + ch0), G);
-        tmem_ld_wait();
-        uint8_t *st = stsm + (st_round & 1) * ST_BYTES;
-        ++st_round;
-        if (threadIdx.x == 0) tma_store_wait_read<1>();
-        __syncthreads();
-        const __nv_bfloat16 *bv = which ? args.b_b : args.b_a;
-        const __nv_bfloat16 *bg = which ? args.b_bg : args.b_ag;
-        __nv_bfloat16 *stv = reinterpret_cast<__nv_bfloat16 *>(st);
+            for (int w = 0; w < 4; ++w)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const int c = ch0 + k;
-            const float pv = __uint_as_float(V[k]) + ld_vec_bf16(bv, c, 0.f);
-            const float pg = __uint_as_float(G[k]) + ld_vec_bf16(bg, c, 0.f);
-            stv[(sub * 32 + k) * TILE + r] = __float2bfloat16_rn(m * sigmoid_fast(pg) * pv);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tma_store_3d(which ? &tmB : &tmA, st, j0, i, hh * 64);
-            tma_store_commit();
-        }
-    };
-
-    bool ok = __syncthreads_and(wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0));
-    if (ok && n_local > 0) {
-        ok = __syncthreads_and(wait_bounded(&zfull[0], 0, abort_flag, ctl, SITE_PRO | 2, 0));
-        if (ok) {
-            layer_norm_tile_sw128(zsm, args.ln_w, args.ln_b, args.eps);
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (threadIdx.x == 0) {
+                for (int kh = 0; kh < 2; ++kh) tma_load_2d(wsm + kh * W_HALF + w * 128 * 128, wm[w], wbar, kh * 64, 0);
+            if (n_local > 0) load_z(0);
+            if (n_local > 1) load_z(1);
+            bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0);
+            for (int lt = 0; ok && lt < n_local; ++lt) {
+                const uint32_t par = (uint32_t)lt & 1u, ppar = (uint32_t)(lt - 1) & 1u;
+                if (!wait_bounded(ln_done, par, abort_flag, ctl, SITE_PRO | 2, lt) ||
+                    (lt > 0 && !wait_bounded(a_free, ppar, abort_flag, ctl, SITE_PRO | 3, lt))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                issue_half(0, 0);
+                issue_half(0, lt & 1);
                 mma_commit(mma_a);
-                issue_half(1, 0);
+                if (lt > 0 && !wait_bounded(b_free, ppar, abort_flag, ctl, SITE_PRO | 4, lt)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                issue_half(1, lt & 1);
                 mma_commit(mma_b);
+                if (lt + 2 < n_local) {
+                    // z buffer lt & 1 is free once both projection halves of tile lt have read it.
+                    if (!wait_bounded(mma_b, par, abort_flag, ctl, SITE_PRO | 5, lt)) {
+                        ok = false;
+                        break;
+                    }
+                    load_z(lt + 2);
+                }
             }
+            if (!ok) {
+                *abort_flag = 1;
+                // Copies that may still be in flight after an abort.
+                wait_drain(wbar, 0, ctl.timeout_ns);
+                if (last_load0 >= 0) wait_drain(&zfull[0], (uint32_t)(last_load0 >> 1) & 1u, ctl.timeout_ns);
+                if (last_load1 >= 0) wait_drain(&zfull[1], (uint32_t)(last_load1 >> 1) & 1u, ctl.timeout_ns);
+            }
+            mma_commit(drain);
+            wait_drain(drain, 0, ctl.timeout_ns);
         }
-    }
-
-    for (int lt = 0; ok && lt < n_local; ++lt) {
-        const int cur = lt & 1, nxt = cur ^ 1;
-        int i, j0;
-        tile_coords(lt, i, j0);
-        const int rr = (warp & 3) * 32 + lane;  // the cell this thread gates
-        const int jj = j0 + rr;
-        float m = 0.f;
-        if (jj < args.N) m = args.mask ? __bfloat162float(args.mask[(size_t)i * args.N + jj]) : 1.f;
-
-        // a-half of tile lt
-        ok = __syncthreads_and(wait_bounded(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 3, lt));
-        if (!ok) break;
-        tc_fence_after();
-        slab(0, 0, m, i, j0);
-        slab(0, 1, m, i, j0);
-
-        // LayerNorm of tile lt+1, then its a-half MMA into the columns just drained
-        if (lt + 1 < n_local) {
-            ok = __syncthreads_and(
-                wait_bounded(&zfull[nxt], (uint32_t)((lt + 1) >> 1) & 1u, abort_flag, ctl, SITE_PRO | 4, lt));
-            if (!ok) break;
-            layer_norm_tile_sw128(zsm + nxt * Z_BYTES, args.ln_w, args.ln_b, args.eps);
+    } else {
+        // ------------------------------ worker warps ------------------------------
+        const int q = warp & 3, sub = warp >> 2;  // TMEM lane quadrant (cells 32q..32q+31), channel half
+        uint8_t *stw = stsm + warp * ST_PER_WARP * ST_BYTES;
+        int st_round = 0;
+        // LayerNorm of this warp's 16 cells of the tile in z buffer `buf`; arrive on ln_done.
+        auto normalise = [&](int buf) {
+            ln_tile_sw128<kVec>(zsm + buf * Z_BYTES, Z_HALF, args.ln_w, args.ln_b, args.eps);
             fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-                issue_half(0, nxt);
-                mma_commit(mma_a);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ln_done);
+        };
+        // Gate 32 cells x 32 channels of a (which = 0) or b (which = 1), channels hh*64 + sub*32 ..,
+        // and store them channel-major.
+        auto slab = [&](int which, int hh, const float (&hm)[4], int i, int j0) {
+            const int ch0 = hh * 64 + sub * 32;
+            uint32_t P[16];  // packed bf16 pairs: [hf][k][e] -> P[hf * 8 + k * 2 + e]
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t V[16], G[16];
+                const uint32_t ta = tmem_base + ((uint32_t)(q * 32 + 16 * hf) << 16) + (uint32_t)(which * 256 + ch0);
+                tmem_ld16x256_x4(ta, V);
+                tmem_ld16x256_x4(ta + 128, G);
+                tmem_ld_wait();
+                const __nv_bfloat16 *bv = which ? args.b_b : args.b_a;
+                const __nv_bfloat16 *bg = which ? args.b_bg : args.b_ag;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float2 g = make_float2(__uint_as_float(G[4 * k + 2 * e]), __uint_as_float(G[4 * k + 2 * e + 1]));
+                        float2 v = make_float2(__uint_as_float(V[4 * k + 2 * e]), __uint_as_float(V[4 * k + 2 * e + 1]));
+                        if (kVec) {
+                            const int c = ch0 + 8 * k + 2 * (lane & 3);
+                            if (bg) g = __fadd2_rn(g, ld_pair_bf16(bg, c));
+                            if (bv) v = __fadd2_rn(v, ld_pair_bf16(bv, c));
+                        }
+                        const float h2 = hm[hf * 2 + e];
+                        const float2 hh2 = make_float2(h2, h2);
+                        const float2 hg = __fmul2_rn(g, make_float2(0.5f, 0.5f));
+                        const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
+                        const float2 y = __fmul2_rn(__ffma2_rn(th, hh2, hh2), v);
+                        P[hf * 8 + k * 2 + e] = pack_bf16x2(y.x, y.y);
+                    }
+                }
             }
-        }
+            uint8_t *buf = stw + (st_round & 1) * ST_BYTES;
+            ++st_round;
+            if (lane == 0) tma_store_wait_read<1>();  // the store that last used `buf` has read it
+            __syncwarp();
+            // Matrix mi of a stmatrix covers channels 8k.. and cells 16hf + 8e..; thread 8mi + j
+            // addresses stored row j = channel 8k + j, whose 8 cells sit in 16-byte chunk 2hf + e
+            // (64-byte swizzle: chunk ^ ((channel >> 1) & 3)).
+            const int mi = lane >> 3, j = lane & 7;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int kp = 0; kp < 4; kp += 2) {
+                    const int k = kp + (mi >> 1), e = mi & 1;
+                    const int ch = 8 * k + j, chunk = 2 * hf + e;
+                    const uint32_t addr = smem_u32(buf) + (uint32_t)(ch * 64 + ((chunk ^ ((ch >> 1) & 3)) << 4));
+                    stmatrix_x4_trans(addr, P[hf * 8 + kp * 2 + 0], P[hf * 8 + kp * 2 + 1], P[hf * 8 + kp * 2 + 2],
+                                      P[hf * 8 + kp * 2 + 3]);
+                }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(which ? &tmB : &tmA, buf, j0 + 32 * q, i, ch0);
+                tma_store_commit();
+            }
+        };
 
-        // b-half of tile lt; its completion also frees z buffer `cur`
-        ok = __syncthreads_and(wait_bounded(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 5, lt));
-        if (!ok) break;
-        tc_fence_after();
-        if (threadIdx.x == 0 && lt + 2 < n_local) load_z(lt + 2);
-        slab(1, 0, m, i, j0);
-        slab(1, 1, m, i, j0);
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0 && lt + 1 < n_local) {
+        bool ok = n_local == 0 || warp_wait(&zfull[0], 0, abort_flag, ctl, SITE_PRO | 6, 0);
+        if (ok && n_local > 0) normalise(0);
+        for (int lt = 0; ok && lt < n_local; ++lt) {
+            int i, j0;
+            tile_coords(lt, i, j0);
+            const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
+            // hm = mask / 2 for the four cells this thread gates: 32q + 16hf + 8e + lane/4.
+            float hm[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int jj = j0 + 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
+                float m = 0.f;
+                if (jj < args.N) m = args.mask ? __bfloat162float(args.mask[(size_t)i * args.N + jj]) : 1.f;
+                hm[c] = 0.5f * m;
+            }
+            // a-half of tile lt
+            if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
             tc_fence_after();
-            issue_half(1, nxt);
-            mma_commit(mma_b);
+            if (live) {
+                slab(0, 0, hm, i, j0);
+                slab(0, 1, hm, i, j0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(a_free);
+            // LayerNorm of tile lt+1 while the b-half MMA of tile lt runs
+            if (lt + 1 < n_local) {
+                if (!(ok = warp_wait(&zfull[(lt + 1) & 1], (uint32_t)((lt + 1) >> 1) & 1u, abort_flag, ctl,
+                                     SITE_PRO | 8, lt)))
+                    break;
+                normalise((lt + 1) & 1);
+            }
+            // b-half of tile lt
+            if (!(ok = warp_wait(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 9, lt))) break;
+            tc_fence_after();
+            if (live) {
+                slab(1, 0, hm, i, j0);
+                slab(1, 1, hm, i, j0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_free);
         }
+        if (!ok && lane == 0) *abort_flag = 1;
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
-    // Teardown: stores drained, loads landed, MMAs finished, TMEM released.
-    if (threadIdx.x == 0) {
-        tma_store_wait_all<0>();
-        if (!ok) {
-            // Copies that may still be in flight after an abort.
-            wait_drain(wbar, 0, ctl.timeout_ns);
-            for (int b = 0; b < 2; ++b)
-                if (last_load[b] >= 0) wait_drain(&zfull[b], (uint32_t)(last_load[b] >> 1) & 1u, ctl.timeout_ns);
-        }
-        mma_commit(drain);
-        wait_drain(drain, 0, ctl.timeout_ns);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem_base, 512);
+    if (warp == WORKERS) tmem_dealloc(tmem_base, 512);
 }
 
 size_t prologue_tc_smem() { return pro::SMEM; }
 
 cudaError_t prologue_tc_setup() {
-    return cudaFuncSetAttribute(prologue_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pro::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(prologue_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pro::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(prologue_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pro::SMEM);
 }
 
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
-    prologue_tc_kernel<<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.a, m.b, a);
+    const bool vec = a.ln_w || a.ln_b || a.b_a || a.b_ag || a.b_b || a.b_bg;
+    if (vec)
+        prologue_tc_kernel<true><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.a, m.b, a);
+    else
+        prologue_tc_kernel<false><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.a, m.b,
+                                                                         a);
     return cudaGetLastError();
 }
 
