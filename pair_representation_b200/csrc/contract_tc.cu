@@ -46,64 +46,6 @@ constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_OUT * OUT_BYTE
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace con
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
-    uint32_t out;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
-    return out;
-}
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void st_remote_u32(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// TMA load into this CTA's shared memory whose bytes complete on a barrier of
-// the leader CTA of the pair (cluster address).
-__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int c0,
-                                                 int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Arrive on `bar` (same offset) in both CTAs of the pair once this thread's MMAs have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"((uint16_t)0x3)
-        : "memory");
-}
-__device__ __forceinline__ void mma_commit_local2(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
     contract_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmX, const ContractArgs args) {
@@ -169,6 +111,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
         *abort_flag = 1;
         st_remote_u32(peer_abort, 1u);
     };
+    // Which 128-row half of a 256-row tile edge starting at `base` CTA `r` loads.
+    // Normally CTA r takes half r. Where the upper half would be only partly
+    // inside [0, N), the CTAs swap, so CTA 1 (whose loads complete on CTA 0's
+    // barrier) always loads a half that is fully inside or fully outside the
+    // matrix; the partial half is loaded by CTA 0 onto its own barrier.
+    auto half_of = [&](int base, uint32_t r) -> int {
+        const bool swap = base + HALF < args.N && args.N < base + 2 * HALF;
+        return (int)(r ^ (swap ? 1u : 0u));
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -185,7 +136,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
                 const int c = tile / tiles_per_c;
                 const int r = tile - c * tiles_per_c;
                 const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
-                const int i0 = ti * 256 + (int)rank * HALF, j0 = tj * BN + (int)rank * HALF;
+                const int i0 = ti * 256 + half_of(ti * 256, rank) * HALF;
+                const int j0 = tj * BN + half_of(tj * BN, rank) * HALF;
                 for (int kb = 0; kb < args.kblocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, ctl, SITE_CON | 1, tile)) {
                         ok = false;
@@ -301,7 +253,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
             const int c = tile / tiles_per_c;
             const int r = tile - c * tiles_per_c;
             const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
-            const int i0 = ti * 256 + (int)rank * HALF, j0 = tj * BN;
+            // This CTA's accumulator rows are the A rows it loaded; accumulator columns
+            // [0,128) come from CTA 0's B rows and [128,256) from CTA 1's.
+            const int i0 = ti * 256 + half_of(ti * 256, rank) * HALF;
+            const int jb0 = tj * BN + half_of(tj * BN, 0) * HALF, jb1 = tj * BN + half_of(tj * BN, 1) * HALF;
             const int acc = lt & 1;
             const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
             if (leader) {
@@ -314,26 +269,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
             tc_fence_after();
             // Chunks whose first column is past N, and whole halves whose first row is past N,
             // are neither read nor stored.
-            const int nch = (i0 < args.N) ? min(BN / OUT_COLS, (args.N - j0 + OUT_COLS - 1) / OUT_COLS) : 0;
-            if (nch == 0) {
-                tc_fence_before();
-                if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
-            }
+            int nst = 0;  // stores issued for this tile
 #pragma unroll 1
-            for (int ch = 0; ch < nch; ++ch) {
+            for (int ch = 0; ch < BN / OUT_COLS; ++ch) {
+                const int jst = (ch < 2 ? jb0 : jb1) + (ch & 1) * OUT_COLS;
+                if (i0 >= args.N || jst >= args.N) continue;
                 uint32_t v[64];
                 const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * OUT_COLS);
                 tmem_ld32(taddr, v);
                 tmem_ld32(taddr + 32, v + 32);
                 tmem_ld_wait();
-                if (ch == nch - 1) {
-                    tc_fence_before();
-                    if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
-                }
                 uint32_t p[32];
 #pragma unroll
                 for (int k = 0; k < 32; ++k) p[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-                uint8_t *ob = outbuf + (ch & 1) * OUT_BYTES;
+                uint8_t *ob = outbuf + (nst & 1) * OUT_BYTES;
+                ++nst;
                 if (leader) tma_store_wait_read<1>();
                 named_bar_sync(1, 128);
 #pragma unroll
@@ -344,10 +294,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (leader) {
-                    tma_store_3d(&tmX, ob, j0 + ch * OUT_COLS, i0, c);
+                    tma_store_3d(&tmX, ob, jst, i0, c);
                     tma_store_commit();
                 }
             }
+            // Every TMEM read of this accumulator is complete: hand it back to the MMA.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
         }
         if (leader) tma_store_wait_all<0>();
     }

@@ -56,7 +56,7 @@ def test_fp32_edge_sizes(N, direction):
 
 # ---------------------------------------------------------------- bf16 stages
 
-@pytest.mark.parametrize("N", [64, 200, 256, 300, 385])
+@pytest.mark.parametrize("N", [64, 129, 200, 256, 300, 385, 386, 513])
 @pytest.mark.parametrize("direction", ["outgoing", "incoming"])
 def test_bf16_contraction_stage(N, direction):
     """x from random bf16 a, b written into the workspace, vs the oracle contraction."""
