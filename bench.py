@@ -66,10 +66,10 @@ def load_peaks():
 
 
 def source_sha(kernel: str) -> str:
-    fname = {"prologue_tc_kernel": "prologue_tc.cu", "contract_tc_kernel": "contract_tc.cu",
-             "epilogue_tc_kernel": "epilogue_tc.cu"}[kernel]
+    files = {"prologue_tc_kernel": ("prologue_tc.cu", "tile_ops.cuh"), "contract_tc_kernel": ("contract_tc.cu",),
+             "epilogue_tc_kernel": ("epilogue_tc.cu", "tile_ops.cuh")}[kernel]
     h = hashlib.sha256()
-    for f in (fname, "common.cuh", "kernels.h"):
+    for f in files + ("common.cuh", "kernels.h"):
         with open(os.path.join(ROOT, "pair_representation_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

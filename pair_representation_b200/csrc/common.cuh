@@ -97,23 +97,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed is
+// suspended in hardware until it completes or `hint_ns` passes, instead of
+// spinning through the issue slots the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kWaitHintNs = 1000000;  // upper bound on one suspension: 1 ms
+
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Returns true on completion. Returns false if another thread of the CTA has
 // raised `abort_flag`, or if this wait ran past ctl.timeout_ns; in the latter
-// case it raises the flag and records DEV_TIMEOUT with `site`.
+// case it raises the flag and records DEV_TIMEOUT with `site`. May be called by
+// one thread or by every lane of a warp.
 static __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           const KernelCtl &ctl, int site, int aux) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0u) {
-            if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > ctl.timeout_ns) {
-                *abort_flag = 1;
-                record_failure(ctl, DEV_TIMEOUT, site, aux);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+            *abort_flag = 1;
+            record_failure(ctl, DEV_TIMEOUT, site, aux);
+            return false;
         }
     }
 }
@@ -123,9 +138,9 @@ static __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
 static __device__ __noinline__ bool wait_drain(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -221,6 +236,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// 32 lanes x 16 consecutive 32-bit columns: thread t gets lane (base + t),
+// columns col..col+15 of `taddr` in r[0..15].
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 16 lanes x 256 bits, 4 repetitions along columns (32 columns): thread t gets, for
@@ -260,12 +285,12 @@ __device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
     return r != 0;
 }
 
-// Bounded wait by lane 0 of a warp, result broadcast to the warp.
+// Bounded wait by every lane of a warp (the warp stays converged and sleeps in
+// try_wait); the outcome is made warp-uniform.
 static __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                  const KernelCtl &ctl, int site, int aux) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, abort_flag, ctl, site, aux) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    const int ok = wait_bounded(bar, parity, abort_flag, ctl, site, aux) ? 1 : 0;
+    return __all_sync(0xffffffffu, ok) != 0;
 }
 
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle.

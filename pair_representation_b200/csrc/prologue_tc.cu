@@ -12,22 +12,25 @@
 //
 // Tiles are 128 consecutive cells of one residue row (z[i][j0 .. j0+127][:],
 // one contiguous 32 KB block). The four weight matrices (128 KB bf16) stay in
-// shared memory for the whole persistent CTA. Roles (288 threads):
-//   warp 8 (control): TMA loads of z, the two projection MMAs per tile
-//     (a-half D[:, 0:256] = zh [W_a; W_ag]^T, b-half D[:, 256:512] = zh [W_b; W_bg]^T,
-//     M = 128 cells, N = 256, K = 128, all 512 TMEM columns), gated by
-//     mbarriers the workers arrive on.
-//   warps 0-7 (workers), each on its own, with no CTA-wide barrier:
-//     * LayerNorm of 16 cells of the next tile in place (fp32 statistics);
-//     * gating of 32 cells x 32 channels of a and of b: TMEM is read in the
-//       16-lane fragment layout, the gate m * sigmoid(g) * v is formed in
-//       packed fp32x2, the bf16 results are written channel-major with
-//       stmatrix.trans into a 64-byte-swizzled 2 KB buffer of the warp and
-//       stored by that warp's own TMA store.
-// Per tile the workers arrive on ln_done (next tile normalised), a_free (a-half
-// TMEM columns read) and b_free; the control warp issues the next tile's MMAs
-// into columns as soon as they are free, so tensor work, gating and the z loads
-// of two tiles ahead overlap.
+// shared memory for the whole persistent CTA. Roles (416 threads), coupled
+// only through mbarriers:
+//   warp 12 (control): TMA loads of z (two tiles ahead), the two projection
+//     MMAs per tile (a-half D[:, 0:256] = zh [W_a; W_ag]^T, b-half
+//     D[:, 256:512] = zh [W_b; W_bg]^T, M = 128 cells, N = 256, K = 128, all
+//     512 TMEM columns).
+//   warps 8-11 (normalisers): LayerNorm of each landed tile in place (fp32
+//     statistics, two threads per cell), ahead of its MMAs.
+//   warps 0-7 (workers): gating of 32 cells x 32 channels of a and of b: TMEM
+//     is read in the 16-lane fragment layout, m * sigmoid(g) * v is formed in
+//     packed fp32x2, the bf16 results are written channel-major with
+//     stmatrix.trans into a 64-byte-swizzled 2 KB buffer of the warp and
+//     stored by that warp's own TMA store, so no warp waits on global writes.
+// The control warp issues the next tile's a-half MMAs as soon as that tile is
+// normalised and the workers have read the a-half columns, and the b-half as
+// soon as they have read the b-half columns: tensor work, gating,
+// normalisation and the z loads of two tiles ahead overlap. Every wait sleeps
+// in mbarrier.try_wait rather than spinning, which keeps issue slots and the
+// shared-memory pipe free for the warps doing work.
 #include "kernels.h"
 #include "tile_ops.cuh"
 
@@ -35,7 +38,9 @@ namespace trimul {
 namespace pro {
 constexpr int TILE = 128;
 constexpr int WORKERS = 8;
-constexpr int THREADS = 32 * (WORKERS + 1);
+constexpr int NORMS = 4;
+constexpr int CTRL_WARP = WORKERS + NORMS;
+constexpr int THREADS = 32 * (CTRL_WARP + 1);
 constexpr int W_HALF = 512 * 128;       // one 64-channel K half of the 4 stacked weights: 64 KB
 constexpr int W_BYTES = 2 * W_HALF;     // 128 KB
 constexpr int Z_HALF = TILE * 128;      // 16 KB
@@ -67,11 +72,11 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     uint64_t *zfull = bars + 1;   // [2] z tile landed
     uint64_t *mma_a = bars + 3;   // a-half projections done
     uint64_t *mma_b = bars + 4;   // b-half projections done
-    uint64_t *ln_done = bars + 5; // workers: next tile normalised (8 arrivals)
-    uint64_t *a_free = bars + 6;  // workers: a-half TMEM columns read (8 arrivals)
-    uint64_t *b_free = bars + 7;  // workers: b-half TMEM columns read (8 arrivals)
-    uint64_t *drain = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+    uint64_t *a_free = bars + 5;  // workers: a-half TMEM columns read (8 arrivals)
+    uint64_t *b_free = bars + 6;  // workers: b-half TMEM columns read (8 arrivals)
+    uint64_t *drain = bars + 7;
+    uint64_t *ln_done = bars + 8; // [2] normalisers: tile in z buffer b normalised (4 arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,14 +91,15 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         mbar_init(&zfull[1], 1);
         mbar_init(mma_a, 1);
         mbar_init(mma_b, 1);
-        mbar_init(ln_done, WORKERS);
+        mbar_init(&ln_done[0], NORMS);
+        mbar_init(&ln_done[1], NORMS);
         mbar_init(a_free, WORKERS);
         mbar_init(b_free, WORKERS);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == WORKERS) {
+    if (warp == CTRL_WARP) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -108,7 +114,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         j0 = (tile - i * args.jt_tiles) * TILE;
     };
 
-    if (warp == WORKERS) {
+    if (warp == CTRL_WARP) {
         // ------------------------------ control warp ------------------------------
         if (lane == 0) {
             int last_load0 = -1, last_load1 = -1;
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0);
             for (int lt = 0; ok && lt < n_local; ++lt) {
                 const uint32_t par = (uint32_t)lt & 1u, ppar = (uint32_t)(lt - 1) & 1u;
-                if (!wait_bounded(ln_done, par, abort_flag, ctl, SITE_PRO | 2, lt) ||
+                if (!wait_bounded(&ln_done[lt & 1], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 2, lt) ||
                     (lt > 0 && !wait_bounded(a_free, ppar, abort_flag, ctl, SITE_PRO | 3, lt))) {
                     ok = false;
                     break;
@@ -180,18 +186,26 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             mma_commit(drain);
             wait_drain(drain, 0, ctl.timeout_ns);
         }
+    } else if (warp >= WORKERS) {
+        // ------------------------------ normalisers ------------------------------
+        const int t = (warp - WORKERS) * 32 + lane;  // 0..127: cells t/2 and 64 + t/2, channel half t % 2
+        bool ok = true;
+        for (int lt = 0; lt < n_local; ++lt) {
+            const int b = lt & 1;
+            if (!(ok = warp_wait(&zfull[b], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 6, lt))) break;
+            uint8_t *tile = zsm + b * Z_BYTES;
+            ln_row_sw128<kVec>(tile, Z_HALF, t >> 1, t & 1, args.ln_w, args.ln_b, args.eps);
+            ln_row_sw128<kVec>(tile, Z_HALF, 64 + (t >> 1), t & 1, args.ln_w, args.ln_b, args.eps);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ln_done[b]);
+        }
+        if (!ok && lane == 0) *abort_flag = 1;
     } else {
         // ------------------------------ worker warps ------------------------------
         const int q = warp & 3, sub = warp >> 2;  // TMEM lane quadrant (cells 32q..32q+31), channel half
         uint8_t *stw = stsm + warp * ST_PER_WARP * ST_BYTES;
         int st_round = 0;
-        // LayerNorm of this warp's 16 cells of the tile in z buffer `buf`; arrive on ln_done.
-        auto normalise = [&](int buf) {
-            ln_tile_sw128<kVec>(zsm + buf * Z_BYTES, Z_HALF, args.ln_w, args.ln_b, args.eps);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ln_done);
-        };
         // Gate 32 cells x 32 channels of a (which = 0) or b (which = 1), channels hh*64 + sub*32 ..,
         // and store them channel-major.
         auto slab = [&](int which, int hh, const float (&hm)[4], int i, int j0) {
@@ -252,14 +266,11 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             }
         };
 
-        bool ok = n_local == 0 || warp_wait(&zfull[0], 0, abort_flag, ctl, SITE_PRO | 6, 0);
-        if (ok && n_local > 0) normalise(0);
-        for (int lt = 0; ok && lt < n_local; ++lt) {
+        // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4.
+        // Fetched one tile ahead, so the loads' latency stays off the gating path.
+        auto fetch_hm = [&](int lt, float (&hm)[4]) {
             int i, j0;
             tile_coords(lt, i, j0);
-            const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
-            // hm = mask / 2 for the four cells this thread gates: 32q + 16hf + 8e + lane/4.
-            float hm[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int jj = j0 + 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
@@ -267,6 +278,17 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                 if (jj < args.N) m = args.mask ? __bfloat162float(args.mask[(size_t)i * args.N + jj]) : 1.f;
                 hm[c] = 0.5f * m;
             }
+        };
+        float nhm[4] = {0.f, 0.f, 0.f, 0.f};
+        if (n_local > 0) fetch_hm(0, nhm);
+
+        bool ok = true;
+        for (int lt = 0; ok && lt < n_local; ++lt) {
+            int i, j0;
+            tile_coords(lt, i, j0);
+            const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
+            const float hm[4] = {nhm[0], nhm[1], nhm[2], nhm[3]};
+            if (lt + 1 < n_local) fetch_hm(lt + 1, nhm);
             // a-half of tile lt
             if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
             tc_fence_after();
@@ -277,13 +299,6 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(a_free);
-            // LayerNorm of tile lt+1 while the b-half MMA of tile lt runs
-            if (lt + 1 < n_local) {
-                if (!(ok = warp_wait(&zfull[(lt + 1) & 1], (uint32_t)((lt + 1) >> 1) & 1u, abort_flag, ctl,
-                                     SITE_PRO | 8, lt)))
-                    break;
-                normalise((lt + 1) & 1);
-            }
             // b-half of tile lt
             if (!(ok = warp_wait(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 9, lt))) break;
             tc_fence_after();
@@ -302,7 +317,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == WORKERS) tmem_dealloc(tmem_base, 512);
+    if (warp == CTRL_WARP) tmem_dealloc(tmem_base, 512);
 }
 
 size_t prologue_tc_smem() { return pro::SMEM; }

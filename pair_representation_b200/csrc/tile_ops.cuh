@@ -21,16 +21,15 @@ __device__ __forceinline__ float2 ld_pair_bf16(const __nv_bfloat16 *v, int c) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(v + c));
 }
 
-// In-place LayerNorm of a 128-cell x 128-channel bf16 tile stored as two
-// 64-channel halves (half_bytes apart) of 128-byte rows with the 128-byte
-// swizzle (16-byte chunk index XOR row & 7). Two threads per cell (one per
-// half, partners in adjacent lanes), fp32 statistics, bf16 result.
-// kAffine: apply gamma/beta (bf16 vectors; a null one means 1 or 0).
+// In-place LayerNorm of one 128-channel cell (row r) of a bf16 tile stored as
+// two 64-channel halves (half_bytes apart) of 128-byte rows with the 128-byte
+// swizzle (16-byte chunk index XOR row & 7). Two threads per cell: this thread
+// takes channel half h and its partner (lane ^ 1) the other half. fp32
+// statistics, bf16 result. kAffine: apply gamma/beta (bf16 vectors; a null
+// one means 1 or 0).
 template <bool kAffine>
-__device__ __forceinline__ void ln_tile_sw128(uint8_t *tile, int half_bytes, const __nv_bfloat16 *gw,
-                                              const __nv_bfloat16 *gb, float eps) {
-    const int t = threadIdx.x;
-    const int r = t >> 1, h = t & 1;
+__device__ __forceinline__ void ln_row_sw128(uint8_t *tile, int half_bytes, int r, int h, const __nv_bfloat16 *gw,
+                                             const __nv_bfloat16 *gb, float eps) {
     uint8_t *rowp = tile + h * half_bytes + r * 128;
     float2 v[32];  // register slot q*4 + e holds logical chunk kc = (q + 4h) & 7, word e
 #pragma unroll
@@ -85,6 +84,13 @@ __device__ __forceinline__ void ln_tile_sw128(uint8_t *tile, int half_bytes, con
         }
         *reinterpret_cast<uint4 *>(rowp + ((kc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+}
+
+// The whole 128-cell tile by 256 threads (thread t: cell t / 2, half t % 2).
+template <bool kAffine>
+__device__ __forceinline__ void ln_tile_sw128(uint8_t *tile, int half_bytes, const __nv_bfloat16 *gw,
+                                              const __nv_bfloat16 *gb, float eps) {
+    ln_row_sw128<kAffine>(tile, half_bytes, (int)threadIdx.x >> 1, (int)threadIdx.x & 1, gw, gb, eps);
 }
 
 }  // namespace trimul
