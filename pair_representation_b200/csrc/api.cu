@@ -250,6 +250,13 @@ int map_pair(CUtensorMap *m, const void *t, int N, uint32_t b0, uint32_t b1, CUt
     return encode(m, 3, t, dims, strides, box, sw);
 }
 
+// mask [N][pitch] as (j, i): one row segment of 128 cells per box, zero past column N.
+int map_mask(CUtensorMap *m, const void *t, int N, size_t pitch) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)N}, strides[1] = {pitch * 2};
+    const uint32_t box[2] = {128, 1};
+    return encode(m, 2, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 // a, b or x [128][N][ld] as (col, row, c) with the given box and swizzle.
 int map_cm(CUtensorMap *m, const void *t, int N, size_t ld, uint32_t b0, uint32_t b1, uint32_t b2,
            CUtensorMapSwizzle sw) {
@@ -308,6 +315,23 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
     for (int k = 0; k < 4; ++k)
         if (int rc = map_weight(&m.w[k], w[k])) return rc;
     if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    // The mask rows travel with the z tiles. A tensor map needs a 16-byte row pitch, so a
+    // mask whose rows do not have one is first copied into plane 0 of x (pitch ld), which the
+    // contraction overwrites later.
+    m.mask = m.z;  // unused without a mask
+    if (mask) {
+        const void *src = mask;
+        size_t pitch = (size_t)p->N;
+        if (p->N % 8 != 0 || !aligned(mask, 16)) {
+            __nv_bfloat16 *pad = reinterpret_cast<__nv_bfloat16 *>(v.x);
+            if (int rc = cuda_rc(launch_mask_pad(static_cast<const __nv_bfloat16 *>(mask), pad, p->N, (int)v.ld, s),
+                                 "mask_pad launch"))
+                return rc;
+            src = pad;
+            pitch = v.ld;
+        }
+        if (int rc = map_mask(&m.mask, src, p->N, pitch)) return rc;
+    }
     // Each worker warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
     if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
@@ -316,7 +340,7 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
     a.jt_tiles = (p->N + 127) / 128;
     a.total_tiles = p->N * a.jt_tiles;
     a.eps = p->ln_eps;
-    a.mask = static_cast<const __nv_bfloat16 *>(mask);
+    a.has_mask = mask != nullptr;
     a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
     a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
     a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);

@@ -18,7 +18,7 @@ struct PrologueArgs {
     int jt_tiles;     // ceil(N / 128): 128-cell tiles per residue row
     int total_tiles;  // N * jt_tiles
     float eps;
-    const __nv_bfloat16 *mask;                 // [N][N] or null
+    int has_mask;                              // mask rows arrive by TMA (tensor map `mask`)
     const __nv_bfloat16 *ln_w, *ln_b;          // [128] or null
     const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
     KernelCtl ctl;
@@ -27,6 +27,7 @@ struct PrologueArgs {
 struct PrologueMaps {
     CUtensorMap w[4];  // W_a, W_ag, W_b, W_bg: 2-D [128 out][128 in], box 64 x 128, swizzle 128B
     CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 128, 1), swizzle 128B
+    CUtensorMap mask;  // 2-D (j, i) over the [N][pitch] bf16 mask, box (128, 1), no swizzle
     CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (32, 1, 32), swizzle 64B
 };
 
@@ -68,6 +69,8 @@ size_t epilogue_tc_smem();
 cudaError_t prologue_tc_setup();
 cudaError_t epilogue_tc_setup();
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s);
+// Copies the [N][N] mask into rows of pitch ld (zero past column N), for a tensor map.
+cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int ld, cudaStream_t s);
 size_t contract_tc_smem();
 cudaError_t contract_tc_setup();
 // Clusters of 2 CTAs, one 256 x 256 output tile per pair; grid = 2 x pairs.

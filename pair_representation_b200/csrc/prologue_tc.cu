@@ -47,9 +47,11 @@ constexpr int Z_HALF = TILE * 128;      // 16 KB
 constexpr int Z_BYTES = 2 * Z_HALF;     // 32 KB
 constexpr int ST_BYTES = 32 * 32 * 2;   // 2 KB per warp buffer: [32 ch][32 cells], 64-byte swizzle
 constexpr int ST_PER_WARP = 2;
+constexpr int MASK_SLOTS = 4;           // mask rows of tiles lt .. lt + 3 (indexed lt % 4)
+constexpr int MASK_BYTES = TILE * 2;     // one bf16 mask row segment per tile
 constexpr int BAR_BYTES = 128;
-constexpr size_t SMEM =
-    1024 + (size_t)W_BYTES + 2 * Z_BYTES + (size_t)WORKERS * ST_PER_WARP * ST_BYTES + BAR_BYTES;
+constexpr size_t SMEM = 1024 + (size_t)W_BYTES + 2 * Z_BYTES + (size_t)WORKERS * ST_PER_WARP * ST_BYTES +
+                        MASK_SLOTS * MASK_BYTES + BAR_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pro
 
@@ -59,7 +61,8 @@ template <bool kVec>
 __global__ void __launch_bounds__(pro::THREADS, 1)
     prologue_tc_kernel(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWag,
                        const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmWbg,
-                       const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmMask,
+                       const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const PrologueArgs args) {
     using namespace pro;
     extern __shared__ uint8_t smem_raw[];
@@ -67,7 +70,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     uint8_t *wsm = smem;
     uint8_t *zsm = smem + W_BYTES;                 // [2] z tiles
     uint8_t *stsm = zsm + 2 * Z_BYTES;             // [8 warps][2] staging buffers
-    uint64_t *bars = reinterpret_cast<uint64_t *>(stsm + WORKERS * ST_PER_WARP * ST_BYTES);
+    uint8_t *msm = stsm + WORKERS * ST_PER_WARP * ST_BYTES;  // [4] mask rows (bf16)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(msm + MASK_SLOTS * MASK_BYTES);
     uint64_t *wbar = bars;        // weights landed
     uint64_t *zfull = bars + 1;   // [2] z tile landed
     uint64_t *mma_a = bars + 3;   // a-half projections done
@@ -123,9 +127,12 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                 tile_coords(lt, i, j0);
                 if (lt & 1) last_load1 = lt; else last_load0 = lt;
                 uint8_t *dst = zsm + (lt & 1) * Z_BYTES;
-                mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES);
+                mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES + (args.has_mask ? MASK_BYTES : 0));
                 tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
                 tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
+                // Mask slot lt % 4 last served tile lt - 4, whose gating ended before the b-half
+                // MMA of tile lt - 2, which this load waited for.
+                if (args.has_mask) tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
             };
             // D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T over K = 128.
             auto issue_half = [&](int half, int buf) {
@@ -266,32 +273,30 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             }
         };
 
-        // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4.
-        // Fetched one tile ahead, so the loads' latency stays off the gating path.
-        auto fetch_hm = [&](int lt, float (&hm)[4]) {
-            int i, j0;
-            tile_coords(lt, i, j0);
+        // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4,
+        // from the mask row that landed with the tile (zero past column N).
+        auto read_hm = [&](int lt, int j0, float (&hm)[4]) {
+            const uint16_t *mrow = reinterpret_cast<const uint16_t *>(msm + (lt & 3) * MASK_BYTES);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int jj = j0 + 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
-                float m = 0.f;
-                if (jj < args.N) m = args.mask ? __bfloat162float(args.mask[(size_t)i * args.N + jj]) : 1.f;
-                hm[c] = 0.5f * m;
+                const int jc = 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
+                if (args.has_mask)
+                    hm[c] = 0.5f * bf16_bits_to_float(mrow[jc]);
+                else
+                    hm[c] = j0 + jc < args.N ? 0.5f : 0.f;
             }
         };
-        float nhm[4] = {0.f, 0.f, 0.f, 0.f};
-        if (n_local > 0) fetch_hm(0, nhm);
 
         bool ok = true;
         for (int lt = 0; ok && lt < n_local; ++lt) {
             int i, j0;
             tile_coords(lt, i, j0);
             const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
-            const float hm[4] = {nhm[0], nhm[1], nhm[2], nhm[3]};
-            if (lt + 1 < n_local) fetch_hm(lt + 1, nhm);
             // a-half of tile lt
             if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
             tc_fence_after();
+            float hm[4];  // tile lt landed (its a-half MMAs ran after it was normalised)
+            read_hm(lt, j0, hm);
             if (live) {
                 slab(0, 0, hm, i, j0);
                 slab(0, 1, hm, i, j0);
@@ -332,10 +337,22 @@ cudaError_t prologue_tc_setup() {
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
     const bool vec = a.ln_w || a.ln_b || a.b_a || a.b_ag || a.b_b || a.b_bg;
     if (vec)
-        prologue_tc_kernel<true><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.a, m.b, a);
+        prologue_tc_kernel<true><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
+                                                                        m.a, m.b, a);
     else
-        prologue_tc_kernel<false><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.a, m.b,
-                                                                         a);
+        prologue_tc_kernel<false><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
+                                                                         m.a, m.b, a);
+    return cudaGetLastError();
+}
+
+__global__ void mask_pad_kernel(const __nv_bfloat16 *__restrict__ mask, __nv_bfloat16 *__restrict__ dst, int N,
+                                int ld) {
+    const size_t i = blockIdx.x;
+    for (int j = threadIdx.x; j < ld; j += blockDim.x) dst[i * ld + j] = j < N ? mask[i * N + j] : __float2bfloat16(0.f);
+}
+
+cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int ld, cudaStream_t s) {
+    mask_pad_kernel<<<N, 128, 0, s>>>(mask, dst, N, ld);
     return cudaGetLastError();
 }
 
