@@ -392,7 +392,8 @@ int run_epilogue(const void *z, const trimul_params *p, void *out, const DevStat
     if (int rc = map_weight(&m.wg, p->w_g)) return rc;
     if (int rc = map_weight(&m.wo, p->w_o)) return rc;
     if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 128, 1, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    // x as the MN-major MMA operand: 64 cells x 128 channels per box, 128-byte swizzle.
+    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     // Each worker warp stores 32 channels x 32 cells (64-byte rows, 64-byte swizzle).
     if (int rc = map_pair(&m.out, out, p->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     EpilogueArgs a;

@@ -9,102 +9,73 @@
 // The gate is recomputed from z rather than stored by the prologue: reading z
 // again costs 256 B per cell against 512 B per cell to write and re-read g.
 //
-// Tiles are 128 consecutive cells of one residue row. Roles (288 threads):
-//   warp 8 (control): TMA loads of the x tile ([128 ch][128 cells], as the
-//     contraction wrote it) and the z tile (128-byte swizzle), two tiles ahead;
-//     per tile two MMAs, G = zh W_g^T and O = xh W_o^T (M = 128 cells,
-//     N = 128, K = 128), into a double-buffered 256-column TMEM accumulator.
-//   warps 0-7 (workers):
-//     * LayerNorm of z in place (16 cells per warp) and of x, read down its
-//       columns and written back in place, transposed, as the swizzled
-//       cell-major MMA operand (32 cells x 64 channels per warp, the
-//       workers meeting at a 256-thread named barrier);
-//     * out = sigmoid(G + b_g) * (O + b_o) for 32 cells x 32 channels per
-//       warp in packed fp32x2, bf16, into a 64-byte-swizzled 2 KB buffer of
-//       the warp and out by that warp's own TMA store.
-// The next tile's LayerNorms run before this tile's gating, so its MMAs
-// overlap the gating; the only barrier in the tile loop is the workers' x LayerNorm.
+// Both LayerNorms are folded into their projections. With per-cell mean mu and
+// rstd r, and W' = W diag(gamma):
+//   W LN(v) + bias = r (W' v - mu s) + t,   s[n] = sum_k W'[n][k],
+//                                            t[n] = sum_k W[n][k] beta[k] + bias[n].
+// The MMAs therefore run on the raw tiles exactly as TMA lands them: z as the
+// K-major operand and x, which the contraction wrote channel-major, as the
+// MN-major operand. No warp rewrites a tile and the tensor work never waits
+// for a LayerNorm. s is summed from the same bf16 W' the MMA reads, so the
+// mean term cancels as it would in exact arithmetic.
+//
+// Tiles are 128 consecutive cells of one residue row. Roles (416 threads):
+//   all, once: W' = W gamma in shared memory, s and t per output channel.
+//   warp 12 (control): TMA loads of the x and z tiles two tiles ahead; per tile
+//     G = z W_g'^T and O = x W_o'^T (M = 128 cells, N = 128, K = 128) into a
+//     double-buffered 256-column TMEM accumulator.
+//   warps 8-11 (statistics): mean and rstd of z and of x for each cell of a
+//     landed tile (one thread per cell), into a two-slot table.
+//   warps 0-7 (gaters): warp w reads TMEM lanes 32(w % 4).. (its 32 cells) and
+//     channels 64(w / 4)..+63 of G and O, forms
+//     sigmoid(r_z (G - mu_z s_g) + t_g) * (r_x (O - mu_x s_o) + t_o) in packed
+//     fp32x2, and writes the bf16 result into a 64-byte-swizzled 2 KB buffer of
+//     the warp, stored by that warp's own TMA store.
 #include "kernels.h"
 #include "tile_ops.cuh"
 
 namespace trimul {
 namespace epi {
 constexpr int TILE = 128;
-constexpr int WORKERS = 8;
-constexpr int THREADS = 32 * (WORKERS + 1);
-constexpr int W_HALF = 128 * 128;        // one 64-channel K half of a 128 x 128 weight: 16 KB
-constexpr int W_BYTES = 2 * W_HALF;      // 32 KB per weight
-constexpr int T_HALF = TILE * 128;       // 16 KB
-constexpr int T_BYTES = 2 * T_HALF;      // 32 KB per tile buffer (x or z)
-constexpr int ST_BYTES = 32 * 32 * 2;    // 2 KB per warp buffer: [32 cells][32 ch], 64-byte swizzle
-constexpr int ST_PER_WARP = 2;
-constexpr int RED_BYTES = 2 * TILE * 4;  // x LayerNorm partials of the two channel halves
+constexpr int GATERS = 8;
+constexpr int STATS = 4;
+constexpr int CTRL_WARP = GATERS + STATS;
+constexpr int THREADS = 32 * (CTRL_WARP + 1);
+constexpr int W_HALF = 128 * 128;          // one 64-channel K half of a 128 x 128 weight: 16 KB
+constexpr int W_BYTES = 2 * W_HALF;        // 32 KB per weight
+constexpr int T_HALF = TILE * 128;         // 16 KB
+constexpr int T_BYTES = 2 * T_HALF;        // 32 KB per tile buffer (x or z)
+constexpr int ST_BYTES = 32 * 32 * 2;      // 2 KB per warp buffer: [32 cells][32 ch], 64-byte swizzle
+constexpr int CST_BYTES = 4 * 128 * 4;     // s_g, s_o, t_g / 2, t_o / 2
+constexpr int STAT_BYTES = 2 * TILE * 16;  // two slots of (-mu_z, r_z / 2, -mu_x, r_x / 2) per cell
 constexpr int BAR_BYTES = 128;
-constexpr size_t SMEM = 1024 + 2 * (size_t)W_BYTES + 2 * 2 * (size_t)T_BYTES +
-                        (size_t)WORKERS * ST_PER_WARP * ST_BYTES + RED_BYTES + BAR_BYTES;
+constexpr size_t SMEM = 1024 + 2 * (size_t)W_BYTES + 2 * 2 * (size_t)T_BYTES + (size_t)GATERS * ST_BYTES +
+                        CST_BYTES + STAT_BYTES + BAR_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace epi
 
-// LayerNorm of a channel-major x tile [128 ch][128 cells], written back in
-// place as the swizzled cell-major [2 halves][128 cells][64 ch] MMA operand.
-// Worker warp w owns cells 32(w & 3) .. +31 and channel half w >> 2; the two
-// halves of a cell meet through `red`. The in-place transposition needs every
-// worker to finish reading before any writes, so the steps are separated by
-// named barrier 1 over the 256 worker threads.
-template <bool kAffine>
-__device__ __forceinline__ void epi_layer_norm_x(uint8_t *xt, float *red, const __nv_bfloat16 *gw,
-                                                 const __nv_bfloat16 *gb, float eps) {
-    const int t = threadIdx.x;
-    const int r = t & 127, h = t >> 7;
-    const uint16_t *col = reinterpret_cast<const uint16_t *>(xt) + h * 64 * epi::TILE + r;
-    float2 v[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-        v[k] = make_float2(bf16_bits_to_float(col[(2 * k) * epi::TILE]), bf16_bits_to_float(col[(2 * k + 1) * epi::TILE]));
-    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-        a0 = __fadd2_rn(a0, v[k]);
-        a1 = __fadd2_rn(a1, v[k + 1]);
-        a2 = __fadd2_rn(a2, v[k + 2]);
-        a3 = __fadd2_rn(a3, v[k + 3]);
-    }
-    red[h * epi::TILE + r] = (a0.x + a0.y) + (a1.x + a1.y) + (a2.x + a2.y) + (a3.x + a3.y);
-    named_bar_sync(1, 256);
-    const float mean = (red[r] + red[epi::TILE + r]) * (1.f / 128.f);
-    named_bar_sync(1, 256);
-    const float2 nm = make_float2(-mean, -mean);
-    a0 = a1 = a2 = a3 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-        const float2 d0 = __fadd2_rn(v[k], nm), d1 = __fadd2_rn(v[k + 1], nm);
-        const float2 d2 = __fadd2_rn(v[k + 2], nm), d3 = __fadd2_rn(v[k + 3], nm);
-        a0 = __ffma2_rn(d0, d0, a0);
-        a1 = __ffma2_rn(d1, d1, a1);
-        a2 = __ffma2_rn(d2, d2, a2);
-        a3 = __ffma2_rn(d3, d3, a3);
-    }
-    red[h * epi::TILE + r] = (a0.x + a0.y) + (a1.x + a1.y) + (a2.x + a2.y) + (a3.x + a3.y);
-    named_bar_sync(1, 256);  // also: every worker has read its x columns before any overwrites them
-    const float rstd = rsqrtf((red[r] + red[epi::TILE + r]) * (1.f / 128.f) + eps);
-    const float2 sc = make_float2(rstd, rstd), sh = make_float2(-mean * rstd, -mean * rstd);
-    uint8_t *rowp = xt + h * epi::T_HALF + r * 128;
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 y = __ffma2_rn(v[kc * 4 + e], sc, sh);
-            if (kAffine) {
-                const int c = h * 64 + kc * 8 + 2 * e;
-                const float2 g = gw ? ld_pair_bf16(gw, c) : make_float2(1.f, 1.f);
-                const float2 b = gb ? ld_pair_bf16(gb, c) : make_float2(0.f, 0.f);
-                y = __ffma2_rn(y, g, b);
-            }
-            w[e] = pack_bf16x2(y.x, y.y);
-        }
-        *reinterpret_cast<uint4 *>(rowp + ((kc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+// Row n of a 128 x 128 bf16 weight held as two 64-column halves of 128-byte
+// rows with the 128-byte swizzle: 16-byte chunk kc of half h sits at chunk
+// kc ^ (n & 7).
+__device__ __forceinline__ uint4 *w_chunk(uint8_t *w, int n, int h, int kc) {
+    return reinterpret_cast<uint4 *>(w + h * epi::W_HALF + n * 128 + ((kc ^ (n & 7)) << 4));
+}
+
+// Mean and rstd of 128 values, accumulated in fp32 around the first value
+// (which keeps E[d^2] - E[d]^2 well conditioned when |mean| >> std).
+struct RowStats {
+    float2 s, ss;
+    float k;
+};
+__device__ __forceinline__ void stats_add(RowStats &st, uint32_t w) {
+    const float2 d = __fadd2_rn(unpack_bf16x2(w), make_float2(-st.k, -st.k));
+    st.s = __fadd2_rn(st.s, d);
+    st.ss = __ffma2_rn(d, d, st.ss);
+}
+__device__ __forceinline__ float2 stats_finish(const RowStats &st, float eps) {
+    const float m = (st.s.x + st.s.y) * (1.f / 128.f);
+    const float var = fmaxf((st.ss.x + st.ss.y) * (1.f / 128.f) - m * m, 0.f);
+    return make_float2(st.k + m, rsqrtf(var + eps));
 }
 
 // kVec: some LayerNorm affine or output bias is present (general path).
@@ -118,18 +89,21 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *wg = smem;
     uint8_t *wo = wg + W_BYTES;
-    uint8_t *xs = wo + W_BYTES;        // [2] x tiles
-    uint8_t *zs = xs + 2 * T_BYTES;    // [2] z tiles
-    uint8_t *st = zs + 2 * T_BYTES;    // [8 warps][2] output staging
-    float *red = reinterpret_cast<float *>(st + WORKERS * ST_PER_WARP * ST_BYTES);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(red) + RED_BYTES);
-    uint64_t *wbar = bars;          // weights landed
-    uint64_t *full = bars + 1;      // [2] x and z tile landed
-    uint64_t *mma = bars + 3;       // [2] MMAs of the tile in buffer b done
-    uint64_t *ln_done = bars + 5;   // workers: tile normalised (8 arrivals)
-    uint64_t *acc_free = bars + 6;  // [2] workers: accumulator b read (8 arrivals)
-    uint64_t *drain = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+    uint8_t *xs = wo + W_BYTES;        // [2] x tiles: [2 cell blocks][128 ch][64 cells]
+    uint8_t *zs = xs + 2 * T_BYTES;    // [2] z tiles: [2 ch halves][128 cells][64 ch]
+    uint8_t *st = zs + 2 * T_BYTES;    // [8 warps] output staging
+    float *cst = reinterpret_cast<float *>(st + GATERS * ST_BYTES);  // s_g, s_o, t_g / 2, t_o / 2
+    float4 *stat = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(cst) + CST_BYTES);  // [2][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(stat) + STAT_BYTES);
+    uint64_t *wbar = bars;             // weights landed
+    uint64_t *full = bars + 1;         // [2] x and z tile landed
+    uint64_t *mma = bars + 3;          // [2] MMAs into accumulator b done
+    uint64_t *xzdone = bars + 5;       // [2] MMAs have read tile buffer b
+    uint64_t *stat_done = bars + 7;    // [2] statistics of the tile in buffer b written (4 arrivals)
+    uint64_t *stat_free = bars + 9;    // [2] gaters have read statistics slot b (8 arrivals)
+    uint64_t *acc_free = bars + 11;    // [2] gaters have read accumulator b (8 arrivals)
+    uint64_t *drain = bars + 13;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,14 +117,16 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&full[b], 1);
             mbar_init(&mma[b], 1);
-            mbar_init(&acc_free[b], WORKERS);
+            mbar_init(&xzdone[b], 1);
+            mbar_init(&stat_done[b], STATS);
+            mbar_init(&stat_free[b], GATERS);
+            mbar_init(&acc_free[b], GATERS);
         }
-        mbar_init(ln_done, WORKERS);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == WORKERS) {
+    if (warp == CTRL_WARP) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -165,64 +141,111 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
         j0 = (tile - i * args.jt_tiles) * TILE;
     };
 
-    if (warp == WORKERS) {
+    int last_load0 = -1, last_load1 = -1;  // control lane: latest tile loaded into each buffer
+    auto load_tile = [&](int lt) {
+        int i, j0;
+        tile_coords(lt, i, j0);
+        const int b = lt & 1;
+        if (b) last_load1 = lt; else last_load0 = lt;
+        mbar_arrive_expect_tx(&full[b], 2 * T_BYTES);
+        tma_load_3d(xs + b * T_BYTES, &tmX, &full[b], j0, i, 0);
+        tma_load_3d(xs + b * T_BYTES + T_HALF, &tmX, &full[b], j0 + 64, i, 0);
+        tma_load_3d(zs + b * T_BYTES, &tmZ, &full[b], 0, j0, i);
+        tma_load_3d(zs + b * T_BYTES + T_HALF, &tmZ, &full[b], 64, j0, i);
+    };
+    if (warp == CTRL_WARP && lane == 0) {
+        mbar_arrive_expect_tx(wbar, 2 * W_BYTES);
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+            tma_load_2d(wg + kh * W_HALF, &tmWg, wbar, kh * 64, 0);
+            tma_load_2d(wo + kh * W_HALF, &tmWo, wbar, kh * 64, 0);
+        }
+        if (n_local > 0) load_tile(0);
+        if (n_local > 1) load_tile(1);
+    }
+
+    // ---- weights: W' = W gamma in place, s = row sums of W', t = W beta + bias --------------
+    // Thread t < 256 owns row t % 128 of weight t / 128 (W_g, then W_o).
+    bool ok = warp_wait(wbar, 0, abort_flag, ctl, SITE_EPI | 1, 0);
+    if (ok && threadIdx.x < 256) {
+        const int w = threadIdx.x >> 7, n = threadIdx.x & 127;
+        uint8_t *W = w ? wo : wg;
+        const __nv_bfloat16 *gamma = w ? args.ln_out_w : args.ln_in_w;
+        const __nv_bfloat16 *beta = w ? args.ln_out_b : args.ln_in_b;
+        const __nv_bfloat16 *bias = w ? args.b_o : args.b_g;
+        float t = 0.f;
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h)
+#pragma unroll 1
+            for (int kc = 0; kc < 8; ++kc) {
+                uint4 *cp = w_chunk(W, n, h, kc);
+                const uint4 u = *cp;
+                uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int k = h * 64 + kc * 8 + 2 * e;
+                    float2 v = unpack_bf16x2(wd[e]);
+                    if (kVec) {
+                        if (beta) t = fmaf(v.x, __bfloat162float(beta[k]), fmaf(v.y, __bfloat162float(beta[k + 1]), t));
+                        if (gamma) {
+                            v = __fmul2_rn(v, make_float2(__bfloat162float(gamma[k]), __bfloat162float(gamma[k + 1])));
+                            wd[e] = pack_bf16x2(v.x, v.y);
+                            v = unpack_bf16x2(wd[e]);  // the rounded W' the MMA reads
+                        }
+                    }
+                    s2 = __fadd2_rn(s2, v);
+                }
+                if (kVec && gamma) *cp = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+        if (kVec && bias) t += __bfloat162float(bias[n]);
+        cst[w * 128 + n] = s2.x + s2.y;
+        cst[256 + w * 128 + n] = 0.5f * t;
+    }
+    fence_proxy_async_smem();  // W' written by threads is read by the tensor core
+    __syncthreads();
+    ok = ok && !*abort_flag;
+
+    if (warp == CTRL_WARP) {
         // ------------------------------ control warp ------------------------------
         if (lane == 0) {
-            int last_load0 = -1, last_load1 = -1;
-            auto load_tile = [&](int lt) {
-                int i, j0;
-                tile_coords(lt, i, j0);
-                const int b = lt & 1;
-                if (b) last_load1 = lt; else last_load0 = lt;
-                mbar_arrive_expect_tx(&full[b], 2 * T_BYTES);
-                tma_load_3d(xs + b * T_BYTES, &tmX, &full[b], j0, i, 0);
-                tma_load_3d(zs + b * T_BYTES, &tmZ, &full[b], 0, j0, i);
-                tma_load_3d(zs + b * T_BYTES + T_HALF, &tmZ, &full[b], 64, j0, i);
-            };
-            // G = zh W_g^T into columns [0,128), O = xh W_o^T into [128,256) of accumulator b.
+            // Accumulator b: G in columns [0, 128), O in [128, 256).
             auto issue_mma = [&](int b) {
-                const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
-                const uint32_t za = smem_u32(zs + b * T_BYTES), xa = smem_u32(xs + b * T_BYTES);
+                const uint32_t zb = smem_u32(zs + b * T_BYTES), xb = smem_u32(xs + b * T_BYTES);
                 const uint32_t gb = smem_u32(wg), ob = smem_u32(wo);
                 const uint32_t d = tmem_base + (uint32_t)(b * 256);
+                const uint32_t idesc_g = idesc_bf16(128, 128, 0, 0), idesc_o = idesc_bf16(128, 128, 1, 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * T_HALF + (kk & 3) * 32);
                     const uint32_t woff = (uint32_t)((kk >> 2) * W_HALF + (kk & 3) * 32);
-                    mma_bf16(d, sdesc_sw128(za + off, 16, 1024), sdesc_sw128(gb + woff, 16, 1024), idesc,
+                    mma_bf16(d, sdesc_sw128(zb + off, 16, 1024), sdesc_sw128(gb + woff, 16, 1024), idesc_g,
                              kk ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * T_HALF + (kk & 3) * 32);
+                    // x is MN-major: 16 channel rows of 128 B per K step, cell blocks T_HALF apart.
                     const uint32_t woff = (uint32_t)((kk >> 2) * W_HALF + (kk & 3) * 32);
-                    mma_bf16(d + 128, sdesc_sw128(xa + off, 16, 1024), sdesc_sw128(ob + woff, 16, 1024), idesc,
-                             kk ? 1u : 0u);
+                    mma_bf16(d + 128, sdesc_sw128(xb + (uint32_t)(kk * 2048), T_HALF, 1024),
+                             sdesc_sw128(ob + woff, 16, 1024), idesc_o, kk ? 1u : 0u);
                 }
             };
-            mbar_arrive_expect_tx(wbar, 2 * W_BYTES);
-#pragma unroll
-            for (int kh = 0; kh < 2; ++kh) {
-                tma_load_2d(wg + kh * W_HALF, &tmWg, wbar, kh * 64, 0);
-                tma_load_2d(wo + kh * W_HALF, &tmWo, wbar, kh * 64, 0);
-            }
-            if (n_local > 0) load_tile(0);
-            if (n_local > 1) load_tile(1);
-            bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_EPI | 1, 0);
             for (int lt = 0; ok && lt < n_local; ++lt) {
                 const int b = lt & 1;
-                if (!wait_bounded(ln_done, (uint32_t)lt & 1u, abort_flag, ctl, SITE_EPI | 2, lt) ||
-                    (lt >= 2 && !wait_bounded(&acc_free[b], (uint32_t)((lt - 2) >> 1) & 1u, abort_flag, ctl,
-                                              SITE_EPI | 3, lt))) {
+                const uint32_t par = (uint32_t)(lt >> 1) & 1u;
+                if (!wait_bounded(&full[b], par, abort_flag, ctl, SITE_EPI | 2, lt) ||
+                    (lt >= 2 && !wait_bounded(&acc_free[b], par ^ 1u, abort_flag, ctl, SITE_EPI | 3, lt))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 issue_mma(b);
                 mma_commit(&mma[b]);
+                mma_commit(&xzdone[b]);
                 if (lt + 2 < n_local) {
-                    // Buffers b are free once the MMAs of tile lt have read them.
-                    if (!wait_bounded(&mma[b], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_EPI | 4, lt)) {
+                    // Buffers b are free once the MMAs and the statistics of tile lt have read them.
+                    if (!wait_bounded(&xzdone[b], par, abort_flag, ctl, SITE_EPI | 4, lt) ||
+                        !wait_bounded(&stat_done[b], par, abort_flag, ctl, SITE_EPI | 5, lt)) {
                         ok = false;
                         break;
                     }
@@ -238,75 +261,98 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
             mma_commit(drain);
             wait_drain(drain, 0, ctl.timeout_ns);
         }
-    } else {
-        // ------------------------------ worker warps ------------------------------
-        const int q = warp & 3, sub = warp >> 2;
-        uint8_t *stw = st + warp * ST_PER_WARP * ST_BYTES;
-        int st_round = 0;
-        auto normalise = [&](int b) {
-            ln_tile_sw128<kVec>(zs + b * T_BYTES, T_HALF, args.ln_in_w, args.ln_in_b, args.eps);
-            epi_layer_norm_x<kVec>(xs + b * T_BYTES, red, args.ln_out_w, args.ln_out_b, args.eps);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ln_done);
-        };
-
-        // Every worker takes the LayerNorm barriers: before each normalisation the
-        // workers agree (bar.red.and) on whether to go on, so none can be left
-        // waiting at a barrier after another has stopped.
-        bool ok = warp_wait(&full[0], 0, abort_flag, ctl, SITE_EPI | 5, 0);
-        ok = bar_red_and(1, 32 * WORKERS, ok);
-        if (ok) normalise(0);
+    } else if (warp >= GATERS) {
+        // ------------------------------ statistics ------------------------------
+        const int cell = (warp - GATERS) * 32 + lane;
+        const int mb = cell >> 6, m = cell & 63;  // x: cell block and cell within it
         for (int lt = 0; ok && lt < n_local; ++lt) {
-            const int cur = lt & 1;
+            const int b = lt & 1;
+            const uint32_t par = (uint32_t)(lt >> 1) & 1u;
+            if (!(ok = warp_wait(&full[b], par, abort_flag, ctl, SITE_EPI | 6, lt))) break;
+            if (lt >= 2 && !(ok = warp_wait(&stat_free[b], par ^ 1u, abort_flag, ctl, SITE_EPI | 7, lt))) break;
+            // z: row `cell` of the two channel halves, 16-byte chunks.
+            const uint8_t *zr = zs + b * T_BYTES + cell * 128;
+            RowStats sz;
+            sz.s = sz.ss = make_float2(0.f, 0.f);
+            sz.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(zr + ((cell & 7) << 4)));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int kc = 0; kc < 8; ++kc) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(zr + h * T_HALF + ((kc ^ (cell & 7)) << 4));
+                    stats_add(sz, u.x);
+                    stats_add(sz, u.y);
+                    stats_add(sz, u.z);
+                    stats_add(sz, u.w);
+                }
+            // x: column `cell` (channel rows of 128 B, 128-byte swizzle), two channels per step.
+            const uint8_t *xc = xs + b * T_BYTES + mb * T_HALF + (m & 7) * 2;
+            RowStats sx;
+            sx.s = sx.ss = make_float2(0.f, 0.f);
+            sx.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xc + ((m >> 3) << 4)));
+#pragma unroll 8
+            for (int c = 0; c < 128; c += 2) {
+                const uint32_t lo = *reinterpret_cast<const uint16_t *>(xc + c * 128 + (((m >> 3) ^ (c & 7)) << 4));
+                const uint32_t hi =
+                    *reinterpret_cast<const uint16_t *>(xc + (c + 1) * 128 + (((m >> 3) ^ ((c + 1) & 7)) << 4));
+                stats_add(sx, lo | (hi << 16));
+            }
+            const float2 fz = stats_finish(sz, args.eps), fx = stats_finish(sx, args.eps);
+            stat[b * TILE + cell] = make_float4(-fz.x, 0.5f * fz.y, -fx.x, 0.5f * fx.y);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stat_done[b]);
+        }
+        if (!ok && lane == 0) *abort_flag = 1;
+    } else {
+        // ------------------------------ gaters ------------------------------
+        const int q = warp & 3, sub = warp >> 2;
+        uint8_t *sb = st + warp * ST_BYTES;
+        for (int lt = 0; ok && lt < n_local; ++lt) {
+            const int b = lt & 1;
+            const uint32_t par = (uint32_t)(lt >> 1) & 1u;
             int i, j0;
             tile_coords(lt, i, j0);
-            // Normalise tile lt+1 first, so its MMAs run while this tile is gated.
-            if (lt + 1 < n_local) {
-                bool got = warp_wait(&full[cur ^ 1], (uint32_t)((lt + 1) >> 1) & 1u, abort_flag, ctl, SITE_EPI | 6, lt);
-                if (!(ok = bar_red_and(1, 32 * WORKERS, got))) break;
-                normalise(cur ^ 1);
-            }
-            if (!warp_wait(&mma[cur], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_EPI | 7, lt)) {
-                // Leave the gating out but stay in step with the other workers' barriers.
-                ok = false;
-                if (lane == 0) *abort_flag = 1;
-                tc_fence_before();
-                if (lane == 0) mbar_arrive(&acc_free[cur]);
-                // Join the agreement the others take at the start of iteration lt + 1
-                // (there is one only if that iteration normalises tile lt + 2).
-                if (lt + 2 < n_local) bar_red_and(1, 32 * WORKERS, false);
-                break;
-            }
+            if (!(ok = warp_wait(&stat_done[b], par, abort_flag, ctl, SITE_EPI | 8, lt))) break;
+            // (-mu_z, r_z / 2, -mu_x, r_x / 2) of this thread's cell
+            const float4 cs = stat[b * TILE + 32 * q + lane];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stat_free[b]);
+            if (!(ok = warp_wait(&mma[b], par, abort_flag, ctl, SITE_EPI | 9, lt))) break;
             tc_fence_after();
             const bool live = j0 + 32 * q < args.N;
-            const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(cur * 256);
+            const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 256);
+            const float2 nmz = make_float2(cs.x, cs.x), hrz = make_float2(cs.y, cs.y);
+            const float2 nmx = make_float2(cs.z, cs.z), hrx = make_float2(cs.w, cs.w);
 #pragma unroll 1
             for (int hh = 0; live && hh < 2; ++hh) {
-                const int ch0 = hh * 64 + sub * 32;
+                const int ch0 = sub * 64 + hh * 32;
                 uint32_t G[32], O[32];
                 tmem_ld32(lane_base + (uint32_t)ch0, G);
                 tmem_ld32(lane_base + 128u + (uint32_t)ch0, O);
                 tmem_ld_wait();
-                // out = sigmoid(G + b_g) * (O + b_o) = (tanh((G + b_g) / 2) / 2 + 1/2) * (O + b_o)
+                // out = sigmoid(2 hg) * 2 ho = (tanh(hg) + 1) * ho with
+                // hg = r_z / 2 (G - mu_z s_g) + t_g / 2 and ho = r_x / 2 (O - mu_x s_o) + t_o / 2.
                 uint32_t p[16];
-                const float2 half = make_float2(0.5f, 0.5f);
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    float2 g = make_float2(__uint_as_float(G[2 * k]), __uint_as_float(G[2 * k + 1]));
-                    float2 o = make_float2(__uint_as_float(O[2 * k]), __uint_as_float(O[2 * k + 1]));
+                    const int n = ch0 + 2 * k;
+                    const float2 sg = *reinterpret_cast<const float2 *>(cst + n);
+                    const float2 so = *reinterpret_cast<const float2 *>(cst + 128 + n);
+                    const float2 g = make_float2(__uint_as_float(G[2 * k]), __uint_as_float(G[2 * k + 1]));
+                    const float2 o = make_float2(__uint_as_float(O[2 * k]), __uint_as_float(O[2 * k + 1]));
+                    float2 hg, ho;
                     if (kVec) {
-                        if (args.b_g) g = __fadd2_rn(g, ld_pair_bf16(args.b_g, ch0 + 2 * k));
-                        if (args.b_o) o = __fadd2_rn(o, ld_pair_bf16(args.b_o, ch0 + 2 * k));
+                        hg = __ffma2_rn(__ffma2_rn(nmz, sg, g), hrz, *reinterpret_cast<const float2 *>(cst + 256 + n));
+                        ho = __ffma2_rn(__ffma2_rn(nmx, so, o), hrx, *reinterpret_cast<const float2 *>(cst + 384 + n));
+                    } else {
+                        hg = __fmul2_rn(__ffma2_rn(nmz, sg, g), hrz);
+                        ho = __fmul2_rn(__ffma2_rn(nmx, so, o), hrx);
                     }
-                    const float2 hg = __fmul2_rn(g, half);
                     const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
-                    const float2 y = __fmul2_rn(__ffma2_rn(th, half, half), o);
+                    const float2 y = __ffma2_rn(th, ho, ho);
                     p[k] = pack_bf16x2(y.x, y.y);
                 }
-                uint8_t *sb = stw + (st_round & 1) * ST_BYTES;
-                ++st_round;
-                if (lane == 0) tma_store_wait_read<1>();
+                if (lane == 0) tma_store_wait_read<0>();  // the previous store has read the buffer
                 __syncwarp();
                 // [32 cells][32 ch]: 64-byte rows, 16-byte chunk c at c ^ ((cell >> 1) & 3).
 #pragma unroll
@@ -322,7 +368,7 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_free[cur]);
+            if (lane == 0) mbar_arrive(&acc_free[b]);
         }
         if (!ok && lane == 0) *abort_flag = 1;
         if (lane == 0) tma_store_wait_all<0>();
@@ -331,7 +377,7 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == WORKERS) tmem_dealloc(tmem_base, 512);
+    if (warp == CTRL_WARP) tmem_dealloc(tmem_base, 512);
 }
 
 size_t epilogue_tc_smem() { return epi::SMEM; }

@@ -60,7 +60,7 @@ struct EpilogueArgs {
 struct EpilogueMaps {
     CUtensorMap wg, wo;  // 2-D [128][128], box 64 x 128, swizzle 128B
     CUtensorMap z;       // as in the prologue
-    CUtensorMap x;       // 3-D (j, i, c) over x, box (128, 1, 128), no swizzle
+    CUtensorMap x;       // 3-D (j, i, c) over x, box (64, 1, 128), swizzle 128B
     CUtensorMap out;     // 3-D (c, j, i) over out, box (32, 32, 1), swizzle 64B
 };
 
