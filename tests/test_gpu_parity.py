@@ -111,6 +111,28 @@ def test_bf16_epilogue_stage(N):
     assert max_abs(got, ref) <= BF16_ABS
 
 
+@pytest.mark.parametrize("offset", [8.0, -30.0])
+def test_bf16_epilogue_stage_large_mean(offset):
+    """Cells whose mean is far from zero relative to their spread, in z and in x:
+    the folded LayerNorms subtract mean * rowsum(W') after the MMA, which must
+    cancel as the normalised inputs would."""
+    N = 200
+    case = pi.random_case(N, 77, bf16=True, affine=True, mask="random")
+    case["z"] = as_bf16(case["z"] + offset)
+    a, b = oracle.project(case)
+    x = as_bf16(oracle.contract(a, b, "incoming") * 0.5 + offset)
+    dc = DeviceCase(case, "bf16")
+    _, _, vx = dc.views()
+    vx[:, :, :N] = torch.from_numpy(x.transpose(2, 0, 1).copy()).to(vx.device).to(torch.bfloat16)
+    tm.trimul_epilogue(dc.z, dc.p, dc.out)
+    torch.cuda.synchronize()
+    assert tm.trimul_device_status(dc.p)[0] == 0
+    got = dc.out.float().cpu().numpy()
+    ref = oracle.finish(case, x)
+    assert rel_l2(got, ref) <= BF16_REL
+    assert max_abs(got, ref) <= BF16_ABS
+
+
 # ---------------------------------------------------------------- bf16 layer
 
 @pytest.mark.parametrize("direction", ["outgoing", "incoming"])
