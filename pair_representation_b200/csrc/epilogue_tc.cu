@@ -19,13 +19,14 @@
 // for a LayerNorm. s is summed from the same bf16 W' the MMA reads, so the
 // mean term cancels as it would in exact arithmetic.
 //
-// Tiles are 128 consecutive cells of one residue row. Roles (416 threads):
+// Tiles are 128 consecutive cells of one residue row. Roles (544 threads):
 //   all, once: W' = W gamma in shared memory, s and t per output channel.
-//   warp 12 (control): TMA loads of the x and z tiles two tiles ahead; per tile
+//   warp 16 (control): TMA loads of the x and z tiles two tiles ahead; per tile
 //     G = z W_g'^T and O = x W_o'^T (M = 128 cells, N = 128, K = 128) into a
 //     double-buffered 256-column TMEM accumulator.
-//   warps 8-11 (statistics): mean and rstd of z and of x for each cell of a
-//     landed tile (one thread per cell), into a two-slot table.
+//   warps 8-15 (statistics): mean and rstd of z and of x for each cell of a
+//     landed tile (two threads per cell, one per channel half), into a
+//     two-slot table.
 //   warps 0-7 (gaters): warp w reads TMEM lanes 32(w % 4).. (its 32 cells) and
 //     channels 64(w / 4)..+63 of G and O, forms
 //     sigmoid(r_z (G - mu_z s_g) + t_g) * (r_x (O - mu_x s_o) + t_o) in packed
@@ -38,7 +39,7 @@ namespace trimul {
 namespace epi {
 constexpr int TILE = 128;
 constexpr int GATERS = 8;
-constexpr int STATS = 4;
+constexpr int STATS = 8;
 constexpr int CTRL_WARP = GATERS + STATS;
 constexpr int THREADS = 32 * (CTRL_WARP + 1);
 constexpr int W_HALF = 128 * 128;          // one 64-channel K half of a 128 x 128 weight: 16 KB
@@ -62,7 +63,8 @@ __device__ __forceinline__ uint4 *w_chunk(uint8_t *w, int n, int h, int kc) {
 }
 
 // Mean and rstd of 128 values, accumulated in fp32 around the first value
-// (which keeps E[d^2] - E[d]^2 well conditioned when |mean| >> std).
+// (which keeps E[d^2] - E[d]^2 well conditioned when |mean| >> std). Each of
+// two partner lanes (lane ^ 1) accumulates one channel half.
 struct RowStats {
     float2 s, ss;
     float k;
@@ -73,8 +75,11 @@ __device__ __forceinline__ void stats_add(RowStats &st, uint32_t w) {
     st.ss = __ffma2_rn(d, d, st.ss);
 }
 __device__ __forceinline__ float2 stats_finish(const RowStats &st, float eps) {
-    const float m = (st.s.x + st.s.y) * (1.f / 128.f);
-    const float var = fmaxf((st.ss.x + st.ss.y) * (1.f / 128.f) - m * m, 0.f);
+    float s = st.s.x + st.s.y, ss = st.ss.x + st.ss.y;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const float m = s * (1.f / 128.f);
+    const float var = fmaxf(ss * (1.f / 128.f) - m * m, 0.f);
     return make_float2(st.k + m, rsqrtf(var + eps));
 }
 
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
     uint64_t *full = bars + 1;         // [2] x and z tile landed
     uint64_t *mma = bars + 3;          // [2] MMAs into accumulator b done
     uint64_t *xzdone = bars + 5;       // [2] MMAs have read tile buffer b
-    uint64_t *stat_done = bars + 7;    // [2] statistics of the tile in buffer b written (4 arrivals)
+    uint64_t *stat_done = bars + 7;    // [2] statistics of the tile in buffer b written (8 arrivals)
     uint64_t *stat_free = bars + 9;    // [2] gaters have read statistics slot b (8 arrivals)
     uint64_t *acc_free = bars + 11;    // [2] gaters have read accumulator b (8 arrivals)
     uint64_t *drain = bars + 13;
@@ -263,42 +268,42 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
         }
     } else if (warp >= GATERS) {
         // ------------------------------ statistics ------------------------------
-        const int cell = (warp - GATERS) * 32 + lane;
+        const int t = (warp - GATERS) * 32 + lane;
+        const int cell = t >> 1, h = t & 1;       // channel half h of this cell
         const int mb = cell >> 6, m = cell & 63;  // x: cell block and cell within it
         for (int lt = 0; ok && lt < n_local; ++lt) {
             const int b = lt & 1;
             const uint32_t par = (uint32_t)(lt >> 1) & 1u;
             if (!(ok = warp_wait(&full[b], par, abort_flag, ctl, SITE_EPI | 6, lt))) break;
             if (lt >= 2 && !(ok = warp_wait(&stat_free[b], par ^ 1u, abort_flag, ctl, SITE_EPI | 7, lt))) break;
-            // z: row `cell` of the two channel halves, 16-byte chunks.
+            // z: channel half h of row `cell`, 16-byte chunks; shift = channel 0.
             const uint8_t *zr = zs + b * T_BYTES + cell * 128;
             RowStats sz;
             sz.s = sz.ss = make_float2(0.f, 0.f);
             sz.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(zr + ((cell & 7) << 4)));
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int kc = 0; kc < 8; ++kc) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(zr + h * T_HALF + ((kc ^ (cell & 7)) << 4));
-                    stats_add(sz, u.x);
-                    stats_add(sz, u.y);
-                    stats_add(sz, u.z);
-                    stats_add(sz, u.w);
-                }
-            // x: column `cell` (channel rows of 128 B, 128-byte swizzle), two channels per step.
+            for (int kc = 0; kc < 8; ++kc) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(zr + h * T_HALF + ((kc ^ (cell & 7)) << 4));
+                stats_add(sz, u.x);
+                stats_add(sz, u.y);
+                stats_add(sz, u.z);
+                stats_add(sz, u.w);
+            }
+            // x: channels 64h .. 64h + 63 of column `cell` (channel rows of 128 B, 128-byte
+            // swizzle), two channels per step; shift = channel 0.
             const uint8_t *xc = xs + b * T_BYTES + mb * T_HALF + (m & 7) * 2;
             RowStats sx;
             sx.s = sx.ss = make_float2(0.f, 0.f);
             sx.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xc + ((m >> 3) << 4)));
 #pragma unroll 8
-            for (int c = 0; c < 128; c += 2) {
+            for (int c = 64 * h; c < 64 * h + 64; c += 2) {
                 const uint32_t lo = *reinterpret_cast<const uint16_t *>(xc + c * 128 + (((m >> 3) ^ (c & 7)) << 4));
                 const uint32_t hi =
                     *reinterpret_cast<const uint16_t *>(xc + (c + 1) * 128 + (((m >> 3) ^ ((c + 1) & 7)) << 4));
                 stats_add(sx, lo | (hi << 16));
             }
             const float2 fz = stats_finish(sz, args.eps), fx = stats_finish(sx, args.eps);
-            stat[b * TILE + cell] = make_float4(-fz.x, 0.5f * fz.y, -fx.x, 0.5f * fx.y);
+            if (h == 0) stat[b * TILE + cell] = make_float4(-fz.x, 0.5f * fz.y, -fx.x, 0.5f * fx.y);
             __syncwarp();
             if (lane == 0) mbar_arrive(&stat_done[b]);
         }
@@ -326,31 +331,34 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
 #pragma unroll 1
             for (int hh = 0; live && hh < 2; ++hh) {
                 const int ch0 = sub * 64 + hh * 32;
-                uint32_t G[32], O[32];
-                tmem_ld32(lane_base + (uint32_t)ch0, G);
-                tmem_ld32(lane_base + 128u + (uint32_t)ch0, O);
-                tmem_ld_wait();
                 // out = sigmoid(2 hg) * 2 ho = (tanh(hg) + 1) * ho with
                 // hg = r_z / 2 (G - mu_z s_g) + t_g / 2 and ho = r_x / 2 (O - mu_x s_o) + t_o / 2.
                 uint32_t p[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int n = ch0 + 2 * k;
-                    const float2 sg = *reinterpret_cast<const float2 *>(cst + n);
-                    const float2 so = *reinterpret_cast<const float2 *>(cst + 128 + n);
-                    const float2 g = make_float2(__uint_as_float(G[2 * k]), __uint_as_float(G[2 * k + 1]));
-                    const float2 o = make_float2(__uint_as_float(O[2 * k]), __uint_as_float(O[2 * k + 1]));
-                    float2 hg, ho;
-                    if (kVec) {
-                        hg = __ffma2_rn(__ffma2_rn(nmz, sg, g), hrz, *reinterpret_cast<const float2 *>(cst + 256 + n));
-                        ho = __ffma2_rn(__ffma2_rn(nmx, so, o), hrx, *reinterpret_cast<const float2 *>(cst + 384 + n));
-                    } else {
-                        hg = __fmul2_rn(__ffma2_rn(nmz, sg, g), hrz);
-                        ho = __fmul2_rn(__ffma2_rn(nmx, so, o), hrx);
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t G[16], O[16];
+                    tmem_ld16(lane_base + (uint32_t)(ch0 + 16 * hc), G);
+                    tmem_ld16(lane_base + 128u + (uint32_t)(ch0 + 16 * hc), O);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int k = 8 * hc + kk, n = ch0 + 2 * k;
+                        const float2 sg = *reinterpret_cast<const float2 *>(cst + n);
+                        const float2 so = *reinterpret_cast<const float2 *>(cst + 128 + n);
+                        const float2 g = make_float2(__uint_as_float(G[2 * kk]), __uint_as_float(G[2 * kk + 1]));
+                        const float2 o = make_float2(__uint_as_float(O[2 * kk]), __uint_as_float(O[2 * kk + 1]));
+                        float2 hg, ho;
+                        if (kVec) {
+                            hg = __ffma2_rn(__ffma2_rn(nmz, sg, g), hrz, *reinterpret_cast<const float2 *>(cst + 256 + n));
+                            ho = __ffma2_rn(__ffma2_rn(nmx, so, o), hrx, *reinterpret_cast<const float2 *>(cst + 384 + n));
+                        } else {
+                            hg = __fmul2_rn(__ffma2_rn(nmz, sg, g), hrz);
+                            ho = __fmul2_rn(__ffma2_rn(nmx, so, o), hrx);
+                        }
+                        const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
+                        const float2 y = __ffma2_rn(th, ho, ho);
+                        p[k] = pack_bf16x2(y.x, y.y);
                     }
-                    const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
-                    const float2 y = __ffma2_rn(th, ho, ho);
-                    p[k] = pack_bf16x2(y.x, y.y);
                 }
                 if (lane == 0) tma_store_wait_read<0>();  // the previous store has read the buffer
                 __syncwarp();
