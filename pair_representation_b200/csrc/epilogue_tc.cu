@@ -25,8 +25,9 @@
 //     G = z W_g'^T and O = x W_o'^T (M = 128 cells, N = 128, K = 128) into a
 //     double-buffered 256-column TMEM accumulator.
 //   warps 8-15 (statistics): mean and rstd of z and of x for each cell of a
-//     landed tile (two threads per cell, one per channel half), into a
-//     two-slot table.
+//     landed tile, into a two-slot table: z by two threads per cell (one per
+//     channel half), x by four threads per pair of adjacent cells (one per
+//     channel quarter, 4-byte loads).
 //   warps 0-7 (gaters): warp w reads TMEM lanes 32(w % 4).. (its 32 cells) and
 //     channels 64(w / 4)..+63 of G and O, forms
 //     sigmoid(r_z (G - mu_z s_g) + t_g) * (r_x (O - mu_x s_o) + t_o) in packed
@@ -47,8 +48,8 @@ constexpr int W_BYTES = 2 * W_HALF;        // 32 KB per weight
 constexpr int T_HALF = TILE * 128;         // 16 KB
 constexpr int T_BYTES = 2 * T_HALF;        // 32 KB per tile buffer (x or z)
 constexpr int ST_BYTES = 32 * 32 * 2;      // 2 KB per warp buffer: [32 cells][32 ch], 64-byte swizzle
-constexpr int CST_BYTES = 4 * 128 * 4;     // s_g, s_o, t_g / 2, t_o / 2
-constexpr int STAT_BYTES = 2 * TILE * 16;  // two slots of (-mu_z, r_z / 2, -mu_x, r_x / 2) per cell
+constexpr int CST_BYTES = 4 * 128 * 4;     // per channel pair: (s_g, s_g, s_o, s_o), (t_g, t_g, t_o, t_o) / 2
+constexpr int STAT_BYTES = 2 * TILE * 16;  // two slots of (-mu_z, r_z / 2) and (-mu_x, r_x / 2) per cell
 constexpr int BAR_BYTES = 128;
 constexpr size_t SMEM = 1024 + 2 * (size_t)W_BYTES + 2 * 2 * (size_t)T_BYTES + (size_t)GATERS * ST_BYTES +
                         CST_BYTES + STAT_BYTES + BAR_BYTES;
@@ -97,9 +98,12 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
     uint8_t *xs = wo + W_BYTES;        // [2] x tiles: [2 cell blocks][128 ch][64 cells]
     uint8_t *zs = xs + 2 * T_BYTES;    // [2] z tiles: [2 ch halves][128 cells][64 ch]
     uint8_t *st = zs + 2 * T_BYTES;    // [8 warps] output staging
-    float *cst = reinterpret_cast<float *>(st + GATERS * ST_BYTES);  // s_g, s_o, t_g / 2, t_o / 2
-    float4 *stat = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(cst) + CST_BYTES);  // [2][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(stat) + STAT_BYTES);
+    // cs4[p] = (s_g[2p], s_g[2p+1], s_o[2p], s_o[2p+1]); ct4[p] = (t_g[2p], t_g[2p+1], t_o[2p], t_o[2p+1]) / 2
+    float4 *cs4 = reinterpret_cast<float4 *>(st + GATERS * ST_BYTES);
+    float4 *ct4 = cs4 + 64;
+    float2 *statz = reinterpret_cast<float2 *>(cs4 + 128);  // [2][128] (-mu_z, r_z / 2)
+    float2 *statx = statz + 2 * TILE;                        // [2][128] (-mu_x, r_x / 2)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(statx + 2 * TILE);
     uint64_t *wbar = bars;             // weights landed
     uint64_t *full = bars + 1;         // [2] x and z tile landed
     uint64_t *mma = bars + 3;          // [2] MMAs into accumulator b done
@@ -204,8 +208,8 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
                 if (kVec && gamma) *cp = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
         if (kVec && bias) t += __bfloat162float(bias[n]);
-        cst[w * 128 + n] = s2.x + s2.y;
-        cst[256 + w * 128 + n] = 0.5f * t;
+        reinterpret_cast<float *>(cs4)[(n >> 1) * 4 + 2 * w + (n & 1)] = s2.x + s2.y;
+        reinterpret_cast<float *>(ct4)[(n >> 1) * 4 + 2 * w + (n & 1)] = 0.5f * t;
     }
     fence_proxy_async_smem();  // W' written by threads is read by the tensor core
     __syncthreads();
@@ -268,42 +272,58 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
         }
     } else if (warp >= GATERS) {
         // ------------------------------ statistics ------------------------------
+        // z: thread (cell, h) reads channel half h of its cell's row. x: thread (pair, quarter)
+        // reads channels 32 quarter .. + 31 of the two adjacent cells 2 pair, 2 pair + 1 with
+        // 4-byte loads; the four quarters of a pair are lanes 4k .. 4k + 3, visiting their
+        // channels in an order staggered by 2 per quarter so that one warp load touches 8
+        // distinct 16-byte chunks (no bank conflicts).
         const int t = (warp - GATERS) * 32 + lane;
-        const int cell = t >> 1, h = t & 1;       // channel half h of this cell
-        const int mb = cell >> 6, m = cell & 63;  // x: cell block and cell within it
+        const int zcell = t >> 1, zh = t & 1;
+        const int pr = t >> 2, quarter = t & 3;
+        const int xcell = 2 * pr, mb = xcell >> 6, m = xcell & 63;
         for (int lt = 0; ok && lt < n_local; ++lt) {
             const int b = lt & 1;
             const uint32_t par = (uint32_t)(lt >> 1) & 1u;
             if (!(ok = warp_wait(&full[b], par, abort_flag, ctl, SITE_EPI | 6, lt))) break;
             if (lt >= 2 && !(ok = warp_wait(&stat_free[b], par ^ 1u, abort_flag, ctl, SITE_EPI | 7, lt))) break;
-            // z: channel half h of row `cell`, 16-byte chunks; shift = channel 0.
-            const uint8_t *zr = zs + b * T_BYTES + cell * 128;
+            const uint8_t *zr = zs + b * T_BYTES + zcell * 128;
             RowStats sz;
             sz.s = sz.ss = make_float2(0.f, 0.f);
-            sz.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(zr + ((cell & 7) << 4)));
+            sz.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(zr + ((zcell & 7) << 4)));
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(zr + h * T_HALF + ((kc ^ (cell & 7)) << 4));
+                const uint4 u = *reinterpret_cast<const uint4 *>(zr + zh * T_HALF + ((kc ^ (zcell & 7)) << 4));
                 stats_add(sz, u.x);
                 stats_add(sz, u.y);
                 stats_add(sz, u.z);
                 stats_add(sz, u.w);
             }
-            // x: channels 64h .. 64h + 63 of column `cell` (channel rows of 128 B, 128-byte
-            // swizzle), two channels per step; shift = channel 0.
             const uint8_t *xc = xs + b * T_BYTES + mb * T_HALF + (m & 7) * 2;
-            RowStats sx;
-            sx.s = sx.ss = make_float2(0.f, 0.f);
-            sx.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(xc + ((m >> 3) << 4)));
+            const float2 kx = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(xc + ((m >> 3) << 4)));
+            float2 xs1 = make_float2(0.f, 0.f), xs2 = xs1;  // per cell: sum of d, sum of d^2
 #pragma unroll 8
-            for (int c = 64 * h; c < 64 * h + 64; c += 2) {
-                const uint32_t lo = *reinterpret_cast<const uint16_t *>(xc + c * 128 + (((m >> 3) ^ (c & 7)) << 4));
-                const uint32_t hi =
-                    *reinterpret_cast<const uint16_t *>(xc + (c + 1) * 128 + (((m >> 3) ^ ((c + 1) & 7)) << 4));
-                stats_add(sx, lo | (hi << 16));
+            for (int it = 0; it < 32; ++it) {
+                const int c = 32 * quarter + ((it + 2 * quarter) & 31);
+                const uint32_t w2 = *reinterpret_cast<const uint32_t *>(xc + c * 128 + (((m >> 3) ^ (c & 7)) << 4));
+                const float2 d = __fadd2_rn(unpack_bf16x2(w2), make_float2(-kx.x, -kx.y));
+                xs1 = __fadd2_rn(xs1, d);
+                xs2 = __ffma2_rn(d, d, xs2);
             }
-            const float2 fz = stats_finish(sz, args.eps), fx = stats_finish(sx, args.eps);
-            if (h == 0) stat[b * TILE + cell] = make_float4(-fz.x, 0.5f * fz.y, -fx.x, 0.5f * fx.y);
+#pragma unroll
+            for (int o = 1; o <= 2; o <<= 1) {
+                xs1.x += __shfl_xor_sync(0xffffffffu, xs1.x, o);
+                xs1.y += __shfl_xor_sync(0xffffffffu, xs1.y, o);
+                xs2.x += __shfl_xor_sync(0xffffffffu, xs2.x, o);
+                xs2.y += __shfl_xor_sync(0xffffffffu, xs2.y, o);
+            }
+            const float2 fz = stats_finish(sz, args.eps);
+            if (zh == 0) statz[b * TILE + zcell] = make_float2(-fz.x, 0.5f * fz.y);
+            if (quarter == 0) {
+                const float2 mx = __fmul2_rn(xs1, make_float2(1.f / 128.f, 1.f / 128.f));
+                const float2 vx = __ffma2_rn(xs2, make_float2(1.f / 128.f, 1.f / 128.f), __fmul2_rn(mx, make_float2(-mx.x, -mx.y)));
+                statx[b * TILE + xcell] = make_float2(-(kx.x + mx.x), 0.5f * rsqrtf(fmaxf(vx.x, 0.f) + args.eps));
+                statx[b * TILE + xcell + 1] = make_float2(-(kx.y + mx.y), 0.5f * rsqrtf(fmaxf(vx.y, 0.f) + args.eps));
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&stat_done[b]);
         }
@@ -318,16 +338,16 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
             int i, j0;
             tile_coords(lt, i, j0);
             if (!(ok = warp_wait(&stat_done[b], par, abort_flag, ctl, SITE_EPI | 8, lt))) break;
-            // (-mu_z, r_z / 2, -mu_x, r_x / 2) of this thread's cell
-            const float4 cs = stat[b * TILE + 32 * q + lane];
+            // (-mu_z, r_z / 2) and (-mu_x, r_x / 2) of this thread's cell
+            const float2 cz = statz[b * TILE + 32 * q + lane], cx = statx[b * TILE + 32 * q + lane];
             __syncwarp();
             if (lane == 0) mbar_arrive(&stat_free[b]);
             if (!(ok = warp_wait(&mma[b], par, abort_flag, ctl, SITE_EPI | 9, lt))) break;
             tc_fence_after();
             const bool live = j0 + 32 * q < args.N;
             const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 256);
-            const float2 nmz = make_float2(cs.x, cs.x), hrz = make_float2(cs.y, cs.y);
-            const float2 nmx = make_float2(cs.z, cs.z), hrx = make_float2(cs.w, cs.w);
+            const float2 nmz = make_float2(cz.x, cz.x), hrz = make_float2(cz.y, cz.y);
+            const float2 nmx = make_float2(cx.x, cx.x), hrx = make_float2(cx.y, cx.y);
 #pragma unroll 1
             for (int hh = 0; live && hh < 2; ++hh) {
                 const int ch0 = sub * 64 + hh * 32;
@@ -343,14 +363,15 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const int k = 8 * hc + kk, n = ch0 + 2 * k;
-                        const float2 sg = *reinterpret_cast<const float2 *>(cst + n);
-                        const float2 so = *reinterpret_cast<const float2 *>(cst + 128 + n);
+                        const float4 s4 = cs4[n >> 1];
+                        const float2 sg = make_float2(s4.x, s4.y), so = make_float2(s4.z, s4.w);
                         const float2 g = make_float2(__uint_as_float(G[2 * kk]), __uint_as_float(G[2 * kk + 1]));
                         const float2 o = make_float2(__uint_as_float(O[2 * kk]), __uint_as_float(O[2 * kk + 1]));
                         float2 hg, ho;
                         if (kVec) {
-                            hg = __ffma2_rn(__ffma2_rn(nmz, sg, g), hrz, *reinterpret_cast<const float2 *>(cst + 256 + n));
-                            ho = __ffma2_rn(__ffma2_rn(nmx, so, o), hrx, *reinterpret_cast<const float2 *>(cst + 384 + n));
+                            const float4 t4 = ct4[n >> 1];
+                            hg = __ffma2_rn(__ffma2_rn(nmz, sg, g), hrz, make_float2(t4.x, t4.y));
+                            ho = __ffma2_rn(__ffma2_rn(nmx, so, o), hrx, make_float2(t4.z, t4.w));
                         } else {
                             hg = __fmul2_rn(__ffma2_rn(nmz, sg, g), hrz);
                             ho = __fmul2_rn(__ffma2_rn(nmx, so, o), hrx);
