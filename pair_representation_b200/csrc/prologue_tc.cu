@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     uint64_t *b_free = bars + 6;  // workers: b-half TMEM columns read (8 arrivals)
     uint64_t *drain = bars + 7;
     uint64_t *ln_done = bars + 8; // [2] normalisers: tile in z buffer b normalised (4 arrivals)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    uint64_t *wprep = bars + 10;  // workers: gate weights halved (8 arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         mbar_init(a_free, WORKERS);
         mbar_init(b_free, WORKERS);
         mbar_init(drain, 1);
+        mbar_init(wprep, WORKERS);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                 for (int kh = 0; kh < 2; ++kh) tma_load_2d(wsm + kh * W_HALF + w * 128 * 128, wm[w], wbar, kh * 64, 0);
             if (n_local > 0) load_z(0);
             if (n_local > 1) load_z(1);
-            bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0);
+            bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0) &&
+                      wait_bounded(wprep, 0, abort_flag, ctl, SITE_PRO | 10, 0);
             for (int lt = 0; ok && lt < n_local; ++lt) {
                 const uint32_t par = (uint32_t)lt & 1u, ppar = (uint32_t)(lt - 1) & 1u;
                 if (!wait_bounded(&ln_done[lt & 1], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 2, lt) ||
@@ -233,15 +236,15 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                     for (int e = 0; e < 2; ++e) {
                         float2 g = make_float2(__uint_as_float(G[4 * k + 2 * e]), __uint_as_float(G[4 * k + 2 * e + 1]));
                         float2 v = make_float2(__uint_as_float(V[4 * k + 2 * e]), __uint_as_float(V[4 * k + 2 * e + 1]));
+                        // g holds (W_g zh) / 2: the gate weights were halved in shared memory.
                         if (kVec) {
                             const int c = ch0 + 8 * k + 2 * (lane & 3);
-                            if (bg) g = __fadd2_rn(g, ld_pair_bf16(bg, c));
+                            if (bg) g = __ffma2_rn(ld_pair_bf16(bg, c), make_float2(0.5f, 0.5f), g);
                             if (bv) v = __fadd2_rn(v, ld_pair_bf16(bv, c));
                         }
                         const float h2 = hm[hf * 2 + e];
                         const float2 hh2 = make_float2(h2, h2);
-                        const float2 hg = __fmul2_rn(g, make_float2(0.5f, 0.5f));
-                        const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
+                        const float2 th = make_float2(tanh_approx(g.x), tanh_approx(g.y));
                         const float2 y = __fmul2_rn(__ffma2_rn(th, hh2, hh2), v);
                         P[hf * 8 + k * 2 + e] = pack_bf16x2(y.x, y.y);
                     }
@@ -287,7 +290,29 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             }
         };
 
-        bool ok = true;
+        // Halve W_ag and W_bg in place (exact in bf16): the MMAs then yield g / 2 for the tanh.
+        bool ok = warp_wait(wbar, 0, abort_flag, ctl, SITE_PRO | 11, 0);
+        if (ok) {
+#pragma unroll 1
+            for (int k = warp * 32 + lane; k < 4 * 1024; k += WORKERS * 32) {  // 4 regions x 1024 uint4
+                const int region = k >> 10;  // (K half, weight) = (0, ag), (0, bg), (1, ag), (1, bg)
+                uint4 *w4 = reinterpret_cast<uint4 *>(wsm + (region >> 1) * W_HALF + (1 + 2 * (region & 1)) * 128 * 128) +
+                            (k & 1023);
+                uint4 u = *w4;
+                const __nv_bfloat162 h = __float2bfloat162_rn(0.5f);
+                uint32_t *pw = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&pw[e]);
+                    x = __hmul2(x, h);
+                    pw[e] = *reinterpret_cast<uint32_t *>(&x);
+                }
+                *w4 = u;
+            }
+            fence_proxy_async_smem();  // read by the tensor core
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wprep);
         for (int lt = 0; ok && lt < n_local; ++lt) {
             int i, j0;
             tile_coords(lt, i, j0);
