@@ -191,6 +191,56 @@ def calibrated_oracle(workload, budget_s: float, threads=None):
 
 # ---------------------------------------------------------------- GPU arm
 
+def per_config_timings(tm, pi, torch, dev, stream, warmup=3, reps=5):
+    """Secondary figures: every workload and each direction separately, one
+    trimul_forward call per timing (CUDA events), L2 flushed before each call
+    (median and best), plus the median with a warm L2 (calls back to back)."""
+    res = {}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for wid, w in sorted(pi.WORKLOADS.items()):
+        case = pi.make_workload(w)
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        z = torch.from_numpy(case["z"]).to(dev).to(tdt)
+        mask = torch.from_numpy(case["mask"]).to(dev).to(tdt)
+        del case["z"]
+        out = torch.empty_like(z)
+        entry = {"N": w.N, "dtype": w.dtype}
+        for d in w.directions:
+            cls = tm.TriangleMultiplicationOutgoing if d == "outgoing" else tm.TriangleMultiplicationIncoming
+            sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+            layer = cls(128, 128).load_state_dict(sd).to(dev, tdt)
+            for _ in range(warmup):
+                layer(z, mask, out=out, stream=stream)
+            cold, warm = [], []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer(z, mask, out=out, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                cold.append(e0.elapsed_time(e1) * 1e3)
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                layer(z, mask, out=out, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                warm.append(e0.elapsed_time(e1) * 1e3)
+            cold.sort()
+            warm.sort()
+            med = cold[len(cold) // 2]
+            entry[d] = {"median_us": round(med, 1), "best_us": round(cold[0], 1),
+                        "warm_l2_median_us": round(warm[len(warm) // 2], 1),
+                        "pair_cells_per_s": round(w.N * w.N / (med * 1e-6)),
+                        "tflops": round(w.N * w.N * flops_per_cell(w.N) / (med * 1e-6) / 1e12, 1)}
+            del layer
+        res[w.name] = entry
+        del z, mask, out
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -350,6 +400,10 @@ def run_ours(args, rank, world, local_rank):
     value = pair_cells_per_s(world, args.steps, len(dirs), N, total_ms)
     tflops = world * args.steps * len(dirs) * N * N * flops_per_cell(N) / (total_ms / 1e3) / 1e12
     clocks = sampler.summary()
+    configs = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        del flush
+        configs = per_config_timings(tm, pi, torch, dev, stream)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -365,6 +419,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": sum(launches.values()),
         "clocks": clocks,
+        "per_config": configs,
     }
     if dist:
         dist.barrier()
@@ -414,6 +469,7 @@ def main(argv=None):
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=(1, 2, 3, 4, 5))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload secondary timings")
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=120.0)
     args = ap.parse_args(argv)
