@@ -157,6 +157,50 @@ const char *trimul_last_error_detail(void);
 int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params *p, int direction,
                            void *out, trimul_stream_t stream);
 
+/* ---- Backward -------------------------------------------------------------
+ * Gradients of a loss L through one forward call. Given dout = dL/dout
+ * ([N][N][c_z], dtype of z), trimul_backward writes dz = dL/dz ([N][N][c_z],
+ * dtype of z) and, into the fp32 buffers of trimul_grads, dL/d(each weight,
+ * bias and LayerNorm affine), overwriting them. The mask is an input and gets
+ * no gradient. A parameter that trimul_params leaves NULL (bias 0, gamma 1,
+ * beta 0) still gets its gradient when its output pointer is set; a NULL output
+ * pointer skips that gradient.
+ *
+ * The forward intermediates are recomputed: the call enqueues the prologue and
+ * the contraction into p->workspace, then the backward steps, which keep their
+ * intermediates (bf16, with fp32 for the LayerNorm adjoints' inputs) in
+ * g->workspace. The plain GEMMs of the backward (projections, weight
+ * gradients and the contraction's adjoint, per channel dA_c = dX_c B_c and
+ * dB_c = dX_c^T A_c outgoing, dA_c = B_c dX_c^T and dB_c = A_c dX_c incoming)
+ * run on cuBLAS with fp32 accumulation; the LayerNorm, gate and mask adjoints
+ * run in the library's kernels. Weight gradients are summed per chunk of 4096
+ * cells by GEMM and over the chunks in double by the library, so they do not
+ * depend on how cuBLAS splits a reduction over N^2 cells; bias and LayerNorm
+ * gradients are fp32 sums (atomic, so their last bits may vary between runs).
+ * cuBLAS (libcublas.so.12) is loaded on first use; one handle per device, given
+ * a slice of g->workspace as its workspace, is shared by all calls under a lock.
+ *
+ * BF16 only in this version (TRIMUL_ERR_UNSUPPORTED for F32). dout and dz
+ * must be 16-byte aligned and must not overlap each other, z, the mask or
+ * either workspace. Asynchronous. */
+typedef struct {
+    float *d_w_a, *d_w_ag, *d_w_b, *d_w_bg; /* [c_h][c_z] */
+    float *d_w_g;                           /* [c_z][c_z] */
+    float *d_w_o;                           /* [c_z][c_h] */
+    float *d_b_a, *d_b_ag, *d_b_b, *d_b_bg; /* [c_h] */
+    float *d_b_g, *d_b_o;                   /* [c_z] */
+    float *d_ln_in_w, *d_ln_in_b;           /* [c_z] */
+    float *d_ln_out_w, *d_ln_out_b;         /* [c_h] */
+    void *workspace;                        /* device memory, 256-byte aligned */
+    size_t workspace_bytes;                 /* >= trimul_backward_workspace_size */
+} trimul_grads;
+
+/* Bytes of backward workspace (trimul_grads.workspace) for N. */
+size_t trimul_backward_workspace_size(int N, int c_z, int c_h);
+
+int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,
+                    void *dz, const trimul_grads *g, trimul_stream_t stream);
+
 /* Library version (major * 100 + minor). */
 int trimul_version(void);
 

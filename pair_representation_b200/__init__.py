@@ -37,7 +37,12 @@ ERR = {v: k for k, v in STATUS.items()}
 # Every symbol include/trimul.h declares.
 EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forward", "trimul_prologue",
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
-           "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc")
+           "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
+           "trimul_backward", "trimul_backward_workspace_size")
+
+# Gradient outputs of trimul_grads, in struct order; each is "d_" + a TrimulParams field.
+GRAD_FIELDS = ("d_w_a", "d_w_ag", "d_w_b", "d_w_bg", "d_w_g", "d_w_o", "d_b_a", "d_b_ag", "d_b_b", "d_b_bg",
+               "d_b_g", "d_b_o", "d_ln_in_w", "d_ln_in_b", "d_ln_out_w", "d_ln_out_b")
 
 
 class TrimulError(RuntimeError):
@@ -66,6 +71,13 @@ class TrimulParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("timeout_ms", ctypes.c_uint32), ("debug_flags", ctypes.c_uint32),
     ]
+
+
+class TrimulGrads(ctypes.Structure):
+    """Mirror of ``trimul_grads`` in include/trimul.h (fp32 gradient outputs + backward workspace)."""
+
+    _fields_ = [(f, ctypes.c_void_p) for f in GRAD_FIELDS] + [
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -97,8 +109,11 @@ def lib():
         L.trimul_last_error_detail.argtypes = []
         L.trimul_last_error_detail.restype = ctypes.c_char_p
         L.trimul_version.argtypes = []
+        L.trimul_backward_workspace_size.argtypes = [I, I, I]
+        L.trimul_backward_workspace_size.restype = S
+        L.trimul_backward.argtypes = [P, P, PP, I, P, P, ctypes.POINTER(TrimulGrads), P]
         for f in ("trimul_forward", "trimul_forward_noalloc", "trimul_prologue", "trimul_contract", "trimul_epilogue",
-                  "trimul_workspace_views", "trimul_device_status", "trimul_version"):
+                  "trimul_workspace_views", "trimul_device_status", "trimul_version", "trimul_backward"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -178,6 +193,20 @@ def trimul_epilogue(z, params: TrimulParams, out, stream=None, check=True) -> in
     return rc
 
 
+def trimul_backward_workspace_size(N: int, c_z: int = 128, c_h: int = 128) -> int:
+    return lib().trimul_backward_workspace_size(N, c_z, c_h)
+
+
+def trimul_backward(z, mask, params: TrimulParams, direction: int, dout, dz, grads: TrimulGrads, stream=None,
+                    check=True) -> int:
+    """dz and the fp32 parameter gradients of sum(out * dout); see trimul_backward in the header."""
+    rc = lib().trimul_backward(_ptr(z), _ptr(mask), ctypes.byref(params), direction, _ptr(dout), _ptr(dz),
+                               ctypes.byref(grads), _stream(stream))
+    if check:
+        _check(rc, "trimul_backward")
+    return rc
+
+
 def trimul_workspace_views(params: TrimulParams):
     """(a, b, x, ld): device addresses of the workspace sections and their leading dimension."""
     a, b, x = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
@@ -242,7 +271,7 @@ class _TriangleMultiplication:
         if dtype not in (torch.float32, torch.bfloat16):
             raise ValueError("dtype must be float32 or bfloat16")
         self.tensors = {k: v.to(device=device, dtype=dtype).contiguous() for k, v in self.tensors.items()}
-        self.device = torch.device(device) if device is not None else self.tensors["w_a"].device
+        self.device = self.tensors["w_a"].device  # resolved (cuda -> cuda:0)
         self.dtype = dtype
         return self
 
@@ -277,6 +306,38 @@ class _TriangleMultiplication:
         p = self.params(z.shape[0])
         trimul_forward(z, mask, p, self.direction, out, stream)
         return out
+
+    def backward(self, z, dout, mask=None, stream=None):
+        """Gradients of sum(layer(z, mask) * dout): (dz, {params field: fp32 gradient}).
+
+        Every parameter gets a gradient, including the optional ones the state
+        dict left out (taken as bias 0, gamma 1, beta 0 in the forward)."""
+        import torch
+        if z.dim() != 3 or z.shape[0] != z.shape[1] or z.shape[2] != self.c_z:
+            raise ValueError("z must be [N, N, c_z]")
+        if z.dtype != self.dtype or z.device != self.device or dout.shape != z.shape or dout.dtype != z.dtype:
+            raise ValueError("z and dout must match each other and the layer's dtype and device")
+        z, dout = z.contiguous(), dout.contiguous()
+        if mask is not None:
+            mask = mask.to(dtype=self.dtype).contiguous()
+        N = z.shape[0]
+        p = self.params(N)
+        g = TrimulGrads()
+        need = trimul_backward_workspace_size(N, self.c_z, self.c_h)
+        if getattr(self, "_bws", None) is None or self._bws.numel() < need:
+            self._bws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        g.workspace, g.workspace_bytes = self._bws.data_ptr(), self._bws.numel()
+        cz, ch = self.c_z, self.c_h
+        shapes = {"w_a": (ch, cz), "w_ag": (ch, cz), "w_b": (ch, cz), "w_bg": (ch, cz), "w_g": (cz, cz),
+                  "w_o": (cz, ch), "b_a": (ch,), "b_ag": (ch,), "b_b": (ch,), "b_bg": (ch,), "b_g": (cz,),
+                  "b_o": (cz,), "ln_in_w": (cz,), "ln_in_b": (cz,), "ln_out_w": (ch,), "ln_out_b": (ch,)}
+        grads = {}
+        for f in GRAD_FIELDS:
+            grads[f[2:]] = torch.empty(shapes[f[2:]], dtype=torch.float32, device=self.device)
+            setattr(g, f, grads[f[2:]].data_ptr())
+        dz = torch.empty_like(z)
+        trimul_backward(z, mask, p, self.direction, dout, dz, g, stream)
+        return dz, grads
 
     def forward_host(self, z_host, mask_host=None, out_host=None, stream=None):
         """End to end from host memory: copy z (and the mask) in, run, copy out back."""

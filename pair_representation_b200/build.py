@@ -17,8 +17,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtrimul_b200.so")
-SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu", "noalloc.cu",
+           "backward.cu", "blas.cu"]
+HEADERS = ["common.cuh", "kernels.h", "tile_ops.cuh"]
 
 
 def nvcc() -> str:
@@ -42,7 +43,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
+           "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "-ldl",
            "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-o", tmp]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]

@@ -72,8 +72,9 @@ int device_state(const DevState **out, bool need_tc) {
             return TRIMUL_ERR_CUDA;
         }
         if (d.cc_major == 10 && d.cc_minor == 0) {
-            if ((e = prologue_tc_setup()) == cudaSuccess && (e = contract_tc_setup()) == cudaSuccess)
-                e = epilogue_tc_setup();
+            if ((e = prologue_tc_setup()) == cudaSuccess && (e = contract_tc_setup()) == cudaSuccess &&
+                (e = epilogue_tc_setup()) == cudaSuccess)
+                e = backward_setup();
             d.tc_setup = e;
         } else {
             d.tc_setup = cudaErrorNoKernelImageForDevice;
@@ -416,6 +417,295 @@ int clear_status(const trimul_params *p, cudaStream_t s) {
     return cuda_rc(cudaMemsetAsync(p->workspace, 0, sizeof(DeviceStatus), s), "status clear");
 }
 
+// ---- backward ----------------------------------------------------------------------
+
+constexpr size_t kBlasWorkspace = 32u << 20;
+constexpr long long kWgradChunk = 4096;  // cells per weight-gradient GEMM partial
+
+long long wgrad_slots(int N) { return ((long long)N * N + kWgradChunk - 1) / kWgradChunk; }
+
+// Sections of the backward workspace (byte offsets, each 256-byte aligned).
+struct BwdLayout {
+    size_t blas, sums, wstack, st_in, st_out, zh, xh, P, Y, dxh, D, dy, dX, dA, dB, partial, total;
+};
+
+BwdLayout bwd_layout(int N) {
+    const size_t M = (size_t)N * N, C = kC, cm = C * (size_t)N * ld_of(N);
+    BwdLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    L.blas = take(kBlasWorkspace);
+    L.sums = take((size_t)kSumCount * C * 4);
+    L.wstack = take((size_t)kProjBlocks * C * C * 2);
+    L.st_in = take(M * 8);
+    L.st_out = take(M * 8);
+    L.zh = take(M * C * 2);                 // LayerNorm_in(z), bf16 [cells][128]
+    L.xh = take(M * C * 2);                 // LayerNorm_out(x), bf16 [cells][128]
+    L.P = take(M * kProjBlocks * C * 2);    // zh W^T pre-activations, bf16; later dL/dzh, fp32 [cells][128]
+    L.Y = take(M * C * 2);                  // xh W_o^T, bf16
+    L.dxh = take(M * C * 4);                // dL/dxh, fp32
+    L.D = take(M * kProjBlocks * C * 2);    // pre-activation gradients, bf16
+    L.dy = take(M * C * 2);                 // dL/dy, bf16
+    L.dX = take(cm * 2);                    // dL/dx, bf16 [128][N][ld]
+    L.dA = take(cm * 2);                    // dL/da, bf16 [128][N][ld]
+    L.dB = take(cm * 2);
+    L.partial = take((size_t)wgrad_slots(N) * kWgradRows * C * 4);
+    L.total = off;
+    return L;
+}
+
+int check_backward(const trimul_params *p, const void *z, const void *mask, const void *dout, const void *dz,
+                   const trimul_grads *g) {
+    if (!dout || !dz || !g) return TRIMUL_ERR_INVALID_ARG;
+    if (p->dtype != TRIMUL_DTYPE_BF16) return TRIMUL_ERR_UNSUPPORTED;
+    if (!aligned(dout, 16) || !aligned(dz, 16)) return TRIMUL_ERR_MISALIGNED;
+    if (!g->workspace || g->workspace_bytes < bwd_layout(p->N).total) return TRIMUL_ERR_WORKSPACE;
+    if (!aligned(g->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
+    const size_t n = pair_bytes(p), mb = mask_bytes(p);
+    const void *gws = g->workspace;
+    const size_t gwn = g->workspace_bytes;
+    if (overlap(dz, n, z, n) || overlap(dz, n, mask, mb) || overlap(dz, n, dout, n) ||
+        overlap(dz, n, p->workspace, p->workspace_bytes) || overlap(dz, n, gws, gwn) ||
+        overlap(dout, n, p->workspace, p->workspace_bytes) || overlap(dout, n, gws, gwn) ||
+        overlap(gws, gwn, p->workspace, p->workspace_bytes) || overlap(gws, gwn, z, n) || overlap(gws, gwn, mask, mb))
+        return TRIMUL_ERR_ALIAS;
+    // Gradient outputs: weights [128][128] (16-byte aligned, written by GEMMs), vectors [128].
+    const void *outs[16] = {g->d_w_a, g->d_w_ag, g->d_w_b, g->d_w_bg, g->d_w_g, g->d_w_o,
+                            g->d_b_a, g->d_b_ag, g->d_b_b, g->d_b_bg, g->d_b_g, g->d_b_o,
+                            g->d_ln_in_w, g->d_ln_in_b, g->d_ln_out_w, g->d_ln_out_b};
+    size_t sz[16];
+    for (int k = 0; k < 16; ++k) {
+        sz[k] = (size_t)(k < 6 ? kC * kC : kC) * 4;
+        if (outs[k] && !aligned(outs[k], k < 6 ? 16 : 4)) return TRIMUL_ERR_MISALIGNED;
+    }
+    for (int k = 0; k < 16; ++k) {
+        if (!outs[k]) continue;
+        if (overlap(outs[k], sz[k], z, n) || overlap(outs[k], sz[k], mask, mb) || overlap(outs[k], sz[k], dout, n) ||
+            overlap(outs[k], sz[k], dz, n) || overlap(outs[k], sz[k], p->workspace, p->workspace_bytes) ||
+            overlap(outs[k], sz[k], gws, gwn))
+            return TRIMUL_ERR_ALIAS;
+        for (int l = k + 1; l < 16; ++l)
+            if (overlap(outs[k], sz[k], outs[l], sz[l])) return TRIMUL_ERR_ALIAS;
+    }
+    return TRIMUL_OK;
+}
+
+int check_backward_on_device(const void *dout, const void *dz, const trimul_grads *g) {
+    const void *all[] = {dout, dz, g->workspace, g->d_w_a, g->d_w_ag, g->d_w_b, g->d_w_bg, g->d_w_g, g->d_w_o,
+                         g->d_b_a, g->d_b_ag, g->d_b_b, g->d_b_bg, g->d_b_g, g->d_b_o,
+                         g->d_ln_in_w, g->d_ln_in_b, g->d_ln_out_w, g->d_ln_out_b};
+    for (const void *v : all)
+        if (int rc = check_device_ptr(v, "backward pointer")) return rc;
+    return TRIMUL_OK;
+}
+
+// Enqueues one GEMM on the bound handle; 0 or TRIMUL_ERR_CUDA.
+int gemm(void *h, const Gemm &g) {
+    if (blas_gemm(h, g, g_detail, sizeof g_detail)) return TRIMUL_ERR_CUDA;
+    return TRIMUL_OK;
+}
+
+// Row-major C[M][N] = op(A) op(B), one problem, bf16 operands.
+Gemm gemm1(bool ta, bool tb, int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C, int ldc,
+           bool c_f32 = true, float beta = 0.f) {
+    Gemm g;
+    g.ta = ta;
+    g.tb = tb;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.A = A;
+    g.lda = lda;
+    g.sA = 0;
+    g.B = B;
+    g.ldb = ldb;
+    g.sB = 0;
+    g.beta = beta;
+    g.C = C;
+    g.c_f32 = c_f32;
+    g.ldc = ldc;
+    g.sC = 0;
+    g.batch = 1;
+    return g;
+}
+
+// The backward's launch sequence; the caller holds blas_lock().
+int run_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout, void *dz,
+                 const trimul_grads *gr, const DevState &d, cudaStream_t s) {
+    typedef __nv_bfloat16 bf;
+    const int N = p->N, C = kC;
+    const long long cells = (long long)N * N;
+    const Views v = views_of(p);
+    const BwdLayout L = bwd_layout(N);
+    uint8_t *base = static_cast<uint8_t *>(gr->workspace);
+    float *sums = reinterpret_cast<float *>(base + L.sums);
+    bf *wstack = reinterpret_cast<bf *>(base + L.wstack);
+    float2 *st_in = reinterpret_cast<float2 *>(base + L.st_in), *st_out = reinterpret_cast<float2 *>(base + L.st_out);
+    bf *zh = reinterpret_cast<bf *>(base + L.zh), *xh = reinterpret_cast<bf *>(base + L.xh);
+    bf *P = reinterpret_cast<bf *>(base + L.P), *Y = reinterpret_cast<bf *>(base + L.Y);
+    float *dzh = reinterpret_cast<float *>(base + L.P), *dxh = reinterpret_cast<float *>(base + L.dxh);
+    bf *D = reinterpret_cast<bf *>(base + L.D), *dy = reinterpret_cast<bf *>(base + L.dy);
+    bf *dX = reinterpret_cast<bf *>(base + L.dX);
+    bf *dA = reinterpret_cast<bf *>(base + L.dA), *dB = reinterpret_cast<bf *>(base + L.dB);
+    float *partial = reinterpret_cast<float *>(base + L.partial);
+    const bf *x = reinterpret_cast<const bf *>(v.x);
+    const int ld = (int)v.ld;
+    const long long cs = (long long)N * ld;  // channel stride of [128][N][ld]
+    int rc;
+
+    // Recompute the forward's a, b and x into the forward workspace.
+    if ((rc = clear_status(p, s)) || (rc = run_prologue(z, mask, p, d, s)) || (rc = run_contract(p, direction, d, s)))
+        return rc;
+    if ((rc = cuda_rc(cudaMemsetAsync(sums, 0, (size_t)kSumCount * C * 4, s), "backward sums clear"))) return rc;
+    const void *wk[kProjBlocks] = {p->w_g, p->w_a, p->w_ag, p->w_b, p->w_bg};
+    for (int k = 0; k < kProjBlocks; ++k)
+        if ((rc = cuda_rc(cudaMemcpyAsync(wstack + (size_t)k * C * C, wk[k], (size_t)C * C * 2,
+                                          cudaMemcpyDeviceToDevice, s), "weight stack copy")))
+            return rc;
+
+    LnFwdArgs lf;
+    lf.src = static_cast<const bf *>(z);
+    lf.channel_major = 0;
+    lf.N = N;
+    lf.ld = v.ld;
+    lf.eps = p->ln_eps;
+    lf.gamma = static_cast<const bf *>(p->ln_in_w);
+    lf.beta = static_cast<const bf *>(p->ln_in_b);
+    lf.out = zh;
+    lf.stats = st_in;
+    if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
+    lf.src = x;
+    lf.channel_major = 1;
+    lf.gamma = static_cast<const bf *>(p->ln_out_w);
+    lf.beta = static_cast<const bf *>(p->ln_out_b);
+    lf.out = xh;
+    lf.stats = st_out;
+    if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
+
+    void *h = nullptr;
+    if (blas_bind(s, base + L.blas, kBlasWorkspace, &h, g_detail, sizeof g_detail)) return TRIMUL_ERR_CUDA;
+    const int M = (int)cells, PB = kProjBlocks * C;
+    // P = zh [W_g; W_a; W_ag; W_b; W_bg]^T and Y = xh W_o^T (before biases), bf16.
+    if ((rc = gemm(h, gemm1(false, true, M, PB, C, zh, C, wstack, C, P, PB, false)))) return rc;
+    if ((rc = gemm(h, gemm1(false, true, M, C, C, xh, C, p->w_o, C, Y, C, false)))) return rc;
+
+    GateBwdArgs ga;
+    ga.dout = static_cast<const bf *>(dout);
+    ga.P = P;
+    ga.Y = Y;
+    ga.b_g = static_cast<const bf *>(p->b_g);
+    ga.b_o = static_cast<const bf *>(p->b_o);
+    ga.dy = dy;
+    ga.D = D;
+    ga.db_g = sums + S_B_G * C;
+    ga.db_o = sums + S_B_O * C;
+    ga.cells = cells;
+    if ((rc = cuda_rc(launch_gate_bwd(ga, d.sms, s), "gate_bwd launch"))) return rc;
+
+    // dL/dxh = dy W_o (fp32).
+    if ((rc = gemm(h, gemm1(false, false, M, C, C, dy, C, p->w_o, C, dxh, C)))) return rc;
+
+    LnBwdArgs lb;
+    lb.dh = dxh;
+    lb.src = x;
+    lb.channel_major = 1;
+    lb.N = N;
+    lb.ld = v.ld;
+    lb.stats = st_out;
+    lb.gamma = static_cast<const bf *>(p->ln_out_w);
+    lb.dsrc = dX;
+    lb.dgamma = sums + S_LN_OUT_W * C;
+    lb.dbeta = sums + S_LN_OUT_B * C;
+    if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+
+    // The contraction's adjoint, one N x N x N product per channel (bf16 out):
+    //   outgoing (X = A B^T): dA = dX B,    dB = dX^T A
+    //   incoming (X = A^T B): dA = B dX^T,  dB = A dX
+    Gemm g = gemm1(false, false, N, N, N, nullptr, ld, nullptr, ld, nullptr, ld, false);
+    g.sA = g.sB = g.sC = cs;
+    g.batch = C;
+    const bf *a = reinterpret_cast<const bf *>(v.a), *b = reinterpret_cast<const bf *>(v.b);
+    Gemm ga1 = g, gb1 = g;
+    if (direction == TRIMUL_OUTGOING) {
+        ga1.A = dX, ga1.B = b;
+        gb1.ta = true, gb1.A = dX, gb1.B = a;
+    } else {
+        ga1.tb = true, ga1.A = b, ga1.B = dX;
+        gb1.A = a, gb1.B = dX;
+    }
+    ga1.C = dA;
+    gb1.C = dB;
+    if ((rc = gemm(h, ga1)) || (rc = gemm(h, gb1))) return rc;
+
+    ProjBwdArgs pa;
+    pa.dA = dA;
+    pa.dB = dB;
+    pa.P = P;
+    pa.mask = static_cast<const bf *>(mask);
+    pa.b_a = static_cast<const bf *>(p->b_a);
+    pa.b_ag = static_cast<const bf *>(p->b_ag);
+    pa.b_b = static_cast<const bf *>(p->b_b);
+    pa.b_bg = static_cast<const bf *>(p->b_bg);
+    pa.D = D;
+    pa.db = sums + S_B_A * C;
+    pa.N = N;
+    pa.ld = v.ld;
+    if ((rc = cuda_rc(launch_proj_bwd(pa, d.sms, s), "proj_bwd launch"))) return rc;
+
+    // Weight gradients, one partial per chunk of kWgradChunk cells:
+    //   rows [0, 640):   D^T zh  ([W_g; W_a; W_ag; W_b; W_bg] gradients)
+    //   rows [640, 768): dy^T xh (W_o gradient)
+    // then summed over the chunks in double.
+    const long long full = cells / kWgradChunk, rem = cells - full * kWgradChunk;
+    const int K = (int)kWgradChunk;
+    const long long pstride = (long long)kWgradRows * C;
+    if (full > 0) {
+        Gemm w1 = gemm1(true, false, PB, C, K, D, PB, zh, C, partial, C);
+        w1.sA = (long long)K * PB, w1.sB = (long long)K * C, w1.sC = pstride, w1.batch = (int)full;
+        Gemm w2 = gemm1(true, false, C, C, K, dy, C, xh, C, partial + (size_t)PB * C, C);
+        w2.sA = (long long)K * C, w2.sB = (long long)K * C, w2.sC = pstride, w2.batch = (int)full;
+        if ((rc = gemm(h, w1)) || (rc = gemm(h, w2))) return rc;
+    }
+    if (rem > 0) {
+        const size_t r0 = (size_t)full * kWgradChunk;
+        float *pr = partial + (size_t)full * pstride;
+        if ((rc = gemm(h, gemm1(true, false, PB, C, (int)rem, D + r0 * PB, PB, zh + r0 * C, C, pr, C))) ||
+            (rc = gemm(h, gemm1(true, false, C, C, (int)rem, dy + r0 * C, C, xh + r0 * C, C, pr + (size_t)PB * C, C))))
+            return rc;
+    }
+    WgradReduceArgs wr;
+    wr.partial = partial;
+    wr.slots = (int)wgrad_slots(N);
+    float *wdst[kProjBlocks + 1] = {gr->d_w_g, gr->d_w_a, gr->d_w_ag, gr->d_w_b, gr->d_w_bg, gr->d_w_o};
+    for (int k = 0; k <= kProjBlocks; ++k) wr.dst[k] = wdst[k];
+    if ((rc = cuda_rc(launch_wgrad_reduce(wr, s), "wgrad_reduce launch"))) return rc;
+
+    // dL/dzh = D [W_g; W_a; W_ag; W_b; W_bg] (fp32, over the spent pre-activations).
+    if ((rc = gemm(h, gemm1(false, false, M, C, PB, D, PB, wstack, C, dzh, C)))) return rc;
+
+    lb.dh = dzh;
+    lb.src = static_cast<const bf *>(z);
+    lb.channel_major = 0;
+    lb.stats = st_in;
+    lb.gamma = static_cast<const bf *>(p->ln_in_w);
+    lb.dsrc = static_cast<bf *>(dz);
+    lb.dgamma = sums + S_LN_IN_W * C;
+    lb.dbeta = sums + S_LN_IN_B * C;
+    if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+
+    float *vec[kSumCount] = {gr->d_b_g, gr->d_b_o, gr->d_b_a, gr->d_b_ag, gr->d_b_b, gr->d_b_bg,
+                             gr->d_ln_out_w, gr->d_ln_out_b, gr->d_ln_in_w, gr->d_ln_in_b};
+    for (int k = 0; k < kSumCount; ++k)
+        if (vec[k] && (rc = cuda_rc(cudaMemcpyAsync(vec[k], sums + k * C, (size_t)C * 4, cudaMemcpyDeviceToDevice, s),
+                                    "gradient copy")))
+            return rc;
+    return TRIMUL_OK;
+}
+
 }  // namespace
 
 // ---- exported symbols -------------------------------------------------------------
@@ -510,6 +800,28 @@ int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *de
     }
     if (st.code == DEV_OK) return TRIMUL_OK;
     return st.code == DEV_TIMEOUT ? TRIMUL_ERR_TIMEOUT : TRIMUL_ERR_DEVICE;
+}
+
+size_t trimul_backward_workspace_size(int N, int c_z, int c_h) {
+    if (N < 1 || N > kMaxN || c_z != kC || c_h != kC) return 0;
+    return bwd_layout(N).total;
+}
+
+int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,
+                    void *dz, const trimul_grads *g, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction)) || (rc = check_z(p, z)) ||
+        (rc = check_mask(p, mask)) || (rc = check_backward(p, z, mask, dout, dz, g)))
+        return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
+        (rc = check_device_ptr(mask, "mask")) || (rc = check_backward_on_device(dout, dz, g)))
+        return rc;
+    blas_lock();
+    rc = run_backward(z, mask, p, direction, dout, dz, g, *d, reinterpret_cast<cudaStream_t>(stream));
+    blas_unlock();
+    return rc;
 }
 
 const char *trimul_error_string(int code) {

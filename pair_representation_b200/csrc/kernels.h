@@ -77,6 +77,117 @@ cudaError_t contract_tc_setup();
 cudaError_t launch_contract_tc(const ContractMaps &m, const ContractArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_epilogue_tc(const EpilogueMaps &m, const EpilogueArgs &a, int grid, cudaStream_t s);
 
+// ---- backward (bf16 forward intermediates, fp32 gradients) -----------------------
+
+// Gradient sums over cells, [kSumCount][128] floats in the backward workspace.
+enum BwdSum { S_B_G, S_B_O, S_B_A, S_B_AG, S_B_B, S_B_BG, S_LN_OUT_W, S_LN_OUT_B, S_LN_IN_W, S_LN_IN_B, kSumCount };
+
+// Projection blocks of the [cells][5 * 128] arrays P (pre-activations) and D
+// (their gradients), and of the stacked weight [5 * 128][128].
+enum ProjBlock { P_G, P_A, P_AG, P_B, P_BG, kProjBlocks };
+
+// LayerNorm of each cell: out = (v - mean) * rstd * gamma + beta as bf16
+// [cells][128], and (mean, rstd) per cell. src is cell-major [N][N][128] or,
+// when channel_major, [128][N][ld].
+struct LnFwdArgs {
+    const __nv_bfloat16 *src;
+    int channel_major;
+    int N;
+    size_t ld;
+    float eps;
+    const __nv_bfloat16 *gamma, *beta;  // or null
+    __nv_bfloat16 *out;
+    float2 *stats;
+};
+
+// LayerNorm adjoint: dsrc = rstd * (dn - mean(dn) - n * mean(dn * n)) with
+// dn = dh * gamma and n recomputed from src and stats; dgamma += dh * n and
+// dbeta += dh over all cells. dsrc has src's layout (bf16).
+struct LnBwdArgs {
+    const float *dh;  // [cells][128]
+    const __nv_bfloat16 *src;
+    int channel_major;
+    int N;
+    size_t ld;
+    const float2 *stats;
+    const __nv_bfloat16 *gamma;  // or null
+    __nv_bfloat16 *dsrc;
+    float *dgamma, *dbeta;
+};
+
+// Output gate adjoint, per cell and channel: g = sigmoid(P_G + b_g),
+// y = Y + b_o, dy = dout * g, dP_G = dout * y * g * (1 - g).
+struct GateBwdArgs {
+    const __nv_bfloat16 *dout;  // [cells][128]
+    const __nv_bfloat16 *P;     // [cells][5 * 128]
+    const __nv_bfloat16 *Y;     // [cells][128]
+    const __nv_bfloat16 *b_g, *b_o;
+    __nv_bfloat16 *dy;  // [cells][128]
+    __nv_bfloat16 *D;   // [cells][5 * 128], block P_G written
+    float *db_g, *db_o;
+    long long cells;
+};
+
+// Gating and mask adjoint of a and b: from dA, dB ([128][N][ld] bf16) and P,
+// writes D blocks P_A .. P_BG and adds their sums over cells to db.
+struct ProjBwdArgs {
+    const __nv_bfloat16 *dA, *dB;
+    const __nv_bfloat16 *P;
+    const __nv_bfloat16 *mask;  // [N][N] or null
+    const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
+    __nv_bfloat16 *D;
+    float *db;  // [4][128]: b_a, b_ag, b_b, b_bg
+    int N;
+    size_t ld;
+};
+
+// Weight gradients: the rows of [W_g; W_a; W_ag; W_b; W_bg; W_o] gradients,
+// each GEMM partial (one per chunk of cells) being [kWgradRows][128] fp32.
+constexpr int kWgradRows = (kProjBlocks + 1) * kC;
+struct WgradReduceArgs {
+    const float *partial;  // [slots][kWgradRows][128]
+    int slots;
+    float *dst[kProjBlocks + 1];  // [128][128] each (block order above), or null
+};
+
+cudaError_t backward_setup();
+// Each launcher sizes its grid as one wave of resident blocks on `sms` SMs.
+cudaError_t launch_ln_fwd(const LnFwdArgs &a, int sms, cudaStream_t s);
+cudaError_t launch_ln_bwd(const LnBwdArgs &a, int sms, cudaStream_t s);
+cudaError_t launch_gate_bwd(const GateBwdArgs &a, int sms, cudaStream_t s);
+cudaError_t launch_proj_bwd(const ProjBwdArgs &a, int sms, cudaStream_t s);
+cudaError_t launch_wgrad_reduce(const WgradReduceArgs &a, cudaStream_t s);
+
+// ---- cuBLAS, loaded on first use (blas.cu) ------------------------------------
+
+// Row-major C = op(A) op(B) (bf16 operands, fp32 accumulation), batched with
+// element strides; op(X) = X^T when tX. C is fp32 when c_f32, else bf16.
+struct Gemm {
+    bool ta, tb;
+    int M, N, K;
+    const void *A;
+    int lda;
+    long long sA;
+    const void *B;
+    int ldb;
+    long long sB;
+    float beta;
+    void *C;
+    bool c_f32;
+    int ldc;
+    long long sC;
+    int batch;
+};
+
+// Serialises use of the per-device handles.
+void blas_lock();
+void blas_unlock();
+// With the lock held: the current device's handle, bound to stream s and the
+// given workspace. Returns 0, or -1 with a message in detail.
+int blas_bind(cudaStream_t s, void *ws, size_t ws_bytes, void **handle, char *detail, size_t detail_n);
+// Returns 0, or the cuBLAS status with a message in detail.
+int blas_gemm(void *handle, const Gemm &g, char *detail, size_t detail_n);
+
 // ---- fp32 CUDA-core path ----------------------------------------------------
 
 struct F32Layer {

@@ -149,3 +149,99 @@ def test_stage_argument_checks(L):
     a, b, x, ld = tm.trimul_workspace_views(p)
     assert a == p.workspace + 256 and ld == 64
     assert b - a == x - b == 128 * 64 * 64 * 2
+
+
+# ---- backward ------------------------------------------------------------------
+
+def _bwd_layout_bytes(N):
+    """Backward workspace: cuBLAS slice, sums, weight stack, per-cell sections, then
+    one [768][128] fp32 weight-gradient partial per 4096-cell chunk."""
+    r = lambda v: (v + 255) // 256 * 256
+    M, C, ld = N * N, 128, (N + 7) // 8 * 8
+    cm = C * N * ld
+    slots = (M + 4095) // 4096
+    parts = [32 << 20, 10 * C * 4, 5 * C * C * 2, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
+             M * C * 4, M * 5 * C * 2, M * C * 2, cm * 2, cm * 2, cm * 2, slots * 768 * C * 4]
+    return sum(r(p) for p in parts)
+
+
+def test_backward_workspace_size(L):
+    for N in (1, 7, 64, 129, 768):
+        assert tm.trimul_backward_workspace_size(N) == _bwd_layout_bytes(N), N
+    assert tm.trimul_backward_workspace_size(0) == 0
+    assert tm.trimul_backward_workspace_size(16385) == 0
+    assert tm.trimul_backward_workspace_size(64, 64, 128) == 0
+
+
+DOUT = BASE + 0x100000000
+DZ = BASE + 0x140000000
+GWS = BASE + 0x200000000
+
+
+def _grads(N=64):
+    g = tm.TrimulGrads()
+    g.workspace = GWS
+    g.workspace_bytes = tm.trimul_backward_workspace_size(N)
+    for k, f in enumerate(tm.GRAD_FIELDS):
+        setattr(g, f, BASE + 0x400000000 + 0x100000 * k)
+    return g
+
+
+def _bwd(p, g, z=Z, mask=MASK, dout=DOUT, dz=DZ, direction=0):
+    return tm.trimul_backward(z, mask, p, direction, dout, dz, g, stream=0, check=False)
+
+
+def test_backward_argument_checks(L):
+    E = tm.ERR
+    p, g = _params(), _grads()
+    assert tm.lib().trimul_backward(Z, MASK, ctypes.byref(p), 0, DOUT, DZ, None, None) == E["TRIMUL_ERR_INVALID_ARG"]
+    assert _bwd(p, g, dout=None) == E["TRIMUL_ERR_INVALID_ARG"]
+    assert _bwd(p, g, dz=None) == E["TRIMUL_ERR_INVALID_ARG"]
+    assert _bwd(p, g, direction=2) == E["TRIMUL_ERR_INVALID_ARG"]
+    assert _bwd(_params(dtype=tm.DTYPE_F32), g) == E["TRIMUL_ERR_UNSUPPORTED"]
+    assert _bwd(p, g, dout=DOUT + 8) == E["TRIMUL_ERR_MISALIGNED"]
+    assert _bwd(p, g, dz=DZ + 2) == E["TRIMUL_ERR_MISALIGNED"]
+    q = _grads(); q.workspace = None
+    assert _bwd(p, q) == E["TRIMUL_ERR_WORKSPACE"]
+    q = _grads(); q.workspace_bytes -= 1
+    assert _bwd(p, q) == E["TRIMUL_ERR_WORKSPACE"]
+    q = _grads(); q.workspace += 128
+    assert _bwd(p, q) == E["TRIMUL_ERR_MISALIGNED"]
+    q = _grads(); q.d_w_o += 4
+    assert _bwd(p, q) == E["TRIMUL_ERR_MISALIGNED"]
+    q = _grads(); q.d_b_g += 2
+    assert _bwd(p, q) == E["TRIMUL_ERR_MISALIGNED"]
+
+
+def test_backward_alias_checks(L):
+    E = tm.ERR
+    p, g = _params(), _grads()
+    zbytes = 64 * 64 * 128 * 2
+    assert _bwd(p, g, dz=Z) == E["TRIMUL_ERR_ALIAS"]
+    assert _bwd(p, g, dz=DOUT + zbytes - 16) == E["TRIMUL_ERR_ALIAS"]
+    assert _bwd(p, g, dz=p.workspace + 256) == E["TRIMUL_ERR_ALIAS"]
+    assert _bwd(p, g, dz=GWS + 4096) == E["TRIMUL_ERR_ALIAS"]
+    assert _bwd(p, g, dout=GWS) == E["TRIMUL_ERR_ALIAS"]
+    q = _grads(); q.workspace = p.workspace
+    assert _bwd(p, q) == E["TRIMUL_ERR_ALIAS"]
+    q = _grads(); q.d_w_a = q.d_w_ag
+    assert _bwd(p, q) == E["TRIMUL_ERR_ALIAS"]
+    q = _grads(); q.d_b_a = DZ
+    assert _bwd(p, q) == E["TRIMUL_ERR_ALIAS"]
+    q = _grads(); q.d_ln_in_w = GWS + 512
+    assert _bwd(p, q) == E["TRIMUL_ERR_ALIAS"]
+
+
+def test_backward_reaches_cuda_and_fails_loudly_without_gpu(L):
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+    p, g = _params(), _grads()
+    assert _bwd(p, g) in (tm.ERR["TRIMUL_ERR_CUDA"], tm.ERR["TRIMUL_ERR_UNSUPPORTED"])
+    q = _grads()
+    for f in tm.GRAD_FIELDS:
+        setattr(q, f, None)  # every gradient output skipped: still a valid call
+    assert _bwd(p, q) in (tm.ERR["TRIMUL_ERR_CUDA"], tm.ERR["TRIMUL_ERR_UNSUPPORTED"])
