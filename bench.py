@@ -13,6 +13,10 @@ layer is one pair-cell); algorithmic TFLOP/s is reported beside it.
 With N > 1 (launched by torchrun) every rank runs an independent replica on its
 own GPU (the layer is not sharded); value = cells of all ranks / max time.
 
+Secondary figures on rank 0 at N = 1: every workload per direction
+("per_config") and one trimul_backward call per direction at N = 768
+("backward"; --backward-only times just that).
+
 Timing: CUDA events on the launching stream; L2 is flushed (512 MB write)
 before every step and the flush is outside the timed events; a barrier and a
 device synchronize bracket the K timed steps on every rank.
@@ -241,6 +245,81 @@ def per_config_timings(tm, pi, torch, dev, stream, warmup=3, reps=5):
     return res
 
 
+def backward_flops_per_cell(N: int) -> int:
+    """GEMM FLOP per cell of one trimul_backward call: the recomputed a, b and x
+    (4 projections + contraction), then P (5 projections), Y, dL/dxh, the
+    contraction's adjoint (2 products), the 6 weight gradients and dL/dzh (5)."""
+    g = 2 * 128 * 128
+    return 4 * g + 256 * N + 5 * g + g + g + 2 * 256 * N + 6 * g + 5 * g
+
+
+# HBM bytes per cell that the backward's steps move at their minimum (each
+# array read or written once per step that uses it), excluding the recomputed
+# forward: LayerNorms 2 x 520, P 1536, Y 512, gate 1280, dL/dxh 768, LN_out
+# adjoint 1032, contraction adjoint 1536, input-gate adjoint 2562, weight
+# gradients 2048, dL/dzh 1792, LN_in adjoint 1032.
+BACKWARD_BYTES_PER_CELL = 2 * 520 + 1536 + 512 + 1280 + 768 + 1032 + 1536 + 2562 + 2048 + 1792 + 1032
+
+
+def backward_timings(tm, pi, torch, dev, stream, peaks, warmup=3, reps=7):
+    """Secondary figure: one trimul_backward call per direction on the N = 768
+    workload (dout drawn N(0, 1), bf16), CUDA events, L2 flushed before each call."""
+    import numpy as np
+    w = pi.WORKLOADS[DEFAULT_WORKLOAD]
+    N = w.N
+    case = pi.make_workload(w)
+    z = torch.from_numpy(case["z"]).to(dev).to(torch.bfloat16)
+    mask = torch.from_numpy(case["mask"]).to(dev).to(torch.bfloat16)
+    dout = torch.from_numpy(np.random.default_rng([7, 8]).standard_normal((N, N, 128), dtype=np.float32)).to(dev)
+    dout = dout.to(torch.bfloat16)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    res = {"workload": w.name, "N": N, "dtype": "bf16", "gemm_flop_per_cell": backward_flops_per_cell(N),
+           "hbm_bytes_per_cell_min": BACKWARD_BYTES_PER_CELL,
+           "recompute": "a, b, x recomputed by the forward kernels inside the call"}
+    for d, cls in (("outgoing", tm.TriangleMultiplicationOutgoing), ("incoming", tm.TriangleMultiplicationIncoming)):
+        sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+        layer = cls(128, 128).load_state_dict(sd).to(dev, torch.bfloat16)
+        for _ in range(warmup):
+            layer.backward(z, dout, mask, stream=stream)
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer.backward(z, dout, mask, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        ts.sort()
+        med = ts[len(ts) // 2]
+        res[d] = {"median_us": round(med, 1), "best_us": round(ts[0], 1),
+                  "pair_cells_per_s": round(N * N / (med * 1e-6)),
+                  "gemm_tflops": round(N * N * backward_flops_per_cell(N) / (med * 1e-6) / 1e12, 1),
+                  "min_bytes_gbs": round(N * N * BACKWARD_BYTES_PER_CELL / (med * 1e-6) / 1e9, 1)}
+        del layer
+    res["hbm_peak_gbs"] = peaks["hbm_gbs"]
+    del z, mask, dout, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_backward_only(args):
+    """--backward-only: the backward secondary figure alone, on one GPU."""
+    import torch
+
+    import pair_inputs as pi
+    import pair_representation_b200 as tm
+    from pair_representation_b200 import build as tmbuild
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tmbuild.build()
+    tm.lib()
+    peaks, _ = load_peaks()
+    res = backward_timings(tm, pi, torch, dev, torch.cuda.current_stream(dev), peaks, args.warmup, args.steps)
+    print(json.dumps({"backward": res}), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -401,9 +480,12 @@ def run_ours(args, rank, world, local_rank):
     tflops = world * args.steps * len(dirs) * N * N * flops_per_cell(N) / (total_ms / 1e3) / 1e12
     clocks = sampler.summary()
     configs = None
+    backward = None
     if rank == 0 and world == 1 and not args.no_configs:
         del flush
         configs = per_config_timings(tm, pi, torch, dev, stream)
+    if rank == 0 and world == 1 and not args.no_backward:
+        backward = backward_timings(tm, pi, torch, dev, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -420,6 +502,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": sum(launches.values()),
         "clocks": clocks,
         "per_config": configs,
+        "backward": backward,
     }
     if dist:
         dist.barrier()
@@ -470,6 +553,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload secondary timings")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward secondary timing")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only trimul_backward (W warm-up and K timed calls per direction) and print that")
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=120.0)
     args = ap.parse_args(argv)
@@ -482,6 +568,8 @@ def main(argv=None):
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.backward_only:
+        run_backward_only(args)
     else:
         run_ours(args, rank, world, local_rank)
 
