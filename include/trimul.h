@@ -169,11 +169,12 @@ int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params 
  * The forward intermediates are recomputed: the call enqueues the prologue and
  * the contraction into p->workspace, then the backward steps, which keep their
  * intermediates (bf16, with fp32 for the LayerNorm adjoints' inputs) in
- * g->workspace. The plain GEMMs of the backward (projections, weight
- * gradients and the contraction's adjoint, per channel dA_c = dX_c B_c and
+ * g->workspace. The contraction's adjoint (per channel dA_c = dX_c B_c and
  * dB_c = dX_c^T A_c outgoing, dA_c = B_c dX_c^T and dB_c = A_c dX_c incoming)
- * run on cuBLAS with fp32 accumulation; the LayerNorm, gate and mask adjoints
- * run in the library's kernels. Weight gradients are summed per chunk of 4096
+ * runs on the forward's tcgen05 contraction kernel with the operands in other
+ * transposes; the LayerNorm, gate and mask adjoints run in the library's own
+ * kernels; the plain GEMMs (projections, weight gradients) run on cuBLAS with
+ * fp32 accumulation. Weight gradients are summed per chunk of 4096
  * cells by GEMM and over the chunks in double by the library, so they do not
  * depend on how cuBLAS splits a reduction over N^2 cells; bias and LayerNorm
  * gradients are fp32 sums (atomic, so their last bits may vary between runs).

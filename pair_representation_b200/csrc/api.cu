@@ -353,31 +353,36 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
     return cuda_rc(launch_prologue_tc(m, a, grid, s), "prologue_tc launch");
 }
 
+// X_c[m][n] = sum_k A_c(m, k) B_c(n, k) for the 128 channels of [128][N][ld] bf16
+// arrays, each operand K-major ([rows][k]) or MN-major ([k][rows]), on the
+// tcgen05 pair kernel. CTA pairs share each 256 x 256 output tile: CTA r loads
+// rows [128 r, 128 r + 128) of the A and B panels (boxes of 128 rows, or 2 x
+// 64-wide blocks when MN-major).
+int run_contract_on(const void *A, int a_mn, const void *B, int b_mn, void *X, int N, size_t ld, const KernelCtl &ctl,
+                    const DevState &d, cudaStream_t s) {
+    ContractMaps m;
+    if (int rc = map_cm(&m.a, A, N, ld, 64, a_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    if (int rc = map_cm(&m.b, B, N, ld, 64, b_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    if (int rc = map_cm(&m.x, X, N, ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    ContractArgs a;
+    a.N = N;
+    a.a_mn = a_mn;
+    a.b_mn = b_mn;
+    a.ti_tiles = (N + 255) / 256;
+    a.tj_tiles = (N + 255) / 256;
+    a.total_tiles = kC * a.ti_tiles * a.tj_tiles;
+    a.kblocks = (N + 63) / 64;
+    a.ctl = ctl;
+    const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
+    return cuda_rc(launch_contract_tc(m, a, 2 * pairs, s), "contract_tc launch");
+}
+
 int run_contract(const trimul_params *p, int direction, const DevState &d, cudaStream_t s) {
     const Views v = views_of(p);
     if (p->dtype == TRIMUL_DTYPE_F32)
         return cuda_rc(launch_contract_f32(f32_layer(p, nullptr, v), direction, s), "contract_f32 launch");
-    // CTA pairs share each 256 x 256 output tile: CTA r loads rows [128 r, 128 r + 128)
-    // of the A and B panels (boxes of 128 rows, or 2 x 64-wide blocks when MN-major).
-    ContractMaps m;
-    if (direction == TRIMUL_OUTGOING) {
-        if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    } else {
-        if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-        if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    }
-    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    ContractArgs a;
-    a.N = p->N;
-    a.incoming = direction == TRIMUL_INCOMING;
-    a.ti_tiles = (p->N + 255) / 256;
-    a.tj_tiles = (p->N + 255) / 256;
-    a.total_tiles = kC * a.ti_tiles * a.tj_tiles;
-    a.kblocks = (p->N + 63) / 64;
-    a.ctl = ctl_of(p, v);
-    const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
-    return cuda_rc(launch_contract_tc(m, a, 2 * pairs, s), "contract_tc launch");
+    const int mn = direction == TRIMUL_INCOMING;
+    return run_contract_on(v.a, mn, v.b, mn, v.x, p->N, v.ld, ctl_of(p, v), d, s);
 }
 
 int run_epilogue(const void *z, const trimul_params *p, void *out, const DevState &d, cudaStream_t s) {
@@ -553,8 +558,6 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     bf *dA = reinterpret_cast<bf *>(base + L.dA), *dB = reinterpret_cast<bf *>(base + L.dB);
     float *partial = reinterpret_cast<float *>(base + L.partial);
     const bf *x = reinterpret_cast<const bf *>(v.x);
-    const int ld = (int)v.ld;
-    const long long cs = (long long)N * ld;  // channel stride of [128][N][ld]
     int rc;
 
     // Recompute the forward's a, b and x into the forward workspace.
@@ -622,24 +625,24 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     lb.dbeta = sums + S_LN_OUT_B * C;
     if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
 
-    // The contraction's adjoint, one N x N x N product per channel (bf16 out):
-    //   outgoing (X = A B^T): dA = dX B,    dB = dX^T A
-    //   incoming (X = A^T B): dA = B dX^T,  dB = A dX
-    Gemm g = gemm1(false, false, N, N, N, nullptr, ld, nullptr, ld, nullptr, ld, false);
-    g.sA = g.sB = g.sC = cs;
-    g.batch = C;
-    const bf *a = reinterpret_cast<const bf *>(v.a), *b = reinterpret_cast<const bf *>(v.b);
-    Gemm ga1 = g, gb1 = g;
+    // The contraction's adjoint on the forward's contraction kernel, in the
+    // form X[m][n] = sum_k A(m, k) B(n, k) with each operand K- or MN-major:
+    //   outgoing (x_ij = sum_k a_ik b_jk):
+    //     dA[i][k] = sum_j dX[i][j] b[j][k]   A = dX (K-major), B = b (MN-major)
+    //     dB[j][k] = sum_i dX[i][j] a[i][k]   A = dX (MN-major), B = a (MN-major)
+    //   incoming (x_ij = sum_k a_ki b_kj):
+    //     dA[k][i] = sum_j b[k][j] dX[i][j]   A = b (K-major), B = dX (K-major)
+    //     dB[k][j] = sum_i a[k][i] dX[i][j]   A = a (K-major), B = dX (MN-major)
+    const KernelCtl ctl = ctl_of(p, v);
     if (direction == TRIMUL_OUTGOING) {
-        ga1.A = dX, ga1.B = b;
-        gb1.ta = true, gb1.A = dX, gb1.B = a;
+        if ((rc = run_contract_on(dX, 0, v.b, 1, dA, N, v.ld, ctl, d, s)) ||
+            (rc = run_contract_on(dX, 1, v.a, 1, dB, N, v.ld, ctl, d, s)))
+            return rc;
     } else {
-        ga1.tb = true, ga1.A = b, ga1.B = dX;
-        gb1.A = a, gb1.B = dX;
+        if ((rc = run_contract_on(v.b, 0, dX, 0, dA, N, v.ld, ctl, d, s)) ||
+            (rc = run_contract_on(v.a, 0, dX, 1, dB, N, v.ld, ctl, d, s)))
+            return rc;
     }
-    ga1.C = dA;
-    gb1.C = dB;
-    if ((rc = gemm(h, ga1)) || (rc = gemm(h, gb1))) return rc;
 
     ProjBwdArgs pa;
     pa.dA = dA;

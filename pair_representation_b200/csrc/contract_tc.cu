@@ -5,7 +5,11 @@
 // biomolecular modeling with context parallelism in NVIDIA BioNeMo", section
 // "Context-parallel implementation of triangle multiplication"), computed by
 // pairs of CTAs on neighbouring SMs (a cluster of 2) that share one
-// 256 x 256 output tile through tcgen05.mma.cta_group::2:
+// 256 x 256 output tile through tcgen05.mma.cta_group::2. In general form
+// X[m][n] = sum_k A(m, k) B(n, k), each operand stored K-major ([rows][k]) or
+// MN-major ([k][rows]) as ContractArgs says: both K-major is the outgoing
+// product, both MN-major the incoming one, and the mixed forms serve the
+// backward's adjoint products.
 //   * CTA r of the pair loads rows [128 r, 128 r + 128) of the tile's A panel
 //     and rows [128 r, 128 r + 128) of its B panel (its half of N) into its own
 //     shared memory, 16 KB + 16 KB per 64-deep K block, 6 stages;
@@ -148,12 +152,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
                     const uint32_t bar = full0 + (uint32_t)(stage * 8);
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const int k0 = kb * BK;
-                    if (!args.incoming) {
+                    // K-major operand [rows][k]: one box of 64 k x 128 rows. MN-major operand
+                    // [k][rows]: two boxes of 64 rows x 64 k.
+                    if (!args.a_mn) {
                         tma_load_3d_pair(sa, &tmA, bar, k0, i0, c);
-                        tma_load_3d_pair(sb, &tmB, bar, k0, j0, c);
                     } else {
                         tma_load_3d_pair(sa, &tmA, bar, i0, k0, c);
                         tma_load_3d_pair(sa + BK * 128, &tmA, bar, i0 + 64, k0, c);
+                    }
+                    if (!args.b_mn) {
+                        tma_load_3d_pair(sb, &tmB, bar, k0, j0, c);
+                    } else {
                         tma_load_3d_pair(sb, &tmB, bar, j0, k0, c);
                         tma_load_3d_pair(sb + BK * 128, &tmB, bar, j0 + 64, k0, c);
                     }
@@ -189,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ---------------- MMA issuer (CTA 0) ----------------
-            const uint32_t idesc = idesc_bf16(256, BN, args.incoming, args.incoming);
+            const uint32_t idesc = idesc_bf16(256, BN, args.a_mn, args.b_mn);
             const bool stall = (ctl.debug_flags & 0x1u) != 0;
             int stage = 0;
             uint32_t phase = 0;
@@ -218,14 +227,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
                     const uint32_t sb = sa + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        uint64_t ad, bd;
-                        if (!args.incoming) {
-                            ad = sdesc_sw128(sa + kk * 32, 16, 1024);
-                            bd = sdesc_sw128(sb + kk * 32, 16, 1024);
-                        } else {
-                            ad = sdesc_sw128(sa + kk * 2048, BK * 128, 1024);
-                            bd = sdesc_sw128(sb + kk * 2048, BK * 128, 1024);
-                        }
+                        const uint64_t ad = args.a_mn ? sdesc_sw128(sa + kk * 2048, BK * 128, 1024)
+                                                      : sdesc_sw128(sa + kk * 32, 16, 1024);
+                        const uint64_t bd = args.b_mn ? sdesc_sw128(sb + kk * 2048, BK * 128, 1024)
+                                                      : sdesc_sw128(sb + kk * 32, 16, 1024);
                         mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[stage]);

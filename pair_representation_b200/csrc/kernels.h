@@ -33,7 +33,7 @@ struct PrologueMaps {
 
 struct ContractArgs {
     int N;
-    int incoming;
+    int a_mn, b_mn;   // operand storage: 0 = K-major [rows][k], 1 = MN-major [k][rows]
     int ti_tiles;     // ceil(N / 256)
     int tj_tiles;     // ceil(N / 256)
     int total_tiles;  // 128 * ti_tiles * tj_tiles
@@ -42,7 +42,7 @@ struct ContractArgs {
 };
 
 struct ContractMaps {
-    CUtensorMap a, b;  // outgoing: box (64 k, 128 rows, 1); incoming: box (64 rows, 64 k, 1); swizzle 128B
+    CUtensorMap a, b;  // K-major: box (64 k, 128 rows, 1); MN-major: box (64 rows, 64 k, 1); swizzle 128B
     CUtensorMap x;     // 3-D (j, i, c) over x, box (64, 128, 1), swizzle 128B
 };
 
