@@ -34,11 +34,12 @@ STATUS = {
 }
 ERR = {v: k for k, v in STATUS.items()}
 
-# Every symbol include/trimul.h declares.
+# Every symbol include/trimul.h and include/atomattn.h declare.
 EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forward", "trimul_prologue",
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
            "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
-           "trimul_backward", "trimul_backward_workspace_size")
+           "trimul_backward", "trimul_backward_workspace_size",
+           "atomattn_forward", "atomattn_workspace_size", "atomattn_device_status")
 
 # Gradient outputs of trimul_grads, in struct order; each is "d_" + a TrimulParams field.
 GRAD_FIELDS = ("d_w_a", "d_w_ag", "d_w_b", "d_w_bg", "d_w_g", "d_w_o", "d_b_a", "d_b_ag", "d_b_b", "d_b_bg",
@@ -80,6 +81,17 @@ class TrimulGrads(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class AtomAttnParams(ctypes.Structure):
+    """Mirror of ``atomattn_params`` in include/atomattn.h."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int), ("n_atoms", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("bias", ctypes.c_void_p), ("atom_mask", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t), ("timeout_ms", ctypes.c_uint32),
+    ]
+
+
 _lib = None
 
 
@@ -112,8 +124,14 @@ def lib():
         L.trimul_backward_workspace_size.argtypes = [I, I, I]
         L.trimul_backward_workspace_size.restype = S
         L.trimul_backward.argtypes = [P, P, PP, I, P, P, ctypes.POINTER(TrimulGrads), P]
+        AP = ctypes.POINTER(AtomAttnParams)
+        L.atomattn_workspace_size.argtypes = []
+        L.atomattn_workspace_size.restype = S
+        L.atomattn_forward.argtypes = [AP, P, P]
+        L.atomattn_device_status.argtypes = [AP, P, ctypes.POINTER(ctypes.c_int)]
         for f in ("trimul_forward", "trimul_forward_noalloc", "trimul_prologue", "trimul_contract", "trimul_epilogue",
-                  "trimul_workspace_views", "trimul_device_status", "trimul_version", "trimul_backward"):
+                  "trimul_workspace_views", "trimul_device_status", "trimul_version", "trimul_backward",
+                  "atomattn_forward", "atomattn_device_status"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -221,6 +239,51 @@ def trimul_device_status(params: TrimulParams, stream=None):
     d = (ctypes.c_int * 4)()
     rc = lib().trimul_device_status(ctypes.byref(params), _stream(stream), d)
     return rc, list(d)
+
+
+# ---- sequence-local atom attention -------------------------------------------
+
+def atomattn_workspace_size() -> int:
+    return lib().atomattn_workspace_size()
+
+
+def atomattn_forward(params: AtomAttnParams, out, stream=None, check=True) -> int:
+    rc = lib().atomattn_forward(ctypes.byref(params), _ptr(out), _stream(stream))
+    if check:
+        _check(rc, "atomattn_forward")
+    return rc
+
+
+def atomattn_device_status(params: AtomAttnParams, stream=None):
+    """(code, [code, site, block, aux]) of the status word (synchronises)."""
+    d = (ctypes.c_int * 4)()
+    rc = lib().atomattn_device_status(ctypes.byref(params), _stream(stream), d)
+    return rc, list(d)
+
+
+def atom_attention(q, k, v, bias=None, atom_mask=None, out=None, workspace=None, stream=None):
+    """Windowed atom attention (include/atomattn.h) on bf16 device tensors.
+
+    q, k, v: [batch][n_atoms][heads][32]; bias: [batch][ceil(n_atoms/32)][heads][32][128]
+    or None; atom_mask: [batch][n_atoms] or None. Returns out (allocated if None)."""
+    import torch
+    if q.dim() != 4 or q.shape[-1] != 32 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be [batch, n_atoms, heads, 32] of one shape")
+    for t in (q, k, v, bias, atom_mask):
+        if t is not None and (t.dtype != torch.bfloat16 or not t.is_contiguous()):
+            raise ValueError("inputs must be contiguous bf16")
+    B, n, H, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.zeros(atomattn_workspace_size(), dtype=torch.uint8, device=q.device)
+    p = AtomAttnParams()
+    p.batch, p.n_atoms, p.heads, p.head_dim = B, n, H, 32
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.bias, p.atom_mask = _ptr(bias), _ptr(atom_mask)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    atomattn_forward(p, out, stream)
+    return out, p
 
 
 # ---- the layer as the pages use it ------------------------------------------

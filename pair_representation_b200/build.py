@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtrimul_b200.so")
 SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu", "noalloc.cu",
-           "backward.cu", "blas.cu"]
+           "backward.cu", "blas.cu", "atomattn_tc.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tile_ops.cuh"]
 
 
@@ -33,7 +33,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "trimul.h")]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [
+        os.path.join(ROOT, "include", h) for h in ("trimul.h", "atomattn.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "atomattn.h"
 #include "kernels.h"
 #include "trimul.h"
 
@@ -73,8 +74,8 @@ int device_state(const DevState **out, bool need_tc) {
         }
         if (d.cc_major == 10 && d.cc_minor == 0) {
             if ((e = prologue_tc_setup()) == cudaSuccess && (e = contract_tc_setup()) == cudaSuccess &&
-                (e = epilogue_tc_setup()) == cudaSuccess)
-                e = backward_setup();
+                (e = epilogue_tc_setup()) == cudaSuccess && (e = backward_setup()) == cudaSuccess)
+                e = atomattn_tc_setup();
             d.tc_setup = e;
         } else {
             d.tc_setup = cudaErrorNoKernelImageForDevice;
@@ -709,6 +710,41 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     return TRIMUL_OK;
 }
 
+// ---- atom attention ------------------------------------------------------------------
+
+size_t attn_elems(const atomattn_params *p) { return (size_t)p->batch * p->n_atoms * p->heads * 32; }
+int attn_windows(const atomattn_params *p) { return (p->n_atoms + 31) / 32; }
+
+int check_attn(const atomattn_params *p, const void *out) {
+    if (!p || !out || !p->q || !p->k || !p->v) return TRIMUL_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->n_atoms < 1 || p->heads < 1) return TRIMUL_ERR_INVALID_ARG;
+    if (p->batch > (1 << 20) || p->n_atoms > (1 << 26)) return TRIMUL_ERR_INVALID_ARG;
+    if (p->head_dim != 32 || p->heads > 64 || (p->heads & 1)) return TRIMUL_ERR_UNSUPPORTED;
+    const void *al16[] = {p->q, p->k, p->v, p->bias, out};
+    for (const void *v : al16)
+        if (v && !aligned(v, 16)) return TRIMUL_ERR_MISALIGNED;
+    if (p->atom_mask && !aligned(p->atom_mask, 2)) return TRIMUL_ERR_MISALIGNED;
+    if (!p->workspace || p->workspace_bytes < atomattn_workspace_size()) return TRIMUL_ERR_WORKSPACE;
+    if (!aligned(p->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
+    const size_t n = attn_elems(p) * 2;
+    const size_t nb = (size_t)p->batch * attn_windows(p) * p->heads * 32 * 128 * 2;
+    const size_t nm = (size_t)p->batch * p->n_atoms * 2;
+    if (overlap(out, n, p->q, n) || overlap(out, n, p->k, n) || overlap(out, n, p->v, n) ||
+        overlap(out, n, p->bias, nb) || overlap(out, n, p->atom_mask, nm) ||
+        overlap(out, n, p->workspace, p->workspace_bytes))
+        return TRIMUL_ERR_ALIAS;
+    return TRIMUL_OK;
+}
+
+// q, k or v [batch][n][heads][32] as (heads * 32, n, batch): boxes of 64 elements (a head pair) x `rows`.
+int map_attn(CUtensorMap *m, const void *t, const atomattn_params *p, uint32_t rows) {
+    const uint64_t row = (uint64_t)p->heads * 32;
+    const uint64_t dims[3] = {row, (uint64_t)p->n_atoms, (uint64_t)p->batch};
+    const uint64_t strides[2] = {row * 2, row * 2 * (uint64_t)p->n_atoms};
+    const uint32_t box[3] = {64, rows, 1};
+    return encode(m, 3, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 }  // namespace
 
 // ---- exported symbols -------------------------------------------------------------
@@ -825,6 +861,59 @@ int trimul_backward(const void *z, const void *mask, const trimul_params *p, int
     rc = run_backward(z, mask, p, direction, dout, dz, g, *d, reinterpret_cast<cudaStream_t>(stream));
     blas_unlock();
     return rc;
+}
+
+size_t atomattn_workspace_size(void) { return kHeader; }
+
+int atomattn_forward(const atomattn_params *p, void *out, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_attn(p, out))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    const void *ptrs[] = {p->q, p->k, p->v, p->bias, p->atom_mask, p->workspace, out};
+    for (const void *v : ptrs)
+        if ((rc = check_device_ptr(v, "atom attention pointer"))) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = cuda_rc(cudaMemsetAsync(p->workspace, 0, sizeof(DeviceStatus), s), "status clear"))) return rc;
+    AttnMaps m;
+    if ((rc = map_attn(&m.q, p->q, p, 128)) || (rc = map_attn(&m.k, p->k, p, 224)) ||
+        (rc = map_attn(&m.v, p->v, p, 256)))
+        return rc;
+    AttnArgs a;
+    a.batch = p->batch;
+    a.n = p->n_atoms;
+    a.heads = p->heads;
+    a.groups = (p->n_atoms + 127) / 128;
+    a.n_windows = attn_windows(p);
+    a.units = (long long)p->batch * p->heads * a.groups;
+    a.bias = static_cast<const __nv_bfloat16 *>(p->bias);
+    a.mask = static_cast<const __nv_bfloat16 *>(p->atom_mask);
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.scale = 0.17677669529663687f;  // 1 / sqrt(32)
+    a.ctl.status = static_cast<DeviceStatus *>(p->workspace);
+    a.ctl.timeout_ns = (unsigned long long)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
+    a.ctl.debug_flags = 0;
+    const int grid = a.units < d->sms ? (int)a.units : d->sms;
+    return cuda_rc(launch_atomattn_tc(m, a, grid, s), "atomattn_tc launch");
+}
+
+int atomattn_device_status(const atomattn_params *p, trimul_stream_t stream, int *detail) {
+    if (!p || !p->workspace) return TRIMUL_ERR_INVALID_ARG;
+    DeviceStatus st;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaMemcpy(&st, p->workspace, sizeof st, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        set_detail("status read", e);
+        return TRIMUL_ERR_CUDA;
+    }
+    if (detail) {
+        detail[0] = st.code;
+        detail[1] = st.site;
+        detail[2] = st.block;
+        detail[3] = st.aux;
+    }
+    if (st.code == DEV_OK) return TRIMUL_OK;
+    return st.code == DEV_TIMEOUT ? TRIMUL_ERR_TIMEOUT : TRIMUL_ERR_DEVICE;
 }
 
 const char *trimul_error_string(int code) {

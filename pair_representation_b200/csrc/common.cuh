@@ -17,7 +17,7 @@ enum DeviceCode : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_FAULT = 2 };
 
 // Where a wait gave up: kernel id * 16 + site.
 enum Site : int {
-    SITE_PRO = 0x10, SITE_CON = 0x20, SITE_EPI = 0x30,
+    SITE_PRO = 0x10, SITE_CON = 0x20, SITE_EPI = 0x30, SITE_ATT = 0x40,
 };
 
 struct DeviceStatus {

@@ -188,6 +188,28 @@ int blas_bind(cudaStream_t s, void *ws, size_t ws_bytes, void **handle, char *de
 // Returns 0, or the cuBLAS status with a message in detail.
 int blas_gemm(void *handle, const Gemm &g, char *detail, size_t detail_n);
 
+// ---- sequence-local atom attention (atomattn_tc.cu) ---------------------------
+
+struct AttnArgs {
+    int batch, n, heads;
+    int groups;      // ceil(n / 128): units of 4 windows per (batch, head)
+    int n_windows;   // ceil(n / 32)
+    long long units; // batch * heads * groups
+    const __nv_bfloat16 *bias;  // [batch][n_windows][heads][32][128] or null
+    const __nv_bfloat16 *mask;  // [batch][n] or null
+    __nv_bfloat16 *out;         // [batch][n][heads][32]
+    float scale;                // 1 / sqrt(32)
+    KernelCtl ctl;
+};
+
+struct AttnMaps {
+    CUtensorMap q, k, v;  // 3-D (heads * 32, n, batch), boxes (64, 128 | 224 | 256, 1), swizzle 128B
+};
+
+size_t atomattn_tc_smem();
+cudaError_t atomattn_tc_setup();
+cudaError_t launch_atomattn_tc(const AttnMaps &m, const AttnArgs &a, int grid, cudaStream_t s);
+
 // ---- fp32 CUDA-core path ----------------------------------------------------
 
 struct F32Layer {

@@ -20,9 +20,13 @@ def L():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "trimul.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(trimul_[a-z_]+)\s*\(", src)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b((?:trimul|atomattn)_[a-z_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
@@ -245,3 +249,49 @@ def test_backward_reaches_cuda_and_fails_loudly_without_gpu(L):
     for f in tm.GRAD_FIELDS:
         setattr(q, f, None)  # every gradient output skipped: still a valid call
     assert _bwd(p, q) in (tm.ERR["TRIMUL_ERR_CUDA"], tm.ERR["TRIMUL_ERR_UNSUPPORTED"])
+
+
+# ---- atom attention -------------------------------------------------------------
+
+def _attn(B=2, n=100, H=4):
+    p = tm.AtomAttnParams()
+    p.batch, p.n_atoms, p.heads, p.head_dim = B, n, H, 32
+    p.q, p.k, p.v = BASE + 0x1000000, BASE + 0x2000000, BASE + 0x3000000
+    p.bias, p.atom_mask = BASE + 0x4000000, BASE + 0x5000000
+    p.workspace, p.workspace_bytes = BASE + 0x6000000, tm.atomattn_workspace_size()
+    return p
+
+
+AOUT = BASE + 0x7000000
+
+
+def test_atomattn_argument_checks(L):
+    E = tm.ERR
+    f = lambda p, out=AOUT: tm.atomattn_forward(p, out, stream=0, check=False)
+    assert tm.atomattn_workspace_size() == 256
+    assert tm.lib().atomattn_forward(None, AOUT, None) == E["TRIMUL_ERR_INVALID_ARG"]
+    assert f(_attn(), out=None) == E["TRIMUL_ERR_INVALID_ARG"]
+    for field, val, code in (("batch", 0, "INVALID_ARG"), ("n_atoms", 0, "INVALID_ARG"), ("heads", 0, "INVALID_ARG"),
+                             ("head_dim", 64, "UNSUPPORTED"), ("heads", 3, "UNSUPPORTED"),
+                             ("heads", 66, "UNSUPPORTED"), ("q", None, "INVALID_ARG"),
+                             ("k", BASE + 8, "MISALIGNED"), ("bias", BASE + 0x4000008, "MISALIGNED"),
+                             ("atom_mask", BASE + 1, "MISALIGNED"), ("workspace", None, "WORKSPACE"),
+                             ("workspace_bytes", 255, "WORKSPACE"), ("workspace", BASE + 0x6000010, "MISALIGNED")):
+        p = _attn()
+        setattr(p, field, val)
+        assert f(p) == E["TRIMUL_ERR_" + code], (field, val)
+    assert f(_attn(), out=AOUT + 8) == E["TRIMUL_ERR_MISALIGNED"]
+    p = _attn()
+    assert f(p, out=p.q) == E["TRIMUL_ERR_ALIAS"]
+    assert f(p, out=p.bias + 4096) == E["TRIMUL_ERR_ALIAS"]
+    assert f(p, out=p.workspace - 2 * 100 * 4 * 32 * 2 + 16) == E["TRIMUL_ERR_ALIAS"]
+    q = _attn()
+    q.bias = None
+    q.atom_mask = None  # optional inputs: still a valid call
+    try:
+        import torch
+        gpu = torch.cuda.is_available()
+    except ImportError:
+        gpu = False
+    if not gpu:
+        assert f(q) in (E["TRIMUL_ERR_CUDA"], E["TRIMUL_ERR_UNSUPPORTED"])
