@@ -14,8 +14,9 @@ With N > 1 (launched by torchrun) every rank runs an independent replica on its
 own GPU (the layer is not sharded); value = cells of all ranks / max time.
 
 Secondary figures on rank 0 at N = 1: every workload per direction
-("per_config") and one trimul_backward call per direction at N = 768
-("backward"; --backward-only times just that).
+("per_config"), one trimul_backward call per direction at N = 768
+("backward"; --backward-only times just that) and one windowed atom-attention
+call on 8 x 18432 atoms ("atom_attention"; --attention-only).
 
 Timing: CUDA events on the launching stream; L2 is flushed (512 MB write)
 before every step and the flush is outside the timed events; a barrier and a
@@ -303,6 +304,86 @@ def backward_timings(tm, pi, torch, dev, stream, peaks, warmup=3, reps=7):
     return res
 
 
+ATTN_SHAPE = {"batch": 8, "n_atoms": 768 * 24, "heads": 4, "head_dim": 32}
+
+
+def attention_inputs(B, n, H, seed=5):
+    """Synthetic q, k, v, bias ~ N(0, 1) and an atom mask with a padded tail (5 %), as bf16-valued numpy."""
+    import numpy as np
+    rng = np.random.default_rng([seed, 31])
+    q, k, v = (rng.standard_normal((B, n, H, 32), dtype=np.float32) for _ in range(3))
+    bias = rng.standard_normal((B, (n + 31) // 32, H, 32, 128), dtype=np.float32)
+    mask = np.ones((B, n), dtype=np.float32)
+    mask[:, n - n // 20:] = 0
+    return q, k, v, bias, mask
+
+
+def attention_timings(tm, torch, dev, stream, peaks, warmup=3, reps=10):
+    """Secondary figure: windowed atom attention (atomattn_forward) on 8 x 18432 atoms
+    (a 768-token crop at 24 atoms per token, 8 samples), 4 heads of 32, with bias and
+    mask; CUDA events, L2 flushed before each call; the float64 oracle timed on
+    batch element 0 (all its windows and heads)."""
+    import numpy as np
+    from oracle.atomattn import atom_attention as oracle_attention
+    B, n, H = ATTN_SHAPE["batch"], ATTN_SHAPE["n_atoms"], ATTN_SHAPE["heads"]
+    arrs = attention_inputs(B, n, H)
+    t = [torch.from_numpy(a).to(dev).to(torch.bfloat16) for a in arrs]
+    q, k, v, bias, mask = t
+    out = torch.empty_like(q)
+    ws = torch.zeros(tm.atomattn_workspace_size(), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        tm.atom_attention(q, k, v, bias, mask, out=out, workspace=ws, stream=stream)
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tm.atom_attention(q, k, v, bias, mask, out=out, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    med = ts[len(ts) // 2]
+    W = (n + 31) // 32
+    # Minimum HBM bytes: q, k, v read and out written once, bias and mask read once.
+    min_bytes = 4 * B * n * H * 32 * 2 + B * W * H * 32 * 128 * 2 + B * n * 2
+    flops = B * W * H * 2 * (32 * 128 * 32 * 2)  # S = Q K^T and O = P V per window
+    # Oracle on a bounded sample: batch element 0.
+    na = n
+    sample = [a[:1] for a in arrs]
+    t0 = time.perf_counter()
+    oracle_attention(*[np.asarray(x, dtype=np.float64) for x in sample])
+    osec = time.perf_counter() - t0
+    res = {"shape": dict(ATTN_SHAPE, bias=True, atom_mask="last 5 % padded"), "dtype": "bf16",
+           "median_us": round(med, 1), "best_us": round(ts[0], 1),
+           "atoms_per_s": round(B * n / (med * 1e-6)),
+           "min_bytes": min_bytes, "min_bytes_gbs": round(min_bytes / (med * 1e-6) / 1e9, 1),
+           "frac_of_hbm_peak": round(min_bytes / (med * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+           "tflops": round(flops / (med * 1e-6) / 1e12, 1),
+           "cpu_oracle": {"atoms_per_s": round(na / osec), "sample": f"{na} atoms x {H} heads of batch element 0",
+                          "kind": "oracle", "seconds": round(osec, 2)}}
+    del q, k, v, bias, mask, out, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_attention_only(args):
+    """--attention-only: the atom-attention secondary figure alone, on one GPU."""
+    import torch
+
+    import pair_representation_b200 as tm
+    from pair_representation_b200 import build as tmbuild
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tmbuild.build()
+    tm.lib()
+    peaks, _ = load_peaks()
+    res = attention_timings(tm, torch, dev, torch.cuda.current_stream(dev), peaks, args.warmup, args.steps)
+    print(json.dumps({"atom_attention": res}), flush=True)
+
+
 def run_backward_only(args):
     """--backward-only: the backward secondary figure alone, on one GPU."""
     import torch
@@ -486,6 +567,9 @@ def run_ours(args, rank, world, local_rank):
         configs = per_config_timings(tm, pi, torch, dev, stream)
     if rank == 0 and world == 1 and not args.no_backward:
         backward = backward_timings(tm, pi, torch, dev, stream, peaks)
+    attention = None
+    if rank == 0 and world == 1 and not args.no_attention:
+        attention = attention_timings(tm, torch, dev, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -503,6 +587,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
         "per_config": configs,
         "backward": backward,
+        "atom_attention": attention,
     }
     if dist:
         dist.barrier()
@@ -556,6 +641,9 @@ def main(argv=None):
     ap.add_argument("--no-backward", action="store_true", help="skip the backward secondary timing")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only trimul_backward (W warm-up and K timed calls per direction) and print that")
+    ap.add_argument("--no-attention", action="store_true", help="skip the atom-attention secondary timing")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time only atomattn_forward (W warm-up and K timed calls) and print that")
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=120.0)
     args = ap.parse_args(argv)
@@ -570,6 +658,8 @@ def main(argv=None):
         run_reference(args, rank, world)
     elif args.backward_only:
         run_backward_only(args)
+    elif args.attention_only:
+        run_attention_only(args)
     else:
         run_ours(args, rank, world, local_rank)
 

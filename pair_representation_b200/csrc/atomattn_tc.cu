@@ -13,7 +13,7 @@
 // [32 (r / 32), 32 (r / 32) + 128) of S; its softmax runs in the thread that
 // owns TMEM lane r, and its probabilities go to shared memory as row r of a
 // [128][256] K-major operand P whose other slots stay 0. Then
-//   O[128][64] = P V               (tcgen05, TMEM columns [256, 320))
+//   O[128][64] = P V               (tcgen05, TMEM columns [256, 320) or [320, 384) by unit parity)
 // over 256 key rows (slots 224 .. 255 have P = 0).
 //
 // Q, K and V are TMA-loaded as rows of 64 bf16: the head pair (h & ~1, h | 1),
@@ -21,12 +21,12 @@
 // head's 32 of them (the K steps at byte offset 64 (h & 1)), and O's columns
 // [32 (h & 1), 32 (h & 1) + 32) are the head's output.
 //
-// Warps 0-3: softmax and epilogue (thread = query row = TMEM lane). Warp 4,
-// one thread: TMA loads (double-buffered stages) and MMA issue. Barriers, all
-// waits bounded:
+// Warps 0-15: softmax and epilogue; warp w serves the query rows of TMEM lane
+// quarter w & 3 and a quarter of their slots. Warp 16, one thread: TMA loads
+// (double-buffered stages) and MMA issue. Barriers, all waits bounded:
 //   full[s]  TMA bytes of stage s landed              (producer -> MMA)
 //   sfull    S of the unit is in TMEM                  (MMA commit -> warps 0-3)
-//   pready   P written, S and the previous O read      (4 warp arrivals -> MMA)
+//   pready   P written, S and the O of two units back read (16 warp arrivals -> MMA)
 //   ofull    O of the unit is in TMEM, stage free      (MMA commit -> warps 0-3, producer)
 #include "kernels.h"
 
@@ -46,9 +46,11 @@ constexpr int STAGE_BYTES = Q_BYTES + K_BYTES + V_BYTES;
 constexpr int P_BLOCK = ROWS * 128;          // one 64-slot block of P (16 KB)
 constexpr int P_BYTES = 4 * P_BLOCK;
 constexpr int S_COL = 0, O_COL = 256, TMEM_COLS = 512;
-constexpr int THREADS = 160;
-constexpr int BAR_BYTES = 128;
-constexpr size_t SMEM = 1024 + 2 * (size_t)STAGE_BYTES + P_BYTES + BAR_BYTES;
+constexpr int WORKER_WARPS = 16;             // 4 per TMEM lane quarter, 32 of a row's 128 slots each
+constexpr int THREADS = (WORKER_WARPS + 1) * 32;
+constexpr int RED_BYTES = 2 * 2 * 4 * ROWS * 4;  // [max, sum][unit parity][key part][row] floats
+constexpr int BAR_BYTES = 128;  // 10 mbarriers, TMEM address, abort flag
+constexpr size_t SMEM = 1024 + 2 * (size_t)STAGE_BYTES + P_BYTES + RED_BYTES + BAR_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace aa
@@ -64,16 +66,44 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// 16-byte load on the read-only path, kept where it is written (an early
+// prefetch that the compiler must not sink to the first use).
+__device__ __forceinline__ uint4 ldg_early(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_early_u16(const uint16_t *p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// Unit u = (b * heads + h) * groups + g. A CTA visits u = blockIdx.x + lu * gridDim.x;
+// the decode is done once and then stepped without division.
 struct Unit {
     int b, h, g;
 };
-__device__ __forceinline__ Unit unit_of(long long u, const AttnArgs &a) {
+__device__ __forceinline__ Unit unit_of(int u, const AttnArgs &a) {
     Unit x;
-    x.g = (int)(u % a.groups);
-    const long long t = u / a.groups;
-    x.h = (int)(t % a.heads);
-    x.b = (int)(t / a.heads);
+    x.g = u % a.groups;
+    const int t = u / a.groups;
+    x.h = t % a.heads;
+    x.b = t / a.heads;
     return x;
+}
+__device__ __forceinline__ void unit_step(Unit &x, const AttnArgs &a) {
+    x.g += gridDim.x;
+    while (x.g >= a.groups) {
+        x.g -= a.groups;
+        if (++x.h == a.heads) {
+            x.h = 0;
+            ++x.b;
+        }
+    }
 }
 
 }  // namespace
@@ -86,13 +116,15 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stage_base = smem;
     uint8_t *pbuf = smem + 2 * STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(pbuf + P_BYTES);
+    float *red = reinterpret_cast<float *>(pbuf + P_BYTES);  // [2][2][4][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(pbuf + P_BYTES + RED_BYTES);
     uint64_t *full = bars;        // [2]
     uint64_t *sfull = bars + 2;
     uint64_t *pready = bars + 3;
     uint64_t *ofull = bars + 4;
     uint64_t *drain = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint64_t *redbar = bars + 6;  // [4] per lane quarter: its 4 warps published their partials
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,9 +136,10 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
         mbar_init(sfull, 1);
-        mbar_init(pready, 4);
+        mbar_init(pready, WORKER_WARPS);
         mbar_init(ofull, 1);
         mbar_init(drain, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&redbar[i], 4);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -118,25 +151,27 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         tmem_relinquish();
     }
     const uint32_t pbase = smem_u32(pbuf);
-    if (warp < 4) {
-        // P slots outside the row's window are 0 for every unit: write them once.
-        const int row = threadIdx.x, q = warp;
-        for (int cu = 0; cu < 32; ++cu)
-            if (cu < 4 * q || cu >= 4 * q + 16) st_shared_v4(p_chunk_addr(pbase, row, cu), 0u, 0u, 0u, 0u);
+    if (warp < WORKER_WARPS) {
+        // P slots outside the row's window are 0 for every unit: write them once
+        // (the four warps of a lane quarter split the chunks).
+        const int qr = warp & 3, kp = warp >> 2, row = qr * 32 + lane;
+        for (int cu = kp; cu < 32; cu += 4)
+            if (cu < 4 * qr || cu >= 4 * qr + 16) st_shared_v4(p_chunk_addr(pbase, row, cu), 0u, 0u, 0u, 0u);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == WORKER_WARPS) {
         if (lane == 0) {
             // ---------------- TMA producer and MMA issuer ----------------
             const uint32_t idesc_s = idesc_bf16(128, UNION, 0, 0);
             const uint32_t idesc_o = idesc_bf16(128, 64, 0, 1);
+            const uint64_t pdesc = sdesc_sw128(pbase, 16, 1024);
             int issued = 0, landed = 0;
             auto issue = [&](int lu) {
-                const Unit un = unit_of(blockIdx.x + (long long)lu * gridDim.x, args);
+                const Unit un = unit_of((int)blockIdx.x + lu * (int)gridDim.x, args);
                 uint8_t *st = stage_base + (lu & 1) * STAGE_BYTES;
                 const int x = (un.h & ~1) * 32, a0 = un.g * ROWS;
                 mbar_arrive_expect_tx(&full[lu & 1], STAGE_BYTES);
@@ -150,7 +185,7 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                     return false;
                 ++landed;
                 tc_fence_after();
-                const Unit un = unit_of(blockIdx.x + (long long)lu * gridDim.x, args);
+                const Unit un = unit_of((int)blockIdx.x + lu * (int)gridDim.x, args);
                 const uint32_t st = smem_u32(stage_base + (lu & 1) * STAGE_BYTES);
                 const uint32_t kofs = (uint32_t)(un.h & 1) * 64;  // the head's 32 elements in the 64-element row
 #pragma unroll
@@ -170,11 +205,15 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t vst = smem_u32(stage_base + (lu & 1) * STAGE_BYTES) + Q_BYTES + K_BYTES;
+                // Descriptor start addresses count 16-byte units in their low bits:
+                // step K by adding to the descriptor.
+                const uint64_t vdesc = sdesc_sw128(smem_u32(stage_base + (lu & 1) * STAGE_BYTES) + Q_BYTES + K_BYTES,
+                                                   V_BYTES, 1024);
+                const uint32_t od = tmem + O_COL + 64 * (lu & 1);
 #pragma unroll
                 for (int kk = 0; kk < VROWS / 16; ++kk)
-                    mma_bf16(tmem + O_COL, sdesc_sw128(pbase + (kk >> 2) * P_BLOCK + (kk & 3) * 32, 16, 1024),
-                             sdesc_sw128(vst + kk * 2048, V_BYTES, 1024), idesc_o, kk ? 1u : 0u);
+                    mma_bf16(od, pdesc + (uint64_t)(((kk >> 2) * P_BLOCK + (kk & 3) * 32) >> 4),
+                             vdesc + (uint64_t)((kk * 2048) >> 4), idesc_o, kk ? 1u : 0u);
                 mma_commit(ofull);
                 if (lu + 1 < my_units && !(ok = mma_s(lu + 1))) break;
                 if (lu + 2 < my_units) {
@@ -194,93 +233,136 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         }
     } else {
         // ---------------- softmax and epilogue: thread = query row ----------------
-        const int q = warp, row = threadIdx.x;
-        const uint32_t lanebase = tmem + ((uint32_t)(q * 32) << 16);
+        // Warp (qr, kp) = (warp & 3, warp >> 2) owns query rows 32 qr .. 32 qr + 31
+        // (TMEM lane quarter qr) and slots 32 kp .. 32 kp + 31 of their window.
+        // Unit lu: its bias slice and key-mask value were loaded during unit lu - 1;
+        // logits stay in registers; partial row maxima and sums are exchanged
+        // among the quarter's 4 warps through `red` (double-buffered by unit
+        // parity) through one mbarrier phase per unit; P is written once the
+        // previous unit's second product has finished reading it; then that
+        // unit's output columns 8 kp .. 8 kp + 7 (O buffer (lu - 1) & 1) are stored.
+        const int qr = warp & 3, kp = warp >> 2, row = qr * 32 + lane;
+        const uint32_t lanebase = tmem + ((uint32_t)(qr * 32) << 16);
         const float log2e = 1.4426950408889634f;
-        for (int lu = 0; lu < my_units; ++lu) {
-            const Unit un = unit_of(blockIdx.x + (long long)lu * gridDim.x, args);
-            const int w = un.g * WPG + q;                 // this warp's window
-            const int atom_q = un.g * ROWS + row;         // this thread's query atom
-            const int k0 = w * QW + KOFF;                 // atom of key slot 0
-            // Bias row of this query (prefetched before S is ready).
-            uint4 bias[16];
-            const bool has_bias = args.bias != nullptr && w < args.n_windows;
-            if (has_bias) {
+        float *red_max = red, *red_sum = red + 2 * 4 * ROWS;
+        uint4 bias[4];
+        uint16_t mk_n = 0;
+        bool hb_n = false;
+        auto prefetch = [&](const Unit &un) {
+            const int w = un.g * WPG + qr, at = w * QW + KOFF + 32 * kp + lane;
+            hb_n = args.bias != nullptr && w < args.n_windows;
+            if (hb_n) {
                 const uint4 *bp = reinterpret_cast<const uint4 *>(
-                    args.bias + ((((size_t)un.b * args.n_windows + w) * args.heads + un.h) * QW + lane) * KW);
+                    args.bias + ((((size_t)un.b * args.n_windows + w) * args.heads + un.h) * QW + lane) * KW + 32 * kp);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) bias[i] = __ldg(bp + i);
+                for (int i = 0; i < 4; ++i) bias[i] = ldg_early(bp + i);
             }
-            // Key validity: lane l decides slots 4l .. 4l + 3; bit e of vb[e] (lane l) <- slot 4l + e.
-            uint32_t vb[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int a = k0 + 4 * lane + e;
-                bool ok = a >= 0 && a < args.n;
-                if (ok && args.mask) ok = __bfloat162float(args.mask[(size_t)un.b * args.n + a]) != 0.f;
-                vb[e] = __ballot_sync(0xffffffffu, ok);
-            }
-            if (!warp_wait(sfull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 4, lu)) break;
+            mk_n = (at < 0 || at >= args.n) ? (uint16_t)0
+                   : args.mask ? ldg_early_u16(reinterpret_cast<const uint16_t *>(args.mask) + (size_t)un.b * args.n + at)
+                               : (uint16_t)0x3f80u;  // bf16 1.0
+        };
+        Unit prev{0, 0, 0};
+        float sum_prev = 0.f;
+        bool ok = true;
+        auto epilogue = [&](int lu) {
+            // Output columns 8 kp .. 8 kp + 7 of unit lu (its second product has completed).
             tc_fence_after();
-            uint32_t s[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(lanebase + (uint32_t)(S_COL + 32 * q + 32 * c), s + 32 * c);
+            uint32_t o[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]),
+                           "=r"(o[7])
+                         : "r"(lanebase + (uint32_t)(O_COL + 64 * (lu & 1) + 32 * (prev.h & 1) + 8 * kp)));
             tmem_ld_wait();
-            // Logits in the log2 domain; invalid slots -inf.
-            float mx = -INFINITY;
+            const int atom_q = prev.g * ROWS + row;
+            if (atom_q < args.n) {
+                const float inv = sum_prev > 0.f ? 1.f / sum_prev : 0.f;
+                uint32_t pk[4];
 #pragma unroll
-            for (int j = 0; j < 128; ++j) {
-                float bj = 0.f;
-                if (has_bias) {
-                    const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bias[j >> 3]);
-                    const float2 f = __bfloat1622float2(bb[(j & 7) >> 1]);
-                    bj = (j & 1) ? f.y : f.x;
+                for (int t = 0; t < 4; ++t) {
+                    const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * t]) * inv,
+                                                                   __uint_as_float(o[2 * t + 1]) * inv);
+                    pk[t] = *reinterpret_cast<const uint32_t *>(&v);
                 }
-                const bool valid = (vb[j & 3] >> (j >> 2)) & 1u;
-                const float l = valid ? (__uint_as_float(s[j]) * args.scale + bj) * log2e : -INFINITY;
-                s[j] = __float_as_uint(l);
-                mx = fmaxf(mx, l);
+                *reinterpret_cast<uint4 *>(args.out + (((size_t)prev.b * args.n + atom_q) * args.heads + prev.h) * 32 +
+                                           8 * kp) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            const float m = mx == -INFINITY ? 0.f : mx;
-            float sum = 0.f;
+        };
+        Unit cur = unit_of((int)blockIdx.x, args);
+        if (my_units > 0) prefetch(cur);
+        for (int lu = 0; lu < my_units; ++lu) {
+            const Unit un = cur;
+            unit_step(cur, args);  // the next unit of this CTA
+            const bool hb = hb_n;
+            const uint32_t vb = __ballot_sync(0xffffffffu, (mk_n & 0x7fffu) != 0);  // slot 32 kp + i valid: bit i
+            if (!(ok = warp_wait(sfull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 4, lu))) break;
+            tc_fence_after();
+            // Logits of the 32 slots in the log2 domain (invalid: -inf) and their maximum.
+            float l[32];
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            {
+                uint32_t sv[32];
+                tmem_ld32(lanebase + (uint32_t)(S_COL + 32 * qr + 32 * kp), sv);
+                tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+                for (int t = 0; t < 32; ++t) {
+                    float bj = 0.f;
+                    if (hb) {
+                        const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bias[t >> 3]);
+                        const float2 f = __bfloat1622float2(bb[(t & 7) >> 1]);
+                        bj = (t & 1) ? f.y : f.x;
+                    }
+                    l[t] = ((vb >> t) & 1u) ? (__uint_as_float(sv[t]) * args.scale + bj) * log2e : -INFINITY;
+                    mx4[t & 3] = fmaxf(mx4[t & 3], l[t]);
+                }
+            }
+            if (lu + 1 < my_units) prefetch(cur);
+            float *rm = red_max + (lu & 1) * 4 * ROWS, *rs = red_sum + (lu & 1) * 4 * ROWS;
+            rm[kp * ROWS + row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&redbar[qr]);
+            if (!(ok = warp_wait(&redbar[qr], (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 7, lu))) break;
+            float mx = fmaxf(fmaxf(rm[row], rm[ROWS + row]), fmaxf(rm[2 * ROWS + row], rm[3 * ROWS + row]));
+            const float m = mx == -INFINITY ? 0.f : mx;
+            if (lu > 0) {
+                // The previous unit's row sum (its partial sums were published before this barrier).
+                const float *ps = red_sum + ((lu - 1) & 1) * 4 * ROWS;
+                sum_prev = ps[row] + ps[ROWS + row] + ps[2 * ROWS + row] + ps[3 * ROWS + row];
+            }
+            // P is free once the previous unit's second product has completed.
+            if (lu > 0 && !(ok = warp_wait(ofull, (uint32_t)(lu - 1) & 1u, abort_flag, ctl, SITE_ATT | 5, lu))) break;
+            // Probabilities (bf16), their partial sum, and this warp's 4 chunks of row `row` of P.
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     const int j = 8 * c + 2 * t;
-                    const __nv_bfloat162 pp =
-                        __floats2bfloat162_rn(exp2f(__uint_as_float(s[j]) - m), exp2f(__uint_as_float(s[j + 1]) - m));
+                    const __nv_bfloat162 pp = __floats2bfloat162_rn(exp2f(l[j] - m), exp2f(l[j + 1] - m));
                     const float2 pr = __bfloat1622float2(pp);
-                    sum += pr.x + pr.y;
+                    s4[t] += pr.x + pr.y;
                     pk[t] = *reinterpret_cast<const uint32_t *>(&pp);
                 }
-                st_shared_v4(p_chunk_addr(pbase, row, 4 * q + c), pk[0], pk[1], pk[2], pk[3]);
+                st_shared_v4(p_chunk_addr(pbase, row, 4 * qr + 4 * kp + c), pk[0], pk[1], pk[2], pk[3]);
             }
+            rs[kp * ROWS + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(pready);
-            if (!warp_wait(ofull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 5, lu)) break;
-            tc_fence_after();
-            uint32_t o[32];
-            tmem_ld32(lanebase + (uint32_t)(O_COL + 32 * (un.h & 1)), o);
-            tmem_ld_wait();
-            if (atom_q < args.n) {
-                const float inv = sum > 0.f ? 1.f / sum : 0.f;
-                uint4 *op = reinterpret_cast<uint4 *>(args.out + (((size_t)un.b * args.n + atom_q) * args.heads + un.h) * 32);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * t]) * inv,
-                                                                       __uint_as_float(o[8 * i + 2 * t + 1]) * inv);
-                        pk[t] = *reinterpret_cast<const uint32_t *>(&v);
-                    }
-                    op[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
+            if (lu > 0) epilogue(lu - 1);
+            prev = un;
+        }
+        if (ok && my_units > 0) {
+            // The last unit's partial sums.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&redbar[qr]);
+            ok = warp_wait(&redbar[qr], (uint32_t)my_units & 1u, abort_flag, ctl, SITE_ATT | 8, 0);
+        }
+        if (ok && my_units > 0) {
+            const float *ps = red_sum + ((my_units - 1) & 1) * 4 * ROWS;
+            sum_prev = ps[row] + ps[ROWS + row] + ps[2 * ROWS + row] + ps[3 * ROWS + row];
+            if (warp_wait(ofull, (uint32_t)(my_units - 1) & 1u, abort_flag, ctl, SITE_ATT | 6, 0)) epilogue(my_units - 1);
         }
     }
 
