@@ -252,10 +252,14 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             const int w = un.g * WPG + qr, at = w * QW + KOFF + 32 * kp + lane;
             hb_n = args.bias != nullptr && w < args.n_windows;
             if (hb_n) {
-                const uint4 *bp = reinterpret_cast<const uint4 *>(
-                    args.bias + ((((size_t)un.b * args.n_windows + w) * args.heads + un.h) * QW + lane) * KW + 32 * kp);
+                // Coalesced: instruction i reads rows 8i .. 8i + 7 of the warp's [32 rows][32 slots]
+                // slice, 64 contiguous bytes per row (lane l: row 8i + l / 4, 16-byte chunk l % 4).
+                // The rows reach their owning lanes (row = lane) by shuffles at first use.
+                const __nv_bfloat16 *slice =
+                    args.bias + (((size_t)un.b * args.n_windows + w) * args.heads + un.h) * QW * KW + 32 * kp;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) bias[i] = ldg_early(bp + i);
+                for (int i = 0; i < 4; ++i)
+                    bias[i] = ldg_early(reinterpret_cast<const uint4 *>(slice + (8 * i + (lane >> 2)) * KW + 8 * (lane & 3)));
             }
             mk_n = (at < 0 || at >= args.n) ? (uint16_t)0
                    : args.mask ? ldg_early_u16(reinterpret_cast<const uint16_t *>(args.mask) + (size_t)un.b * args.n + at)
@@ -297,6 +301,8 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             if (!(ok = warp_wait(sfull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 4, lu))) break;
             tc_fence_after();
             // Logits of the 32 slots in the log2 domain (invalid: -inf) and their maximum.
+            // Chunk c (slots 8c .. 8c + 7) of this lane's bias row sits in bias[lane / 8] of
+            // lane 4 (lane % 8) + c: fetched by shuffles right before its logits.
             float l[32];
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             {
@@ -304,15 +310,29 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 tmem_ld32(lanebase + (uint32_t)(S_COL + 32 * qr + 32 * kp), sv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    float bj = 0.f;
+                for (int c = 0; c < 4; ++c) {
+                    uint4 bc = make_uint4(0u, 0u, 0u, 0u);
                     if (hb) {
-                        const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bias[t >> 3]);
-                        const float2 f = __bfloat1622float2(bb[(t & 7) >> 1]);
-                        bj = (t & 1) ? f.y : f.x;
+                        const int src = 4 * (lane & 7) + c;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint4 t;
+                            t.x = __shfl_sync(0xffffffffu, bias[i].x, src);
+                            t.y = __shfl_sync(0xffffffffu, bias[i].y, src);
+                            t.z = __shfl_sync(0xffffffffu, bias[i].z, src);
+                            t.w = __shfl_sync(0xffffffffu, bias[i].w, src);
+                            if ((lane >> 3) == i) bc = t;
+                        }
                     }
-                    l[t] = ((vb >> t) & 1u) ? (__uint_as_float(sv[t]) * args.scale + bj) * log2e : -INFINITY;
-                    mx4[t & 3] = fmaxf(mx4[t & 3], l[t]);
+                    const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bc);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int t = 8 * c + u;
+                        const float2 f = __bfloat1622float2(bb[u >> 1]);
+                        const float bj = (u & 1) ? f.y : f.x;
+                        l[t] = ((vb >> t) & 1u) ? (__uint_as_float(sv[t]) * args.scale + bj) * log2e : -INFINITY;
+                        mx4[t & 3] = fmaxf(mx4[t & 3], l[t]);
+                    }
                 }
             }
             if (lu + 1 < my_units) prefetch(cur);
