@@ -3,9 +3,9 @@
 Bars (written in each test):
   fp32 path: rel-L2 <= 1e-4 on the layer output.
   bf16 path: rel-L2 <= 1.5e-2 and max-abs <= 5e-2 on the layer output.
-  bf16 stages (derived from bf16 storage of the stage outputs, unit roundoff
-  2^-9 = 2e-3 per element): prologue a, b and contraction x rel-L2 <= 1e-2,
-  max-abs <= 4 * 2^-9 * max|ref|.
+  bf16 stages (derived from bf16 storage of the stage outputs: 8 significant
+  bits, unit roundoff u = 2^-8, about 2^-9 on average): prologue a, b and
+  contraction x rel-L2 <= 1e-2, max-abs <= 4 * 2^-9 * max|ref| (= 2u).
 """
 import numpy as np
 import pytest
