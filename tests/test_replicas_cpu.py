@@ -68,3 +68,31 @@ def test_flop_and_byte_accounting():
     assert alg["contract_tc_kernel"][0] == 2 * N ** 3 * 128
     assert alg["prologue_tc_kernel"][0] == N * N * 770 + 131072
     assert alg["epilogue_tc_kernel"][0] == N * N * 768 + 65536
+
+
+def test_backward_and_attention_accounting():
+    """The secondary figures' work counts, restated from the shapes the steps run."""
+    N, c = 768, 128
+    gemm = lambda m, n, k: 2 * m * n * k
+    cells = N * N
+    per_call = (gemm(cells, 4 * c, c) + 2 * N ** 3 * c          # recomputed projections a, b and x
+                + gemm(cells, 5 * c, c) + gemm(cells, c, c)      # P and Y
+                + gemm(cells, c, c)                              # dL/dxh
+                + 2 * 2 * N ** 3 * c                             # contraction adjoint dA, dB
+                + gemm(6 * c, c, cells)                          # weight gradients (K = cells)
+                + gemm(cells, c, 5 * c))                         # dL/dzh
+    assert bench.backward_flops_per_cell(N) * cells == per_call
+    # minimum bytes per cell, bf16 = 2 B, fp32 = 4 B, stats 8 B
+    steps = [256 + 256 + 8, 256 + 256 + 8,             # LayerNorms
+             256 + 5 * 256, 256 + 256,                 # P (bf16 out), Y
+             256 + 256 + 256 + 256 + 256,              # gate adjoint: P_g, Y, dout in; dy, dP_g out
+             256 + 512,                                # dL/dxh (fp32 out)
+             512 + 256 + 8 + 256,                      # LN_out adjoint
+             2 * (256 + 256 + 256),                    # contraction adjoint
+             512 + 1024 + 2 + 1024,                    # input-gate adjoint
+             1280 + 256 + 256 + 256,                   # weight-gradient partials
+             1280 + 512,                               # dL/dzh
+             512 + 256 + 8 + 256]                      # LN_in adjoint
+    assert bench.BACKWARD_BYTES_PER_CELL == sum(steps)
+    B, n, H = bench.ATTN_SHAPE["batch"], bench.ATTN_SHAPE["n_atoms"], bench.ATTN_SHAPE["heads"]
+    assert (B, n, H, bench.ATTN_SHAPE["head_dim"]) == (8, 768 * 24, 4, 32)
