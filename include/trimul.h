@@ -121,7 +121,9 @@ int trimul_workspace_views(const trimul_params *p, void **a, void **b, void **x,
 /* Synchronises `stream`, then returns the status word the kernels wrote
  * since it was last cleared: TRIMUL_OK, TRIMUL_ERR_TIMEOUT or
  * TRIMUL_ERR_DEVICE (or TRIMUL_ERR_CUDA if reading it failed). If `detail` is
- * not NULL it receives 4 ints: code, site, block index, auxiliary value. */
+ * not NULL it receives 4 ints: code, site, block index, auxiliary value.
+ * With p->workspace NULL it reads the status word of the static scratch that
+ * trimul_forward_noalloc uses on the current device. */
 int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *detail);
 
 /* Static description of a status code. */
@@ -152,8 +154,9 @@ const char *trimul_last_error_detail(void);
  * overlaps, on different streams or from different host threads, race and
  * give wrong results. The first call with a given device current looks up
  * the array's device address for that device; make that first call before
- * any stream capture. trimul_device_status cannot read this scratch's status
- * word; an in-kernel timeout still leaves the output invalid. */
+ * any stream capture. trimul_device_status, given a params block whose
+ * workspace is NULL, reads the status word this entry point's kernels wrote
+ * (an in-kernel timeout leaves the output invalid and is reported there). */
 int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params *p, int direction,
                            void *out, trimul_stream_t stream);
 

@@ -195,15 +195,17 @@ def random_case(N: int, seed: int, c_z: int = 128, c_h: int = 128, bf16: bool = 
     return d
 
 
-def sample_grid(N: int, seed: int, n_random: int = 24, tile: int = 128) -> np.ndarray:
+def sample_grid(N: int, seed: int, n_random: int = 24, tile: int = 128, pair_tile: int = 256) -> np.ndarray:
     """Sorted residue indices for a sampled check: tile edges, ragged tail, random.
 
-    Used on both axes, so the sampled cells are the grid I x I: corners, every
-    128-tile boundary listed here, the last (ragged) tile, and random rows.
+    Used on both axes, so the sampled cells are the grid I x I: corners, the
+    first two 128-tile boundaries and those near the end, every boundary of a
+    256-wide pair tile (255/256, 511/512, 767/768, ...), the last (ragged)
+    tile, and random rows.
     """
     s = {0, 1, N - 2, N - 1}
     for t in range(tile, N, tile):
-        if t in (tile, 2 * tile) or t >= N - tile:
+        if t in (tile, 2 * tile) or t >= N - tile or t % pair_tile == 0:
             s.update((t - 1, t))
     last_tile = (N - 1) // tile * tile
     s.update((last_tile, min(N - 1, last_tile + 1)))

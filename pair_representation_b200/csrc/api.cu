@@ -823,11 +823,19 @@ int trimul_workspace_views(const trimul_params *p, void **a, void **b, void **x,
 }
 
 int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *detail) {
-    if (!p || !p->workspace) return TRIMUL_ERR_INVALID_ARG;
+    if (!p) return TRIMUL_ERR_INVALID_ARG;
+    // Without a workspace the status word is the one in the static scratch of
+    // trimul_forward_noalloc on the current device.
+    const void *word = p->workspace;
+    if (!word) {
+        void *scratch = nullptr;
+        if (int rc = noalloc_scratch_address(&scratch)) return rc;
+        word = scratch;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     DeviceStatus st;
     cudaError_t e = cudaStreamSynchronize(s);
-    if (e == cudaSuccess) e = cudaMemcpy(&st, p->workspace, sizeof st, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(&st, word, sizeof st, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) {
         set_detail("status read", e);
         return TRIMUL_ERR_CUDA;

@@ -115,15 +115,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
         *abort_flag = 1;
         st_remote_u32(peer_abort, 1u);
     };
-    // Which 128-row half of a 256-row tile edge starting at `base` CTA `r` loads.
-    // Normally CTA r takes half r. Where the upper half would be only partly
-    // inside [0, N), the CTAs swap, so CTA 1 (whose loads complete on CTA 0's
-    // barrier) always loads a half that is fully inside or fully outside the
-    // matrix; the partial half is loaded by CTA 0 onto its own barrier.
-    auto half_of = [&](int base, uint32_t r) -> int {
-        const bool swap = base + HALF < args.N && args.N < base + 2 * HALF;
-        return (int)(r ^ (swap ? 1u : 0u));
-    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -140,8 +131,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
                 const int c = tile / tiles_per_c;
                 const int r = tile - c * tiles_per_c;
                 const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
-                const int i0 = ti * 256 + half_of(ti * 256, rank) * HALF;
-                const int j0 = tj * BN + half_of(tj * BN, rank) * HALF;
+                const int i0 = ti * 256 + (int)rank * HALF;
+                const int j0 = tj * BN + (int)rank * HALF;
                 for (int kb = 0; kb < args.kblocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, ctl, SITE_CON | 1, tile)) {
                         ok = false;
@@ -253,15 +244,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
         const bool leader = (threadIdx.x == 64);
         const uint32_t tempty0 = map_to_rank(&tempty[0], 0);
         const uint32_t tempty1 = map_to_rank(&tempty[1], 0);
+        // Stores issued so far by this CTA, over all its tiles: store n stages
+        // through buffer n & 1, and before it is written the store that last used
+        // that buffer (n - 2) must have read it, which wait_group.read 1 ensures
+        // only because the count runs on across tiles. A count restarted per tile
+        // would, after a tile with an odd number of stores (one in the ragged last
+        // column of tiles), give the next tile's first chunk the buffer that the
+        // still-pending last store of that tile is reading.
+        int nst = 0;
         int lt = 0;
         for (int tile = pair; tile < args.total_tiles; tile += npairs, ++lt) {
             const int c = tile / tiles_per_c;
             const int r = tile - c * tiles_per_c;
             const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
             // This CTA's accumulator rows are the A rows it loaded; accumulator columns
-            // [0,128) come from CTA 0's B rows and [128,256) from CTA 1's.
-            const int i0 = ti * 256 + half_of(ti * 256, rank) * HALF;
-            const int jb0 = tj * BN + half_of(tj * BN, 0) * HALF, jb1 = tj * BN + half_of(tj * BN, 1) * HALF;
+            // [0,128) come from CTA 0's B rows and [128,256) from CTA 1's, i.e. tile
+            // columns j0 .. j0 + 255 in order.
+            const int i0 = ti * 256 + (int)rank * HALF;
+            const int j0 = tj * BN;
             const int acc = lt & 1;
             const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
             if (leader) {
@@ -274,10 +274,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
             tc_fence_after();
             // Chunks whose first column is past N, and whole halves whose first row is past N,
             // are neither read nor stored.
-            int nst = 0;  // stores issued for this tile
 #pragma unroll 1
             for (int ch = 0; ch < BN / OUT_COLS; ++ch) {
-                const int jst = (ch < 2 ? jb0 : jb1) + (ch & 1) * OUT_COLS;
+                const int jst = j0 + ch * OUT_COLS;
                 if (i0 >= args.N || jst >= args.N) continue;
                 uint32_t v[64];
                 const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * OUT_COLS);

@@ -210,6 +210,12 @@ size_t atomattn_tc_smem();
 cudaError_t atomattn_tc_setup();
 cudaError_t launch_atomattn_tc(const AttnMaps &m, const AttnArgs &a, int grid, cudaStream_t s);
 
+// ---- static scratch of trimul_forward_noalloc (noalloc.cu) --------------------
+
+// Device address of the library's static scratch array on the current device;
+// TRIMUL_OK or TRIMUL_ERR_CUDA.
+int noalloc_scratch_address(void **out);
+
 // ---- fp32 CUDA-core path ----------------------------------------------------
 
 struct F32Layer {

@@ -17,7 +17,8 @@
 //
 // The device address of the array is looked up once per device, on the first
 // call made with that device current; that first call should therefore come
-// before any stream capture.
+// before any stream capture. The status word at the start of the array is read
+// with trimul_device_status on a params block whose workspace is NULL.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -33,7 +34,14 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
 
-int scratch_address(void **out) {
+}  // namespace
+
+namespace trimul {
+
+// Device address of the static scratch for the current device (looked up once
+// per device). Used by trimul_forward_noalloc and, for a params block without
+// a workspace, by trimul_device_status.
+int noalloc_scratch_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRIMUL_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
@@ -51,7 +59,7 @@ int scratch_address(void **out) {
     return TRIMUL_OK;
 }
 
-}  // namespace
+}  // namespace trimul
 
 extern "C" int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params *p, int direction,
                                       void *out, trimul_stream_t stream) {
@@ -62,7 +70,7 @@ extern "C" int trimul_forward_noalloc(const void *z, const void *mask, const tri
                                                                        : TRIMUL_ERR_UNSUPPORTED;
     if (need > (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES) return TRIMUL_ERR_WORKSPACE;  // beyond the static scratch
     void *scratch = nullptr;
-    int rc = scratch_address(&scratch);
+    int rc = trimul::noalloc_scratch_address(&scratch);
     if (rc) return rc;
     trimul_params q = *p;
     q.workspace = scratch;

@@ -56,7 +56,7 @@ def test_fp32_edge_sizes(N, direction):
 
 # ---------------------------------------------------------------- bf16 stages
 
-@pytest.mark.parametrize("N", [64, 129, 200, 256, 300, 385, 386, 513])
+@pytest.mark.parametrize("N", [64, 129, 200, 256, 300, 385, 386, 513, 769, 1025])
 @pytest.mark.parametrize("direction", ["outgoing", "incoming"])
 def test_bf16_contraction_stage(N, direction):
     """x from random bf16 a, b written into the workspace, vs the oracle contraction."""
@@ -174,14 +174,42 @@ def test_bf16_null_mask_equals_ones():
     assert np.array_equal(a, b)
 
 
-@pytest.mark.parametrize("wid", [3, 4, 5])
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_bf16_workload3_full(direction):
+    """The Boltz-2 crop (N = 768, per-channel scale on z): every output cell against
+    the full oracle, in the launch configuration the bench times."""
+    w = pi.WORKLOADS[3]
+    case = pi.make_workload(w)
+    got = DeviceCase(case, "bf16").forward(DIRS[direction])
+    ref = oracle.trimul(case, direction)
+    assert rel_l2(got, ref) <= BF16_REL
+    assert max_abs(got, ref) <= BF16_ABS
+
+
+@pytest.mark.parametrize("N", [385, 386, 513, 769, 1025])
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_bf16_ragged_pair_tiles_full(N, direction):
+    """Sizes whose last 256-wide pair tile is ragged (a partial upper half, or one
+    64-column store chunk), where the contraction issues an odd number of stores per
+    tile: every output cell against the oracle."""
+    case = pi.random_case(N, 400 + N, bf16=True, affine=True, mask="random")
+    got = DeviceCase(case, "bf16").forward(DIRS[direction])
+    ref = oracle.trimul(case, direction)
+    assert rel_l2(got, ref) <= BF16_REL
+    assert max_abs(got, ref) <= BF16_ABS
+
+
+@pytest.mark.parametrize("wid", [4, 5])
 def test_bf16_large_workloads_sampled(wid):
-    """Full-size workloads (N = 768, 2048, 3605) in the launch configuration the
-    bench times; the oracle computes the sampled grid I x I (tile edges, the
-    ragged tail and random residues) cell by cell."""
+    """Full-size workloads (N = 2048, 3605) in the launch configuration the bench
+    times; the oracle computes the sampled grid I x I cell by cell: every 256-wide
+    pair-tile edge, the first 128-tile edges, the ragged tail, the padding boundary
+    of the mask and random residues."""
     w = pi.WORKLOADS[wid]
     case = pi.make_workload(w)
     I = pi.sample_grid(w.N, w.seed, n_random=16)
+    if w.n_valid < w.N:
+        I = np.unique(np.concatenate([I, [w.n_valid - 1, w.n_valid]])).astype(np.int32)
     dc = DeviceCase(case, "bf16")
     for direction in w.directions:
         got = dc.forward(DIRS[direction])[np.ix_(I, I)]

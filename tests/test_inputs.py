@@ -53,3 +53,5 @@ def test_sample_grid_covers_edges():
         assert np.all(np.diff(I) > 0)
         if N > 256:
             assert {127, 128, 255, 256} <= set(I.tolist())
+        # every pair-tile (256) boundary inside the matrix
+        assert {t - 1 for t in range(256, N, 256)} | set(range(256, N, 256)) <= set(I.tolist())

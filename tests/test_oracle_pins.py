@@ -255,3 +255,49 @@ def test_planted_mistake_is_caught():
     expect = torch.sigmoid(lin(zh, "w_g", "b_g")) * lin(_ln(a * b, d["ln_out_w"], d["ln_out_b"]), "w_o", "b_o")
     got = oracle.trimul(bad, "outgoing")[0, 0]
     assert np.abs(got - expect.numpy()).max() > 1e-3
+
+
+def _einsum_layer(d, direction, eps=EPS):
+    """The whole layer restated with numpy float64 einsum, every weight random.
+
+    Written from the definition, independent of the oracle: LayerNorm with the
+    biased variance and eps inside the root; Linear in [out][in] layout; mask on
+    a and b at their own cell; the contraction summed over the shared residue
+    index (a_ik b_jk outgoing, a_ki b_kj incoming).
+    """
+    f = lambda k: np.asarray(d[k], dtype=np.float64)
+
+    def ln(v, w, b):
+        mu = v.mean(-1, keepdims=True)
+        var = ((v - mu) ** 2).mean(-1, keepdims=True)
+        return (v - mu) / np.sqrt(var + eps) * f(w) + f(b)
+
+    def lin(v, w, b):
+        return np.einsum("ijc,oc->ijo", v, f(w)) + f(b)
+
+    sig = lambda t: 1.0 / (1.0 + np.exp(-t))
+    zh = ln(f("z"), "ln_in_w", "ln_in_b")
+    m = f("mask")[:, :, None]
+    a = m * sig(lin(zh, "w_ag", "b_ag")) * lin(zh, "w_a", "b_a")
+    b = m * sig(lin(zh, "w_bg", "b_bg")) * lin(zh, "w_b", "b_b")
+    x = np.einsum("ikc,jkc->ijc", a, b) if direction == "outgoing" else np.einsum("kic,kjc->ijc", a, b)
+    return sig(lin(zh, "w_g", "b_g")) * lin(ln(x, "ln_out_w", "ln_out_b"), "w_o", "b_o")
+
+
+@pytest.mark.parametrize("N", [2, 3, 5, 8])
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_brute_force_einsum_random_weights(N, direction):
+    """Brute force at tiny N: random weights, LayerNorm affines, biases and a random
+    0/1 mask, against the einsum restatement above, to 1e-12 relative. Unlike the
+    special-weight pins, every step interacts with every other one here."""
+    d = _case(N, 500 + N, mask="random")
+    got = oracle.trimul(d, direction)
+    ref = _einsum_layer(d, direction)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_brute_force_einsum_catches_swapped_contraction():
+    """The einsum pin separates the directions: outgoing and incoming differ at N = 5
+    with random weights, so a direction mix-up in the oracle would fail it."""
+    d = _case(5, 505, mask="random")
+    assert np.abs(_einsum_layer(d, "outgoing") - _einsum_layer(d, "incoming")).max() > 1e-3
