@@ -160,6 +160,73 @@ const char *trimul_last_error_detail(void);
 int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params *p, int direction,
                            void *out, trimul_stream_t stream);
 
+/* ---- Shard stage calls (the layer split over several GPUs) -------------------
+ * The pages' subject is running this layer on many GPUs ("Scaling
+ * biomolecular modeling with context parallelism in NVIDIA BioNeMo", sections
+ * "2-D tiling of the pair representation" and "Context-parallel
+ * implementation of triangle multiplication"). These calls are the per-GPU
+ * pieces of the plainest such split: each GPU projects a block of residue
+ * rows (all channels), the channels are exchanged so that each GPU contracts
+ * a block of channels over all rows, x is exchanged back to row blocks, and
+ * each GPU finishes its rows. The exchanges are the caller's (NCCL send/recv
+ * through torch.distributed in pair_representation_b200.sharded); the
+ * prologue and epilogue are per cell, so a row block is just a grid of
+ * rows x N cells. All buffers are caller-owned device memory, 16-byte
+ * aligned; ld = N rounded up to 8. BF16 only (TRIMUL_ERR_UNSUPPORTED
+ * otherwise); p->N is the full residue count and p->workspace holds the status
+ * word and scratch for re-pitching mask rows:
+ * trimul_shard_workspace_size(N, rows) bytes. Asynchronous. */
+size_t trimul_shard_workspace_size(int N, int rows);
+
+/* z_rows [rows][N][c_z] and mask_rows [rows][N] (or NULL) of a block of
+ * residue rows -> a, b [c_h][rows][ld] (channel-major). Clears the status word. */
+int trimul_prologue_rows(const void *z_rows, const void *mask_rows, const trimul_params *p, int rows,
+                         void *a, void *b, trimul_stream_t stream);
+
+/* The triangle contraction of `channels` (1..c_h) channels over all N rows:
+ * a, b, x [channels][N][ld]; x_c = a_c b_c^T (outgoing) or a_c^T b_c. */
+int trimul_contract_channels(const trimul_params *p, int direction, int channels, const void *a,
+                             const void *b, void *x, trimul_stream_t stream);
+
+/* z_rows [rows][N][c_z] and x_rows [c_h][rows][ld] of a block of residue rows
+ * -> out_rows [rows][N][c_z]. */
+int trimul_epilogue_rows(const void *z_rows, const void *x_rows, const trimul_params *p, int rows,
+                         void *out_rows, trimul_stream_t stream);
+
+/* ---- MXFP8 contraction ------------------------------------------------------
+ * The layer with its triangle contraction in MXFP8, the Blackwell
+ * microscaling format the BioNeMo recipes list among their training
+ * precisions ("Scaling biomolecular modeling with context parallelism in
+ * NVIDIA BioNeMo", the precision list), read as OCP Microscaling (MX) v1.0:
+ * a and b, as the prologue stores them in bf16, are quantised in blocks of 32
+ * along the contracted index k (along the rows of a and b for
+ * TRIMUL_OUTGOING, down their columns for TRIMUL_INCOMING) to E4M3 elements
+ * (round to nearest even, saturated at +-448) sharing an E8M0 scale
+ * 2^(floor(log2 max|v|) - 8); the contraction then runs on tcgen05
+ * block-scaled MMAs (kind::mxf8f6f4) with fp32 accumulation and writes x in
+ * bf16. The prologue and epilogue are those of trimul_forward.
+ *
+ * BF16 only (TRIMUL_ERR_UNSUPPORTED otherwise). p->workspace must hold
+ * trimul_workspace_size_mxfp8(N, c_z, c_h) bytes: the bf16 sections of
+ * trimul_forward followed by the E4M3 operands and their scales
+ * (TRIMUL_ERR_WORKSPACE if smaller). Everything else as for trimul_forward:
+ * asynchronous, nothing allocated, status word in the workspace. */
+size_t trimul_workspace_size_mxfp8(int N, int c_z, int c_h);
+int trimul_forward_mxfp8(const void *z, const void *mask, const trimul_params *p, int direction,
+                         void *out, trimul_stream_t stream);
+
+/* The MXFP8 contraction stage alone: a, b (bf16, in the workspace) -> x. */
+int trimul_contract_mxfp8(const trimul_params *p, int direction, trimul_stream_t stream);
+
+/* Device pointers of the quantised operands inside p->workspace (host-only):
+ * aq, bq are [c_h][N][ldq] E4M3 codes, operand row m with k contiguous (for
+ * TRIMUL_INCOMING the transposes of a_c and b_c); sa, sb the E8M0 scale bytes
+ * (exponent + 127) of a (per 128-row half of each 256-row output tile) and b
+ * (per 192-row output tile), each per 128-wide K chunk in 512-byte chunks of
+ * 128 rows x 4 blocks: row r, block kb at (r % 32) * 16 + ((r % 128) / 32) * 4
+ * + kb % 4. */
+int trimul_mxfp8_views(const trimul_params *p, void **aq, void **bq, void **sa, void **sb, size_t *ldq);
+
 /* ---- Backward -------------------------------------------------------------
  * Gradients of a loss L through one forward call. Given dout = dL/dout
  * ([N][N][c_z], dtype of z), trimul_backward writes dz = dL/dz ([N][N][c_z],

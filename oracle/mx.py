@@ -88,3 +88,20 @@ def mx_contract(a, b, direction):
     if incoming:
         return np.einsum("kic,kjc->ijc", aq, bq)
     return np.einsum("ikc,jkc->ijc", aq, bq)
+
+
+def mx_contract_grid(a, b, direction, I):
+    """The MXFP8 contraction on the cells I x I only: x [len(I)][len(I)][c].
+
+    The operands are quantised in full (blocks along k need every k), then only
+    the rows (outgoing) or columns (incoming) of the sampled residues are
+    contracted, exactly as mx_contract would for those cells.
+    """
+    incoming = direction in ("incoming", 1)
+    axis = 0 if incoming else 1
+    I = np.asarray(I)
+    _, _, aq = mx_quantize_blocks(a, axis)
+    _, _, bq = mx_quantize_blocks(b, axis)
+    if incoming:
+        return np.einsum("kic,kjc->ijc", aq[:, I], bq[:, I])
+    return np.einsum("ikc,jkc->ijc", aq[I], bq[I])

@@ -39,6 +39,8 @@ EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forwa
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
            "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
            "trimul_backward", "trimul_backward_workspace_size",
+           "trimul_workspace_size_mxfp8", "trimul_forward_mxfp8", "trimul_contract_mxfp8", "trimul_mxfp8_views",
+           "trimul_shard_workspace_size", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows",
            "atomattn_forward", "atomattn_workspace_size", "atomattn_device_status")
 
 # Gradient outputs of trimul_grads, in struct order; each is "d_" + a TrimulParams field.
@@ -124,6 +126,16 @@ def lib():
         L.trimul_backward_workspace_size.argtypes = [I, I, I]
         L.trimul_backward_workspace_size.restype = S
         L.trimul_backward.argtypes = [P, P, PP, I, P, P, ctypes.POINTER(TrimulGrads), P]
+        L.trimul_workspace_size_mxfp8.argtypes = [I, I, I]
+        L.trimul_workspace_size_mxfp8.restype = S
+        L.trimul_forward_mxfp8.argtypes = [P, P, PP, I, P, P]
+        L.trimul_contract_mxfp8.argtypes = [PP, I, P]
+        L.trimul_mxfp8_views.argtypes = [PP] + [ctypes.POINTER(P)] * 4 + [ctypes.POINTER(S)]
+        L.trimul_shard_workspace_size.argtypes = [I, I]
+        L.trimul_shard_workspace_size.restype = S
+        L.trimul_prologue_rows.argtypes = [P, P, PP, I, P, P, P]
+        L.trimul_contract_channels.argtypes = [PP, I, I, P, P, P, P]
+        L.trimul_epilogue_rows.argtypes = [P, P, PP, I, P, P]
         AP = ctypes.POINTER(AtomAttnParams)
         L.atomattn_workspace_size.argtypes = []
         L.atomattn_workspace_size.restype = S
@@ -131,7 +143,8 @@ def lib():
         L.atomattn_device_status.argtypes = [AP, P, ctypes.POINTER(ctypes.c_int)]
         for f in ("trimul_forward", "trimul_forward_noalloc", "trimul_prologue", "trimul_contract", "trimul_epilogue",
                   "trimul_workspace_views", "trimul_device_status", "trimul_version", "trimul_backward",
-                  "atomattn_forward", "atomattn_device_status"):
+                  "atomattn_forward", "atomattn_device_status", "trimul_forward_mxfp8", "trimul_contract_mxfp8",
+                  "trimul_mxfp8_views", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -222,6 +235,63 @@ def trimul_backward(z, mask, params: TrimulParams, direction: int, dout, dz, gra
                                ctypes.byref(grads), _stream(stream))
     if check:
         _check(rc, "trimul_backward")
+    return rc
+
+
+def trimul_workspace_size_mxfp8(N: int, c_z: int = 128, c_h: int = 128) -> int:
+    return lib().trimul_workspace_size_mxfp8(N, c_z, c_h)
+
+
+def trimul_forward_mxfp8(z, mask, params: TrimulParams, direction: int, out, stream=None, check=True) -> int:
+    """The layer with the contraction in MXFP8 (E4M3 in blocks of 32 along k, E8M0 scales)."""
+    rc = lib().trimul_forward_mxfp8(_ptr(z), _ptr(mask), ctypes.byref(params), direction, _ptr(out), _stream(stream))
+    if check:
+        _check(rc, "trimul_forward_mxfp8")
+    return rc
+
+
+def trimul_contract_mxfp8(params: TrimulParams, direction: int, stream=None, check=True) -> int:
+    rc = lib().trimul_contract_mxfp8(ctypes.byref(params), direction, _stream(stream))
+    if check:
+        _check(rc, "trimul_contract_mxfp8")
+    return rc
+
+
+def trimul_mxfp8_views(params: TrimulParams):
+    """(aq, bq, sa, sb, ldq): device addresses of the quantised operands and scales in the workspace."""
+    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    ldq = ctypes.c_size_t()
+    _check(lib().trimul_mxfp8_views(ctypes.byref(params), *[ctypes.byref(x) for x in ptrs], ctypes.byref(ldq)),
+           "trimul_mxfp8_views")
+    return ptrs[0].value, ptrs[1].value, ptrs[2].value, ptrs[3].value, ldq.value
+
+
+def trimul_shard_workspace_size(N: int, rows: int) -> int:
+    return lib().trimul_shard_workspace_size(N, rows)
+
+
+def trimul_prologue_rows(z_rows, mask_rows, params: TrimulParams, rows: int, a, b, stream=None, check=True) -> int:
+    rc = lib().trimul_prologue_rows(_ptr(z_rows), _ptr(mask_rows), ctypes.byref(params), rows, _ptr(a), _ptr(b),
+                                    _stream(stream))
+    if check:
+        _check(rc, "trimul_prologue_rows")
+    return rc
+
+
+def trimul_contract_channels(params: TrimulParams, direction: int, channels: int, a, b, x, stream=None,
+                             check=True) -> int:
+    rc = lib().trimul_contract_channels(ctypes.byref(params), direction, channels, _ptr(a), _ptr(b), _ptr(x),
+                                        _stream(stream))
+    if check:
+        _check(rc, "trimul_contract_channels")
+    return rc
+
+
+def trimul_epilogue_rows(z_rows, x_rows, params: TrimulParams, rows: int, out_rows, stream=None, check=True) -> int:
+    rc = lib().trimul_epilogue_rows(_ptr(z_rows), _ptr(x_rows), ctypes.byref(params), rows, _ptr(out_rows),
+                                    _stream(stream))
+    if check:
+        _check(rc, "trimul_epilogue_rows")
     return rc
 
 

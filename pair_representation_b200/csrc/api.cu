@@ -7,7 +7,9 @@
 
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
+#include <utility>
 
 #include "atomattn.h"
 #include "kernels.h"
@@ -74,8 +76,9 @@ int device_state(const DevState **out, bool need_tc) {
         }
         if (d.cc_major == 10 && d.cc_minor == 0) {
             if ((e = prologue_tc_setup()) == cudaSuccess && (e = contract_tc_setup()) == cudaSuccess &&
-                (e = epilogue_tc_setup()) == cudaSuccess && (e = backward_setup()) == cudaSuccess)
-                e = atomattn_tc_setup();
+                (e = epilogue_tc_setup()) == cudaSuccess && (e = backward_setup()) == cudaSuccess &&
+                (e = atomattn_tc_setup()) == cudaSuccess)
+                e = contract_mx_setup();
             d.tc_setup = e;
         } else {
             d.tc_setup = cudaErrorNoKernelImageForDevice;
@@ -126,7 +129,18 @@ int check_device_ptr(const void *p, const char *name) {
 
 // ---- argument checks (pure host logic, no CUDA calls) ------------------------
 
+int check_params_core(const trimul_params *p);
+
 int check_params(const trimul_params *p) {
+    if (int rc = check_params_core(p)) return rc;
+    if (!p->workspace || p->workspace_bytes < trimul_workspace_size_dtype(p->N, p->c_z, p->c_h, p->dtype))
+        return TRIMUL_ERR_WORKSPACE;
+    if (!aligned(p->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
+    return TRIMUL_OK;
+}
+
+// Everything check_params checks except the size of the workspace.
+int check_params_core(const trimul_params *p) {
     if (!p) return TRIMUL_ERR_INVALID_ARG;
     if (p->N < 1 || p->N > kMaxN || p->c_z < 1 || p->c_h < 1) return TRIMUL_ERR_INVALID_ARG;
     if (p->c_z != kC || p->c_h != kC || !valid_dtype(p->dtype)) return TRIMUL_ERR_UNSUPPORTED;
@@ -141,9 +155,35 @@ int check_params(const trimul_params *p) {
                          p->b_g, p->ln_out_w, p->ln_out_b, p->b_o};
     for (const void *v : vec)
         if (v && !aligned(v, es)) return TRIMUL_ERR_MISALIGNED;
-    if (!p->workspace || p->workspace_bytes < trimul_workspace_size_dtype(p->N, p->c_z, p->c_h, p->dtype))
-        return TRIMUL_ERR_WORKSPACE;
+    return TRIMUL_OK;
+}
+
+// ---- shard stage calls: explicit buffers, a grid of rows x N cells or a subset of channels ----
+
+size_t shard_ws_bytes(int N, int rows) { return kHeader + round_up((size_t)rows * ld_of(N) * 2, 256); }
+
+int check_shard(const trimul_params *p, int rows) {
+    if (int rc = check_params_core(p)) return rc;
+    if (p->dtype != TRIMUL_DTYPE_BF16) return TRIMUL_ERR_UNSUPPORTED;
+    if (rows < 1 || rows > p->N) return TRIMUL_ERR_INVALID_ARG;
+    if (!p->workspace || p->workspace_bytes < shard_ws_bytes(p->N, rows)) return TRIMUL_ERR_WORKSPACE;
     if (!aligned(p->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
+    return TRIMUL_OK;
+}
+
+int check_buffers(std::initializer_list<std::pair<const void *, size_t>> in,
+                  std::initializer_list<std::pair<const void *, size_t>> out, const trimul_params *p) {
+    for (auto &b : in)
+        if (b.first && !aligned(b.first, 16)) return TRIMUL_ERR_MISALIGNED;
+    for (auto &o : out) {
+        if (!o.first) return TRIMUL_ERR_INVALID_ARG;
+        if (!aligned(o.first, 16)) return TRIMUL_ERR_MISALIGNED;
+        if (overlap(o.first, o.second, p->workspace, p->workspace_bytes)) return TRIMUL_ERR_ALIAS;
+        for (auto &b : in)
+            if (overlap(o.first, o.second, b.first, b.second)) return TRIMUL_ERR_ALIAS;
+        for (auto &q : out)
+            if (&q != &o && overlap(o.first, o.second, q.first, q.second)) return TRIMUL_ERR_ALIAS;
+    }
     return TRIMUL_OK;
 }
 
@@ -218,7 +258,8 @@ KernelCtl ctl_of(const trimul_params *p, const Views &v) {
 // ---- tensor maps ----------------------------------------------------------------
 
 int encode(CUtensorMap *m, int rank, const void *base, const uint64_t *dims, const uint64_t *strides,
-           const uint32_t *box, CUtensorMapSwizzle sw) {
+           const uint32_t *box, CUtensorMapSwizzle sw,
+           CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     cuuint64_t gd[5], gs[4];
     cuuint32_t bd[5], es[5];
     for (int r = 0; r < rank; ++r) {
@@ -227,7 +268,7 @@ int encode(CUtensorMap *m, int rank, const void *base, const uint64_t *dims, con
         es[r] = 1;
         if (r < rank - 1) gs[r] = strides[r];
     }
-    CUresult res = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gd, gs,
+    CUresult res = g_encode(m, dt, (cuuint32_t)rank, const_cast<void *>(base), gd, gs,
                             bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (res != CUDA_SUCCESS) {
@@ -244,26 +285,27 @@ int map_weight(CUtensorMap *m, const void *w) {
     return encode(m, 2, w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// z or out [N][N][128] as (c, j, i): box of b0 channels x b1 cells of one row.
-int map_pair(CUtensorMap *m, const void *t, int N, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
-    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)N};
+// z or out [rows][N][128] as (c, j, i): box of b0 channels x b1 cells of one row.
+int map_pair(CUtensorMap *m, const void *t, int N, int rows, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)rows};
     const uint64_t strides[2] = {128 * 2, (uint64_t)N * 128 * 2};
     const uint32_t box[3] = {b0, b1, 1};
     return encode(m, 3, t, dims, strides, box, sw);
 }
 
-// mask [N][pitch] as (j, i): one row segment of 128 cells per box, zero past column N.
-int map_mask(CUtensorMap *m, const void *t, int N, size_t pitch) {
-    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)N}, strides[1] = {pitch * 2};
-    const uint32_t box[2] = {128, 1};
+// mask [rows][pitch] as (j, i): one row segment of 64 cells per box, zero past column N.
+int map_mask(CUtensorMap *m, const void *t, int N, int rows, size_t pitch) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)rows}, strides[1] = {pitch * 2};
+    const uint32_t box[2] = {64, 1};
     return encode(m, 2, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// a, b or x [128][N][ld] as (col, row, c) with the given box and swizzle.
+// a, b or x [channels][rows][ld] (N columns) as (col, row, c) with the given box and swizzle.
 int map_cm(CUtensorMap *m, const void *t, int N, size_t ld, uint32_t b0, uint32_t b1, uint32_t b2,
-           CUtensorMapSwizzle sw) {
-    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, 128};
-    const uint64_t strides[2] = {ld * 2, (uint64_t)N * ld * 2};
+           CUtensorMapSwizzle sw, int rows = 0, int channels = 128) {
+    if (rows == 0) rows = N;
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)rows, (uint64_t)channels};
+    const uint64_t strides[2] = {ld * 2, (uint64_t)rows * ld * 2};
     const uint32_t box[3] = {b0, b1, b2};
     return encode(m, 3, t, dims, strides, box, sw);
 }
@@ -304,6 +346,54 @@ int cuda_rc(cudaError_t e, const char *what) {
 
 // ---- stages ------------------------------------------------------------------------
 
+// The bf16 prologue over a grid of rows x N cells: z [rows][N][128], mask [rows][N]
+// or null, a and b written as [128][rows][ld]. mask_scratch holds rows * ld bf16
+// for a mask whose rows lack a 16-byte pitch.
+int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int rows, void *a_out, void *b_out,
+                    void *mask_scratch, const KernelCtl &ctl, const DevState &d, cudaStream_t s) {
+    const size_t ld = ld_of(p->N);
+    PrologueMaps m;
+    if (int rc = map_pair(&m.z, z, p->N, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    // The mask rows travel with the z tiles. A tensor map needs a 16-byte row pitch, so a
+    // mask whose rows do not have one is first copied into the scratch with pitch ld.
+    m.mask = m.z;  // unused without a mask
+    if (mask) {
+        const void *src = mask;
+        size_t pitch = (size_t)p->N;
+        if (p->N % 8 != 0 || !aligned(mask, 16)) {
+            __nv_bfloat16 *pad = reinterpret_cast<__nv_bfloat16 *>(mask_scratch);
+            if (int rc = cuda_rc(launch_mask_pad(static_cast<const __nv_bfloat16 *>(mask), pad, p->N, rows, (int)ld, s),
+                                 "mask_pad launch"))
+                return rc;
+            src = pad;
+            pitch = ld;
+        }
+        if (int rc = map_mask(&m.mask, src, p->N, rows, pitch)) return rc;
+    }
+    // Each lane quadrant stores 64 cells x 32 channels (128-byte rows, 128-byte swizzle).
+    if (int rc = map_cm(&m.a, a_out, p->N, ld, 64, 1, 32, CU_TENSOR_MAP_SWIZZLE_128B, rows)) return rc;
+    if (int rc = map_cm(&m.b, b_out, p->N, ld, 64, 1, 32, CU_TENSOR_MAP_SWIZZLE_128B, rows)) return rc;
+    PrologueArgs a;
+    a.N = p->N;
+    a.jt_tiles = (p->N + 63) / 64;
+    a.total_tiles = rows * a.jt_tiles;
+    a.eps = p->ln_eps;
+    a.has_mask = mask != nullptr;
+    a.w_a = static_cast<const __nv_bfloat16 *>(p->w_a);
+    a.w_ag = static_cast<const __nv_bfloat16 *>(p->w_ag);
+    a.w_b = static_cast<const __nv_bfloat16 *>(p->w_b);
+    a.w_bg = static_cast<const __nv_bfloat16 *>(p->w_bg);
+    a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
+    a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
+    a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
+    a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
+    a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
+    a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
+    a.ctl = ctl;
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_prologue_tc(m, a, grid, s), "prologue_tc launch");
+}
+
 int run_prologue(const void *z, const void *mask, const trimul_params *p, const DevState &d, cudaStream_t s) {
     const Views v = views_of(p);
     if (p->dtype == TRIMUL_DTYPE_F32) {
@@ -312,46 +402,8 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
         return cuda_rc(launch_prologue_f32(static_cast<const float *>(z), f32_layer(p, mask, v), grid, s),
                        "prologue_f32 launch");
     }
-    PrologueMaps m;
-    const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
-    for (int k = 0; k < 4; ++k)
-        if (int rc = map_weight(&m.w[k], w[k])) return rc;
-    if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    // The mask rows travel with the z tiles. A tensor map needs a 16-byte row pitch, so a
-    // mask whose rows do not have one is first copied into plane 0 of x (pitch ld), which the
-    // contraction overwrites later.
-    m.mask = m.z;  // unused without a mask
-    if (mask) {
-        const void *src = mask;
-        size_t pitch = (size_t)p->N;
-        if (p->N % 8 != 0 || !aligned(mask, 16)) {
-            __nv_bfloat16 *pad = reinterpret_cast<__nv_bfloat16 *>(v.x);
-            if (int rc = cuda_rc(launch_mask_pad(static_cast<const __nv_bfloat16 *>(mask), pad, p->N, (int)v.ld, s),
-                                 "mask_pad launch"))
-                return rc;
-            src = pad;
-            pitch = v.ld;
-        }
-        if (int rc = map_mask(&m.mask, src, p->N, pitch)) return rc;
-    }
-    // Each worker warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
-    if (int rc = map_cm(&m.a, v.a, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
-    if (int rc = map_cm(&m.b, v.b, p->N, v.ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
-    PrologueArgs a;
-    a.N = p->N;
-    a.jt_tiles = (p->N + 127) / 128;
-    a.total_tiles = p->N * a.jt_tiles;
-    a.eps = p->ln_eps;
-    a.has_mask = mask != nullptr;
-    a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
-    a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
-    a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
-    a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
-    a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
-    a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
-    a.ctl = ctl_of(p, v);
-    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
-    return cuda_rc(launch_prologue_tc(m, a, grid, s), "prologue_tc launch");
+    // A re-pitched mask goes to plane 0 of x, which the contraction overwrites later.
+    return run_prologue_tc(z, mask, p, p->N, v.a, v.b, v.x, ctl_of(p, v), d, s);
 }
 
 // X_c[m][n] = sum_k A_c(m, k) B_c(n, k) for the 128 channels of [128][N][ld] bf16
@@ -360,18 +412,18 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
 // rows [128 r, 128 r + 128) of the A and B panels (boxes of 128 rows, or 2 x
 // 64-wide blocks when MN-major).
 int run_contract_on(const void *A, int a_mn, const void *B, int b_mn, void *X, int N, size_t ld, const KernelCtl &ctl,
-                    const DevState &d, cudaStream_t s) {
+                    const DevState &d, cudaStream_t s, int channels = kC) {
     ContractMaps m;
-    if (int rc = map_cm(&m.a, A, N, ld, 64, a_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    if (int rc = map_cm(&m.b, B, N, ld, 64, b_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    if (int rc = map_cm(&m.x, X, N, ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    if (int rc = map_cm(&m.a, A, N, ld, 64, a_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
+    if (int rc = map_cm(&m.b, B, N, ld, 64, b_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
+    if (int rc = map_cm(&m.x, X, N, ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
     ContractArgs a;
     a.N = N;
     a.a_mn = a_mn;
     a.b_mn = b_mn;
     a.ti_tiles = (N + 255) / 256;
     a.tj_tiles = (N + 255) / 256;
-    a.total_tiles = kC * a.ti_tiles * a.tj_tiles;
+    a.total_tiles = channels * a.ti_tiles * a.tj_tiles;
     a.kblocks = (N + 63) / 64;
     a.ctl = ctl;
     const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
@@ -386,6 +438,33 @@ int run_contract(const trimul_params *p, int direction, const DevState &d, cudaS
     return run_contract_on(v.a, mn, v.b, mn, v.x, p->N, v.ld, ctl_of(p, v), d, s);
 }
 
+// The bf16 epilogue over a grid of rows x N cells: z and out [rows][N][128], x [128][rows][ld].
+int run_epilogue_tc(const void *z, const void *x, const trimul_params *p, int rows, void *out, const KernelCtl &ctl,
+                    const DevState &d, cudaStream_t s) {
+    EpilogueMaps m;
+    if (int rc = map_weight(&m.wg, p->w_g)) return rc;
+    if (int rc = map_weight(&m.wo, p->w_o)) return rc;
+    if (int rc = map_pair(&m.z, z, p->N, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    // x as the MN-major MMA operand: 64 cells x 128 channels per box, 128-byte swizzle.
+    if (int rc = map_cm(&m.x, x, p->N, ld_of(p->N), 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B, rows)) return rc;
+    // Each worker warp stores 32 channels x 32 cells (64-byte rows, 64-byte swizzle).
+    if (int rc = map_pair(&m.out, out, p->N, rows, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
+    EpilogueArgs a;
+    a.N = p->N;
+    a.jt_tiles = (p->N + 127) / 128;
+    a.total_tiles = rows * a.jt_tiles;
+    a.eps = p->ln_eps;
+    a.ln_in_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
+    a.ln_in_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
+    a.ln_out_w = static_cast<const __nv_bfloat16 *>(p->ln_out_w);
+    a.ln_out_b = static_cast<const __nv_bfloat16 *>(p->ln_out_b);
+    a.b_g = static_cast<const __nv_bfloat16 *>(p->b_g);
+    a.b_o = static_cast<const __nv_bfloat16 *>(p->b_o);
+    a.ctl = ctl;
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_epilogue_tc(m, a, grid, s), "epilogue_tc launch");
+}
+
 int run_epilogue(const void *z, const trimul_params *p, void *out, const DevState &d, cudaStream_t s) {
     const Views v = views_of(p);
     if (p->dtype == TRIMUL_DTYPE_F32) {
@@ -395,32 +474,109 @@ int run_epilogue(const void *z, const trimul_params *p, void *out, const DevStat
                                            f32_layer(p, nullptr, v), grid, s),
                        "epilogue_f32 launch");
     }
-    EpilogueMaps m;
-    if (int rc = map_weight(&m.wg, p->w_g)) return rc;
-    if (int rc = map_weight(&m.wo, p->w_o)) return rc;
-    if (int rc = map_pair(&m.z, z, p->N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    // x as the MN-major MMA operand: 64 cells x 128 channels per box, 128-byte swizzle.
-    if (int rc = map_cm(&m.x, v.x, p->N, v.ld, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
-    // Each worker warp stores 32 channels x 32 cells (64-byte rows, 64-byte swizzle).
-    if (int rc = map_pair(&m.out, out, p->N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
-    EpilogueArgs a;
-    a.N = p->N;
-    a.jt_tiles = (p->N + 127) / 128;
-    a.total_tiles = p->N * a.jt_tiles;
-    a.eps = p->ln_eps;
-    a.ln_in_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
-    a.ln_in_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
-    a.ln_out_w = static_cast<const __nv_bfloat16 *>(p->ln_out_w);
-    a.ln_out_b = static_cast<const __nv_bfloat16 *>(p->ln_out_b);
-    a.b_g = static_cast<const __nv_bfloat16 *>(p->b_g);
-    a.b_o = static_cast<const __nv_bfloat16 *>(p->b_o);
-    a.ctl = ctl_of(p, v);
-    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
-    return cuda_rc(launch_epilogue_tc(m, a, grid, s), "epilogue_tc launch");
+    return run_epilogue_tc(z, v.x, p, p->N, out, ctl_of(p, v), d, s);
 }
 
 int clear_status(const trimul_params *p, cudaStream_t s) {
     return cuda_rc(cudaMemsetAsync(p->workspace, 0, sizeof(DeviceStatus), s), "status clear");
+}
+
+// ---- MXFP8 contraction -----------------------------------------------------------------
+
+// Sections after the bf16 workspace (each 256-byte aligned): the E4M3 operands
+// aq, bq [128][N][ldq] and their scales sa (per 128-row half of a 256-row pair
+// tile), sb (per 192-row tile), both per 128-wide K chunk.
+struct MxLayout {
+    size_t aq, bq, sa, sb, total, ldq;
+    int ti, tj, kc;
+};
+
+MxLayout mx_layout(int N) {
+    MxLayout L;
+    L.ldq = ((size_t)N + 15) & ~(size_t)15;
+    L.ti = (N + 255) / 256;
+    L.tj = (N + 191) / 192;
+    L.kc = (N + 127) / 128;
+    size_t off = kHeader + 3 * section_bytes(N, TRIMUL_DTYPE_BF16);
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    L.aq = take((size_t)kC * N * L.ldq);
+    L.bq = take((size_t)kC * N * L.ldq);
+    L.sa = take((size_t)kC * 2 * L.ti * L.kc * 512);
+    L.sb = take((size_t)kC * L.tj * L.kc * 1024);
+    L.total = off;
+    return L;
+}
+
+int check_mx(const trimul_params *p) {
+    if (p->dtype != TRIMUL_DTYPE_BF16) return TRIMUL_ERR_UNSUPPORTED;
+    if (p->workspace_bytes < mx_layout(p->N).total) return TRIMUL_ERR_WORKSPACE;
+    return TRIMUL_OK;
+}
+
+int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cudaStream_t s) {
+    const Views v = views_of(p);
+    const int N = p->N;
+    const MxLayout L = mx_layout(N);
+    uint8_t *base = static_cast<uint8_t *>(p->workspace);
+    const int tr = direction == TRIMUL_INCOMING;  // incoming: operand row m is the column of a and b
+    // The last 192-row tile of b has scale slots no row reaches; they must not hold NaN codes.
+    if (int rc = cuda_rc(cudaMemsetAsync(base + L.sb, 0, (size_t)kC * L.tj * L.kc * 1024, s), "mx scale clear"))
+        return rc;
+    MxQuantArgs q;
+    q.N = N;
+    q.ld = v.ld;
+    q.ldq = L.ldq;
+    q.kchunks = L.kc;
+    q.src = reinterpret_cast<const __nv_bfloat16 *>(v.a);
+    q.q = base + L.aq;
+    q.sf = base + L.sa;
+    q.rows_per_tile = 128;
+    q.row_tiles = 2 * L.ti;
+    q.chunks_per_tile = 1;
+    if (int rc = cuda_rc(launch_mx_quant(q, tr, s), "mx_quant launch")) return rc;
+    q.src = reinterpret_cast<const __nv_bfloat16 *>(v.b);
+    q.q = base + L.bq;
+    q.sf = base + L.sb;
+    q.rows_per_tile = 192;
+    q.row_tiles = L.tj;
+    q.chunks_per_tile = 2;
+    if (int rc = cuda_rc(launch_mx_quant(q, tr, s), "mx_quant launch")) return rc;
+
+    ContractMxMaps m;
+    const uint64_t qdims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)kC};
+    const uint64_t qstr[2] = {L.ldq, (uint64_t)N * L.ldq};
+    const uint32_t abox[3] = {128, 128, 1}, bbox[3] = {128, 96, 1};
+    if (int rc = encode(&m.a, 3, base + L.aq, qdims, qstr, abox, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    if (int rc = encode(&m.b, 3, base + L.bq, qdims, qstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    const uint64_t sadims[2] = {16, (uint64_t)kC * 2 * L.ti * L.kc * 32}, sbdims[2] = {16, (uint64_t)kC * L.tj * L.kc * 64};
+    const uint64_t sstr[1] = {16};
+    const uint32_t sabox[2] = {16, 32}, sbbox[2] = {16, 64};
+    if (int rc = encode(&m.sa, 2, base + L.sa, sadims, sstr, sabox, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    if (int rc = encode(&m.sb, 2, base + L.sb, sbdims, sstr, sbbox, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    if (int rc = map_cm(&m.x, v.x, N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    ContractMxArgs a;
+    a.N = N;
+    a.ti_tiles = L.ti;
+    a.tj_tiles = L.tj;
+    a.total_tiles = kC * L.ti * L.tj;
+    a.kchunks = L.kc;
+    a.a_row_tiles = 2 * L.ti;
+    a.b_row_tiles = L.tj;
+    a.ctl = ctl_of(p, v);
+    const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
+    return cuda_rc(launch_contract_mx(m, a, 2 * pairs, s), "contract_mx launch");
 }
 
 // ---- backward ----------------------------------------------------------------------
@@ -809,6 +965,117 @@ int trimul_forward(const void *z, const void *mask, const trimul_params *p, int 
     if ((rc = run_prologue(z, mask, p, *d, s))) return rc;
     if ((rc = run_contract(p, direction, *d, s))) return rc;
     return run_epilogue(z, p, out, *d, s);
+}
+
+size_t trimul_workspace_size_mxfp8(int N, int c_z, int c_h) {
+    if (N < 1 || N > kMaxN || c_z != kC || c_h != kC) return 0;
+    return mx_layout(N).total;
+}
+
+int trimul_contract_mxfp8(const trimul_params *p, int direction, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction)) || (rc = check_mx(p))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    if ((rc = check_device_ptr(p->workspace, "workspace"))) return rc;
+    return run_contract_mx(p, direction, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int trimul_forward_mxfp8(const void *z, const void *mask, const trimul_params *p, int direction, void *out,
+                         trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction)) || (rc = check_mx(p)) || (rc = check_z(p, z)) ||
+        (rc = check_mask(p, mask)) || (rc = check_out(p, out, z, mask)))
+        return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
+        (rc = check_device_ptr(mask, "mask")) || (rc = check_device_ptr(out, "out")))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(p, s))) return rc;
+    if ((rc = run_prologue(z, mask, p, *d, s))) return rc;
+    if ((rc = run_contract_mx(p, direction, *d, s))) return rc;
+    return run_epilogue(z, p, out, *d, s);
+}
+
+int trimul_mxfp8_views(const trimul_params *p, void **aq, void **bq, void **sa, void **sb, size_t *ldq) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_mx(p))) return rc;
+    const MxLayout L = mx_layout(p->N);
+    uint8_t *base = static_cast<uint8_t *>(p->workspace);
+    if (aq) *aq = base + L.aq;
+    if (bq) *bq = base + L.bq;
+    if (sa) *sa = base + L.sa;
+    if (sb) *sb = base + L.sb;
+    if (ldq) *ldq = L.ldq;
+    return TRIMUL_OK;
+}
+
+size_t trimul_shard_workspace_size(int N, int rows) {
+    if (N < 1 || N > kMaxN || rows < 1 || rows > N) return 0;
+    return shard_ws_bytes(N, rows);
+}
+
+int trimul_prologue_rows(const void *z_rows, const void *mask_rows, const trimul_params *p, int rows, void *a,
+                         void *b, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_shard(p, rows))) return rc;
+    if (!z_rows) return TRIMUL_ERR_INVALID_ARG;
+    const size_t nz = (size_t)rows * p->N * kC * 2, nm = (size_t)rows * p->N * 2;
+    const size_t nab = (size_t)kC * rows * ld_of(p->N) * 2;
+    if ((rc = check_buffers({{z_rows, nz}}, {{a, nab}, {b, nab}}, p))) return rc;
+    // The mask needs only element alignment: rows without a 16-byte pitch are re-pitched.
+    if (mask_rows && !aligned(mask_rows, 2)) return TRIMUL_ERR_MISALIGNED;
+    if (overlap(a, nab, mask_rows, nm) || overlap(b, nab, mask_rows, nm) ||
+        overlap(mask_rows, nm, p->workspace, p->workspace_bytes))
+        return TRIMUL_ERR_ALIAS;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    const void *dev[] = {z_rows, mask_rows, a, b};
+    for (const void *v : dev)
+        if ((rc = check_device_ptr(v, "shard buffer"))) return rc;
+    if ((rc = check_weights_on_device(p))) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(p, s))) return rc;
+    const Views v = views_of(p);
+    return run_prologue_tc(z_rows, mask_rows, p, rows, a, b, static_cast<uint8_t *>(p->workspace) + kHeader,
+                           ctl_of(p, v), *d, s);
+}
+
+int trimul_contract_channels(const trimul_params *p, int direction, int channels, const void *a, const void *b,
+                             void *x, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_shard(p, 1)) || (rc = check_direction(direction))) return rc;
+    if (channels < 1 || channels > kC || !a || !b) return TRIMUL_ERR_INVALID_ARG;
+    const size_t n = (size_t)channels * p->N * ld_of(p->N) * 2;
+    if ((rc = check_buffers({{a, n}, {b, n}}, {{x, n}}, p))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    const void *dev[] = {a, b, x, p->workspace};
+    for (const void *v : dev)
+        if ((rc = check_device_ptr(v, "shard buffer"))) return rc;
+    const int mn = direction == TRIMUL_INCOMING;
+    const Views v = views_of(p);
+    return run_contract_on(a, mn, b, mn, x, p->N, ld_of(p->N), ctl_of(p, v), *d,
+                           reinterpret_cast<cudaStream_t>(stream), channels);
+}
+
+int trimul_epilogue_rows(const void *z_rows, const void *x_rows, const trimul_params *p, int rows, void *out_rows,
+                         trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_shard(p, rows))) return rc;
+    if (!z_rows || !x_rows) return TRIMUL_ERR_INVALID_ARG;
+    const size_t nz = (size_t)rows * p->N * kC * 2, nx = (size_t)kC * rows * ld_of(p->N) * 2;
+    if ((rc = check_buffers({{z_rows, nz}, {x_rows, nx}}, {{out_rows, nz}}, p))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    const void *dev[] = {z_rows, x_rows, out_rows};
+    for (const void *v : dev)
+        if ((rc = check_device_ptr(v, "shard buffer"))) return rc;
+    if ((rc = check_weights_on_device(p))) return rc;
+    const Views v = views_of(p);
+    return run_epilogue_tc(z_rows, x_rows, p, rows, out_rows, ctl_of(p, v), *d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int trimul_workspace_views(const trimul_params *p, void **a, void **b, void **x, size_t *ld) {

@@ -15,20 +15,20 @@ constexpr int kC = 128;  // c_z == c_h in this version
 
 struct PrologueArgs {
     int N;
-    int jt_tiles;     // ceil(N / 128): 128-cell tiles per residue row
+    int jt_tiles;     // ceil(N / 64): 64-cell tiles per residue row
     int total_tiles;  // N * jt_tiles
     float eps;
     int has_mask;                              // mask rows arrive by TMA (tensor map `mask`)
+    const __nv_bfloat16 *w_a, *w_ag, *w_b, *w_bg;  // [128][128], put into tensor memory by the kernel
     const __nv_bfloat16 *ln_w, *ln_b;          // [128] or null
     const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
     KernelCtl ctl;
 };
 
 struct PrologueMaps {
-    CUtensorMap w[4];  // W_a, W_ag, W_b, W_bg: 2-D [128 out][128 in], box 64 x 128, swizzle 128B
-    CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 128, 1), swizzle 128B
-    CUtensorMap mask;  // 2-D (j, i) over the [N][pitch] bf16 mask, box (128, 1), no swizzle
-    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (32, 1, 32), swizzle 64B
+    CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 64, 1), swizzle 128B
+    CUtensorMap mask;  // 2-D (j, i) over the [N][pitch] bf16 mask, box (64, 1), no swizzle
+    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (64, 1, 32), swizzle 128B
 };
 
 struct ContractArgs {
@@ -69,13 +69,55 @@ size_t epilogue_tc_smem();
 cudaError_t prologue_tc_setup();
 cudaError_t epilogue_tc_setup();
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s);
-// Copies the [N][N] mask into rows of pitch ld (zero past column N), for a tensor map.
-cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int ld, cudaStream_t s);
+// Copies the [rows][N] mask into rows of pitch ld (zero past column N), for a tensor map.
+cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int rows, int ld, cudaStream_t s);
 size_t contract_tc_smem();
 cudaError_t contract_tc_setup();
 // Clusters of 2 CTAs, one 256 x 256 output tile per pair; grid = 2 x pairs.
 cudaError_t launch_contract_tc(const ContractMaps &m, const ContractArgs &a, int grid, cudaStream_t s);
 cudaError_t launch_epilogue_tc(const EpilogueMaps &m, const EpilogueArgs &a, int grid, cudaStream_t s);
+
+// ---- MXFP8 contraction (mx_tc.cu) ------------------------------------------------
+
+// Quantizer: src [128][N][ld] bf16 (operand rows m, K index k: src[c][m][k], or
+// src[c][k][m] when transposed) -> q [128][N][ldq] E4M3 (row m, k contiguous)
+// and E8M0 scales per block of 32 along k, laid out per row tile of
+// rows_per_tile rows (chunks_per_tile chunks of 128 rows) and per 128-wide K
+// chunk (512 bytes per chunk, see mx_tc.cu).
+struct MxQuantArgs {
+    const __nv_bfloat16 *src;
+    int N;
+    size_t ld;
+    uint8_t *q;
+    size_t ldq;        // multiple of 16
+    uint8_t *sf;
+    int rows_per_tile;  // 128 (A) or 192 (B)
+    int row_tiles;
+    int kchunks;       // ceil(N / 128)
+    int chunks_per_tile;
+};
+
+struct ContractMxArgs {
+    int N;
+    int ti_tiles;      // ceil(N / 256)
+    int tj_tiles;      // ceil(N / 192)
+    int total_tiles;   // 128 * ti_tiles * tj_tiles
+    int kchunks;       // ceil(N / 128)
+    int a_row_tiles;   // 2 * ti_tiles (128-row halves)
+    int b_row_tiles;   // tj_tiles
+    KernelCtl ctl;
+};
+
+struct ContractMxMaps {
+    CUtensorMap a, b;    // 3-D (k, m, c) over q [128][N][ldq] uint8, boxes (128, 128 | 96, 1), swizzle 128B
+    CUtensorMap sa, sb;  // 2-D (16 bytes, rows) over the scale arrays, boxes (16, 32 | 64)
+    CUtensorMap x;       // 3-D (j, i, c) over x, box (64, 128, 1), swizzle 128B
+};
+
+cudaError_t launch_mx_quant(const MxQuantArgs &a, int transposed, cudaStream_t s);
+cudaError_t contract_mx_setup();
+// Clusters of 2 CTAs, one 256 x 192 output tile per pair; grid = 2 x pairs.
+cudaError_t launch_contract_mx(const ContractMxMaps &m, const ContractMxArgs &a, int grid, cudaStream_t s);
 
 // ---- backward (bf16 forward intermediates, fp32 gradients) -----------------------
 

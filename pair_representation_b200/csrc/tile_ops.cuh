@@ -93,4 +93,25 @@ __device__ __forceinline__ void ln_tile_sw128(uint8_t *tile, int half_bytes, con
     ln_row_sw128<kAffine>(tile, half_bytes, (int)threadIdx.x >> 1, (int)threadIdx.x & 1, gw, gb, eps);
 }
 
+// Mean and rstd of 128 values, accumulated in fp32 around the first value
+// (which keeps E[d^2] - E[d]^2 well conditioned when |mean| >> std). Each of
+// two partner lanes (lane ^ 1) accumulates one channel half.
+struct RowStats {
+    float2 s, ss;
+    float k;
+};
+__device__ __forceinline__ void stats_add(RowStats &st, uint32_t w) {
+    const float2 d = __fadd2_rn(unpack_bf16x2(w), make_float2(-st.k, -st.k));
+    st.s = __fadd2_rn(st.s, d);
+    st.ss = __ffma2_rn(d, d, st.ss);
+}
+__device__ __forceinline__ float2 stats_finish(const RowStats &st, float eps) {
+    float s = st.s.x + st.s.y, ss = st.ss.x + st.ss.y;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const float m = s * (1.f / 128.f);
+    const float var = fmaxf(ss * (1.f / 128.f) - m * m, 0.f);
+    return make_float2(st.k + m, rsqrtf(var + eps));
+}
+
 }  // namespace trimul

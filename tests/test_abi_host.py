@@ -25,7 +25,7 @@ def _declared():
         if h.endswith(".h"):
             src = open(os.path.join(ROOT, "include", h)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names |= set(re.findall(r"\b((?:trimul|atomattn)_[a-z_]+)\s*\(", src))
+            names |= set(re.findall(r"\b((?:trimul|atomattn)_[a-z0-9_]+)\s*\(", src))
     return sorted(names)
 
 

@@ -14,7 +14,7 @@ Checked against things other than the oracle itself:
 import numpy as np
 import pytest
 
-from oracle.mx import BLOCK, e4m3_round, mx_contract, mx_quantize_blocks
+from oracle.mx import BLOCK, e4m3_round, mx_contract, mx_contract_grid, mx_quantize_blocks
 
 
 def e4m3_values():
@@ -135,3 +135,15 @@ def test_planted_mistakes_fail():
     Xb = np.exp2(np.repeat(e + 1, BLOCK, axis=1))[:, :64]
     coarse = e4m3_round(a / Xb) * Xb
     assert np.abs(coarse - mx_quantize_blocks(a, 1)[2]).max() > 0
+
+
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_grid_mode_equals_full_contraction(direction):
+    """mx_contract_grid on I x I is the full mx_contract restricted to I x I."""
+    rng = np.random.default_rng(77)
+    N = 45
+    a = rng.standard_normal((N, N, 3)) * np.exp2(rng.integers(-6, 7, size=(N, 1, 3)))
+    b = rng.standard_normal((N, N, 3))
+    I = np.array([0, 3, 31, 32, 44])
+    full = mx_contract(a, b, direction)
+    np.testing.assert_array_equal(mx_contract_grid(a, b, direction, I), full[np.ix_(I, I)])
