@@ -15,8 +15,10 @@ own GPU (the layer is not sharded); value = cells of all ranks / max time.
 
 Secondary figures on rank 0 at N = 1: every workload per direction
 ("per_config"), one trimul_backward call per direction at N = 768
-("backward"; --backward-only times just that) and one windowed atom-attention
-call on 8 x 18432 atoms ("atom_attention"; --attention-only).
+("backward"; --backward-only times just that), one windowed atom-attention
+call on 8 x 18432 atoms ("atom_attention"; --attention-only) and the MXFP8
+contraction beside the bf16 one at N = 768, 2048 and 3605 ("mxfp8";
+--mxfp8-only).
 
 Timing: CUDA events on the launching stream; L2 is flushed (512 MB write)
 before every step and the flush is outside the timed events; a barrier and a
@@ -368,6 +370,84 @@ def attention_timings(tm, torch, dev, stream, peaks, warmup=3, reps=10):
     return res
 
 
+def mxfp8_timings(tm, pi, torch, dev, stream, peaks, wids=(3, 4, 5), warmup=3, reps=5):
+    """Secondary figure: the MXFP8 contraction (trimul_contract_mxfp8: quantizer and
+    block-scaled MMA kernel) beside the bf16 one (trimul_contract) on the same a, b
+    (written by the prologue), per workload and direction, CUDA events, L2 flushed
+    before each call; and the whole MXFP8 layer (trimul_forward_mxfp8) at N = 768."""
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    code = {"outgoing": tm.OUTGOING, "incoming": tm.INCOMING}
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    res = {"format": "E4M3 elements, E8M0 scale per 32 along k (OCP MX v1.0); fp32 accumulation; x in bf16"}
+    for wid in wids:
+        w = pi.WORKLOADS[wid]
+        case = pi.make_workload(w)
+        z = torch.from_numpy(case["z"]).to(dev).to(torch.bfloat16)
+        mask = torch.from_numpy(case["mask"]).to(dev).to(torch.bfloat16)
+        del case["z"]
+        sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+        layer = tm.TriangleMultiplicationOutgoing(128, 128).load_state_dict(sd).to(dev, torch.bfloat16)
+        p = layer.params(w.N)
+        ws = torch.empty(tm.trimul_workspace_size_mxfp8(w.N, 128, 128), dtype=torch.uint8, device=dev)
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+        tm.trimul_prologue(z, mask, p, stream)
+        flop = 2 * w.N ** 3 * 128
+        entry = {"N": w.N}
+        for d in w.directions:
+            t_mx = timed(lambda: tm.trimul_contract_mxfp8(p, code[d], stream))
+            t_bf = timed(lambda: tm.trimul_contract(p, code[d], stream))
+            entry[d] = {"mxfp8_us": round(t_mx, 1), "bf16_us": round(t_bf, 1),
+                        "mxfp8_tflops": round(flop / (t_mx * 1e-6) / 1e12, 1),
+                        "bf16_tflops": round(flop / (t_bf * 1e-6) / 1e12, 1),
+                        "speedup": round(t_bf / t_mx, 3)}
+        if wid == DEFAULT_WORKLOAD:
+            out = torch.empty_like(z)
+            for d in w.directions:
+                t = timed(lambda: tm.trimul_forward_mxfp8(z, mask, p, code[d], out, stream))
+                entry[d]["layer_us"] = round(t, 1)
+                entry[d]["layer_pair_cells_per_s"] = round(w.N * w.N / (t * 1e-6))
+        res[w.name] = entry
+        rc, detail = tm.trimul_device_status(p, stream)
+        if rc != 0:
+            raise RuntimeError(f"device status {rc} {detail}")
+        del z, mask, ws, layer
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_mxfp8_only(args):
+    """--mxfp8-only: the MXFP8 secondary figure alone, on one GPU."""
+    import torch
+
+    import pair_inputs as pi
+    import pair_representation_b200 as tm
+    from pair_representation_b200 import build as tmbuild
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tmbuild.build()
+    tm.lib()
+    peaks, _ = load_peaks()
+    res = mxfp8_timings(tm, pi, torch, dev, torch.cuda.current_stream(dev), peaks, warmup=args.warmup,
+                        reps=args.steps)
+    print(json.dumps({"mxfp8": res}), flush=True)
+
+
 def run_attention_only(args):
     """--attention-only: the atom-attention secondary figure alone, on one GPU."""
     import torch
@@ -570,6 +650,9 @@ def run_ours(args, rank, world, local_rank):
     attention = None
     if rank == 0 and world == 1 and not args.no_attention:
         attention = attention_timings(tm, torch, dev, stream, peaks)
+    mxfp8 = None
+    if rank == 0 and world == 1 and not args.no_mxfp8:
+        mxfp8 = mxfp8_timings(tm, pi, torch, dev, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -588,6 +671,7 @@ def run_ours(args, rank, world, local_rank):
         "per_config": configs,
         "backward": backward,
         "atom_attention": attention,
+        "mxfp8": mxfp8,
     }
     if dist:
         dist.barrier()
@@ -644,6 +728,9 @@ def main(argv=None):
     ap.add_argument("--no-attention", action="store_true", help="skip the atom-attention secondary timing")
     ap.add_argument("--attention-only", action="store_true",
                     help="time only atomattn_forward (W warm-up and K timed calls) and print that")
+    ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 secondary timing")
+    ap.add_argument("--mxfp8-only", action="store_true",
+                    help="time only the MXFP8 contraction beside the bf16 one and print that")
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=120.0)
     args = ap.parse_args(argv)
@@ -660,6 +747,8 @@ def main(argv=None):
         run_backward_only(args)
     elif args.attention_only:
         run_attention_only(args)
+    elif args.mxfp8_only:
+        run_mxfp8_only(args)
     else:
         run_ours(args, rank, world, local_rank)
 

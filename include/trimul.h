@@ -242,14 +242,12 @@ int trimul_mxfp8_views(const trimul_params *p, void **aq, void **bq, void **sa, 
  * g->workspace. The contraction's adjoint (per channel dA_c = dX_c B_c and
  * dB_c = dX_c^T A_c outgoing, dA_c = B_c dX_c^T and dB_c = A_c dX_c incoming)
  * runs on the forward's tcgen05 contraction kernel with the operands in other
- * transposes; the LayerNorm, gate and mask adjoints run in the library's own
- * kernels; the plain GEMMs (projections, weight gradients) run on cuBLAS with
- * fp32 accumulation. Weight gradients are summed per chunk of 4096
- * cells by GEMM and over the chunks in double by the library, so they do not
- * depend on how cuBLAS splits a reduction over N^2 cells; bias and LayerNorm
+ * transposes, and so do the plain GEMMs (projections, weight gradients) as
+ * batched rectangular products with fp32 accumulation; the LayerNorm, gate and
+ * mask adjoints run in the library's own per-cell kernels. No vendor library
+ * is called. Weight gradients are summed per chunk of 4096 cells by GEMM and
+ * over the chunks in double, so they are deterministic; bias and LayerNorm
  * gradients are fp32 sums (atomic, so their last bits may vary between runs).
- * cuBLAS (libcublas.so.12) is loaded on first use; one handle per device, given
- * a slice of g->workspace as its workspace, is shared by all calls under a lock.
  *
  * BF16 only in this version (TRIMUL_ERR_UNSUPPORTED for F32). dout and dz
  * must be 16-byte aligned and must not overlap each other, z, the mask or

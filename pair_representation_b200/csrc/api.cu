@@ -293,10 +293,10 @@ int map_pair(CUtensorMap *m, const void *t, int N, int rows, uint32_t b0, uint32
     return encode(m, 3, t, dims, strides, box, sw);
 }
 
-// mask [rows][pitch] as (j, i): one row segment of 64 cells per box, zero past column N.
+// mask [rows][pitch] as (j, i): one row segment of 128 cells per box, zero past column N.
 int map_mask(CUtensorMap *m, const void *t, int N, int rows, size_t pitch) {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)rows}, strides[1] = {pitch * 2};
-    const uint32_t box[2] = {64, 1};
+    const uint32_t box[2] = {128, 1};
     return encode(m, 2, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -353,7 +353,10 @@ int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int
                     void *mask_scratch, const KernelCtl &ctl, const DevState &d, cudaStream_t s) {
     const size_t ld = ld_of(p->N);
     PrologueMaps m;
-    if (int rc = map_pair(&m.z, z, p->N, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
+    for (int k = 0; k < 4; ++k)
+        if (int rc = map_weight(&m.w[k], w[k])) return rc;
+    if (int rc = map_pair(&m.z, z, p->N, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     // The mask rows travel with the z tiles. A tensor map needs a 16-byte row pitch, so a
     // mask whose rows do not have one is first copied into the scratch with pitch ld.
     m.mask = m.z;  // unused without a mask
@@ -370,19 +373,15 @@ int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int
         }
         if (int rc = map_mask(&m.mask, src, p->N, rows, pitch)) return rc;
     }
-    // Each lane quadrant stores 64 cells x 32 channels (128-byte rows, 128-byte swizzle).
-    if (int rc = map_cm(&m.a, a_out, p->N, ld, 64, 1, 32, CU_TENSOR_MAP_SWIZZLE_128B, rows)) return rc;
-    if (int rc = map_cm(&m.b, b_out, p->N, ld, 64, 1, 32, CU_TENSOR_MAP_SWIZZLE_128B, rows)) return rc;
+    // Each gating warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
+    if (int rc = map_cm(&m.a, a_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
+    if (int rc = map_cm(&m.b, b_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
     PrologueArgs a;
     a.N = p->N;
-    a.jt_tiles = (p->N + 63) / 64;
+    a.jt_tiles = (p->N + 127) / 128;
     a.total_tiles = rows * a.jt_tiles;
     a.eps = p->ln_eps;
     a.has_mask = mask != nullptr;
-    a.w_a = static_cast<const __nv_bfloat16 *>(p->w_a);
-    a.w_ag = static_cast<const __nv_bfloat16 *>(p->w_ag);
-    a.w_b = static_cast<const __nv_bfloat16 *>(p->w_b);
-    a.w_bg = static_cast<const __nv_bfloat16 *>(p->w_bg);
     a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
     a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
     a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
@@ -406,28 +405,65 @@ int run_prologue(const void *z, const void *mask, const trimul_params *p, const 
     return run_prologue_tc(z, mask, p, p->N, v.a, v.b, v.x, ctl_of(p, v), d, s);
 }
 
-// X_c[m][n] = sum_k A_c(m, k) B_c(n, k) for the 128 channels of [128][N][ld] bf16
-// arrays, each operand K-major ([rows][k]) or MN-major ([k][rows]), on the
-// tcgen05 pair kernel. CTA pairs share each 256 x 256 output tile: CTA r loads
-// rows [128 r, 128 r + 128) of the A and B panels (boxes of 128 rows, or 2 x
-// 64-wide blocks when MN-major).
-int run_contract_on(const void *A, int a_mn, const void *B, int b_mn, void *X, int N, size_t ld, const KernelCtl &ctl,
-                    const DevState &d, cudaStream_t s, int channels = kC) {
+// A matrix operand of the pair kernel: element (row, col) of batch b at
+// ptr + b * batch_stride + row * row_stride + col (elements).
+struct MatView {
+    const void *ptr;
+    size_t row_stride, batch_stride;
+};
+
+// 3-D (col, row, batch) tensor map over a MatView with `cols` x `rows` elements.
+int map_view(CUtensorMap *m, const MatView &v, int cols, int rows, int batch, uint32_t b0, uint32_t b1, int es,
+             CUtensorMapDataType dt) {
+    const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)batch};
+    // A single matrix still needs a valid (non-zero, 16-byte multiple) batch stride.
+    const size_t bs = batch > 1 ? v.batch_stride : v.row_stride * (size_t)rows;
+    const uint64_t strides[2] = {v.row_stride * es, bs * es};
+    const uint32_t box[3] = {b0, b1, 1};
+    return encode(m, 3, v.ptr, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, dt);
+}
+
+// X_b[m][n] = sum_k A_b(m, k) B_b(n, k) on the tcgen05 pair kernel for m < M,
+// n < Ncols, k < K and every batch index b; A and B bf16, each K-major
+// ([rows][k]: row = m or n) or MN-major ([k][rows]); X bf16 or fp32. CTA pairs
+// share each 256 x 256 output tile: CTA r loads rows [128 r, 128 r + 128) of the
+// A and B panels (boxes of 128 rows, or 2 x 64-wide blocks when MN-major).
+int run_gemm(const MatView &A, int a_mn, const MatView &B, int b_mn, const MatView &X, int out_f32, int M, int Ncols,
+             int K, int batch, const KernelCtl &ctl, const DevState &d, cudaStream_t s) {
     ContractMaps m;
-    if (int rc = map_cm(&m.a, A, N, ld, 64, a_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
-    if (int rc = map_cm(&m.b, B, N, ld, 64, b_mn ? 64 : 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
-    if (int rc = map_cm(&m.x, X, N, ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B, N, channels)) return rc;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (int rc = a_mn ? map_view(&m.a, A, M, K, batch, 64, 64, 2, bf) : map_view(&m.a, A, K, M, batch, 64, 128, 2, bf))
+        return rc;
+    if (int rc = b_mn ? map_view(&m.b, B, Ncols, K, batch, 64, 64, 2, bf)
+                      : map_view(&m.b, B, K, Ncols, batch, 64, 128, 2, bf))
+        return rc;
+    // X is stored by each drain warp in blocks of 32 rows x 128 bytes.
+    if (int rc = out_f32 ? map_view(&m.x, X, Ncols, M, batch, 32, 32, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                         : map_view(&m.x, X, Ncols, M, batch, 64, 32, 2, bf))
+        return rc;
     ContractArgs a;
-    a.N = N;
+    a.M = M;
+    a.Ncols = Ncols;
+    a.K = K;
     a.a_mn = a_mn;
     a.b_mn = b_mn;
-    a.ti_tiles = (N + 255) / 256;
-    a.tj_tiles = (N + 255) / 256;
-    a.total_tiles = channels * a.ti_tiles * a.tj_tiles;
-    a.kblocks = (N + 63) / 64;
+    a.ti_tiles = (M + 255) / 256;
+    a.tj_tiles = (Ncols + 255) / 256;
+    a.total_tiles = batch * a.ti_tiles * a.tj_tiles;
+    a.kblocks = (K + 63) / 64;
+    a.out_f32 = out_f32;
     a.ctl = ctl;
     const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
     return cuda_rc(launch_contract_tc(m, a, 2 * pairs, s), "contract_tc launch");
+}
+
+// The triangle contraction X_c = A_c B_c^T in general form over `channels`
+// channel-major [channels][N][ld] bf16 arrays, each operand K-major ([rows][k])
+// or MN-major ([k][rows]).
+int run_contract_on(const void *A, int a_mn, const void *B, int b_mn, void *X, int N, size_t ld, const KernelCtl &ctl,
+                    const DevState &d, cudaStream_t s, int channels = kC) {
+    const size_t cs = (size_t)N * ld;
+    return run_gemm({A, ld, cs}, a_mn, {B, ld, cs}, b_mn, {X, ld, cs}, 0, N, N, N, channels, ctl, d, s);
 }
 
 int run_contract(const trimul_params *p, int direction, const DevState &d, cudaStream_t s) {
@@ -565,7 +601,7 @@ int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cu
     if (int rc = encode(&m.sb, 2, base + L.sb, sbdims, sstr, sbbox, CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_DATA_TYPE_UINT8))
         return rc;
-    if (int rc = map_cm(&m.x, v.x, N, v.ld, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    if (int rc = map_cm(&m.x, v.x, N, v.ld, 64, 32, 1, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     ContractMxArgs a;
     a.N = N;
     a.ti_tiles = L.ti;
@@ -581,14 +617,13 @@ int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cu
 
 // ---- backward ----------------------------------------------------------------------
 
-constexpr size_t kBlasWorkspace = 32u << 20;
 constexpr long long kWgradChunk = 4096;  // cells per weight-gradient GEMM partial
 
 long long wgrad_slots(int N) { return ((long long)N * N + kWgradChunk - 1) / kWgradChunk; }
 
 // Sections of the backward workspace (byte offsets, each 256-byte aligned).
 struct BwdLayout {
-    size_t blas, sums, wstack, st_in, st_out, zh, xh, P, Y, dxh, D, dy, dX, dA, dB, partial, total;
+    size_t sums, wstack, st_in, st_out, zh, xh, P, Y, dxh, D, dy, dX, dA, dB, partial, total;
 };
 
 BwdLayout bwd_layout(int N) {
@@ -600,7 +635,6 @@ BwdLayout bwd_layout(int N) {
         off = round_up(off + bytes, 256);
         return o;
     };
-    L.blas = take(kBlasWorkspace);
     L.sums = take((size_t)kSumCount * C * 4);
     L.wstack = take((size_t)kProjBlocks * C * C * 2);
     L.st_in = take(M * 8);
@@ -665,37 +699,7 @@ int check_backward_on_device(const void *dout, const void *dz, const trimul_grad
     return TRIMUL_OK;
 }
 
-// Enqueues one GEMM on the bound handle; 0 or TRIMUL_ERR_CUDA.
-int gemm(void *h, const Gemm &g) {
-    if (blas_gemm(h, g, g_detail, sizeof g_detail)) return TRIMUL_ERR_CUDA;
-    return TRIMUL_OK;
-}
-
-// Row-major C[M][N] = op(A) op(B), one problem, bf16 operands.
-Gemm gemm1(bool ta, bool tb, int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C, int ldc,
-           bool c_f32 = true, float beta = 0.f) {
-    Gemm g;
-    g.ta = ta;
-    g.tb = tb;
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.A = A;
-    g.lda = lda;
-    g.sA = 0;
-    g.B = B;
-    g.ldb = ldb;
-    g.sB = 0;
-    g.beta = beta;
-    g.C = C;
-    g.c_f32 = c_f32;
-    g.ldc = ldc;
-    g.sC = 0;
-    g.batch = 1;
-    return g;
-}
-
-// The backward's launch sequence; the caller holds blas_lock().
+// The backward's launch sequence.
 int run_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout, void *dz,
                  const trimul_grads *gr, const DevState &d, cudaStream_t s) {
     typedef __nv_bfloat16 bf;
@@ -746,12 +750,15 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     lf.stats = st_out;
     if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
 
-    void *h = nullptr;
-    if (blas_bind(s, base + L.blas, kBlasWorkspace, &h, g_detail, sizeof g_detail)) return TRIMUL_ERR_CUDA;
+    // The plain GEMMs run on the pair kernel (run_gemm): X[m][n] = sum_k A(m, k) B(n, k),
+    // each operand K-major or MN-major (mn = 1), bf16 in, fp32 accumulation.
+    const KernelCtl ctl = ctl_of(p, v);
     const int M = (int)cells, PB = kProjBlocks * C;
     // P = zh [W_g; W_a; W_ag; W_b; W_bg]^T and Y = xh W_o^T (before biases), bf16.
-    if ((rc = gemm(h, gemm1(false, true, M, PB, C, zh, C, wstack, C, P, PB, false)))) return rc;
-    if ((rc = gemm(h, gemm1(false, true, M, C, C, xh, C, p->w_o, C, Y, C, false)))) return rc;
+    if ((rc = run_gemm({zh, (size_t)C, 0}, 0, {wstack, (size_t)C, 0}, 0, {P, (size_t)PB, 0}, 0, M, PB, C, 1, ctl, d,
+                       s)) ||
+        (rc = run_gemm({xh, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 0, {Y, (size_t)C, 0}, 0, M, C, C, 1, ctl, d, s)))
+        return rc;
 
     GateBwdArgs ga;
     ga.dout = static_cast<const bf *>(dout);
@@ -766,8 +773,10 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     ga.cells = cells;
     if ((rc = cuda_rc(launch_gate_bwd(ga, d.sms, s), "gate_bwd launch"))) return rc;
 
-    // dL/dxh = dy W_o (fp32).
-    if ((rc = gemm(h, gemm1(false, false, M, C, C, dy, C, p->w_o, C, dxh, C)))) return rc;
+    // dL/dxh = dy W_o (fp32): B(n, k) = W_o[k][n] is MN-major.
+    if ((rc = run_gemm({dy, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 1, {dxh, (size_t)C, 0}, 1, M, C, C, 1, ctl, d,
+                       s)))
+        return rc;
 
     LnBwdArgs lb;
     lb.dh = dxh;
@@ -790,7 +799,6 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     //   incoming (x_ij = sum_k a_ki b_kj):
     //     dA[k][i] = sum_j b[k][j] dX[i][j]   A = b (K-major), B = dX (K-major)
     //     dB[k][j] = sum_i a[k][i] dX[i][j]   A = a (K-major), B = dX (MN-major)
-    const KernelCtl ctl = ctl_of(p, v);
     if (direction == TRIMUL_OUTGOING) {
         if ((rc = run_contract_on(dX, 0, v.b, 1, dA, N, v.ld, ctl, d, s)) ||
             (rc = run_contract_on(dX, 1, v.a, 1, dB, N, v.ld, ctl, d, s)))
@@ -819,24 +827,21 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     // Weight gradients, one partial per chunk of kWgradChunk cells:
     //   rows [0, 640):   D^T zh  ([W_g; W_a; W_ag; W_b; W_bg] gradients)
     //   rows [640, 768): dy^T xh (W_o gradient)
-    // then summed over the chunks in double.
+    // then summed over the chunks in double. Both operands are MN-major here (the
+    // contracted index is the cell, the row index of D, dy, zh and xh); the chunks
+    // are the GEMM's batch.
     const long long full = cells / kWgradChunk, rem = cells - full * kWgradChunk;
-    const int K = (int)kWgradChunk;
-    const long long pstride = (long long)kWgradRows * C;
-    if (full > 0) {
-        Gemm w1 = gemm1(true, false, PB, C, K, D, PB, zh, C, partial, C);
-        w1.sA = (long long)K * PB, w1.sB = (long long)K * C, w1.sC = pstride, w1.batch = (int)full;
-        Gemm w2 = gemm1(true, false, C, C, K, dy, C, xh, C, partial + (size_t)PB * C, C);
-        w2.sA = (long long)K * C, w2.sB = (long long)K * C, w2.sC = pstride, w2.batch = (int)full;
-        if ((rc = gemm(h, w1)) || (rc = gemm(h, w2))) return rc;
-    }
-    if (rem > 0) {
-        const size_t r0 = (size_t)full * kWgradChunk;
-        float *pr = partial + (size_t)full * pstride;
-        if ((rc = gemm(h, gemm1(true, false, PB, C, (int)rem, D + r0 * PB, PB, zh + r0 * C, C, pr, C))) ||
-            (rc = gemm(h, gemm1(true, false, C, C, (int)rem, dy + r0 * C, C, xh + r0 * C, C, pr + (size_t)PB * C, C))))
-            return rc;
-    }
+    const size_t ck = (size_t)kWgradChunk, pstride = (size_t)kWgradRows * C;
+    auto wgrad = [&](size_t r0, int K, int batch, float *dst) {
+        int r;
+        if ((r = run_gemm({D + r0 * PB, (size_t)PB, ck * PB}, 1, {zh + r0 * C, (size_t)C, ck * C}, 1,
+                          {dst, (size_t)C, pstride}, 1, PB, C, K, batch, ctl, d, s)))
+            return r;
+        return run_gemm({dy + r0 * C, (size_t)C, ck * C}, 1, {xh + r0 * C, (size_t)C, ck * C}, 1,
+                        {dst + (size_t)PB * C, (size_t)C, pstride}, 1, C, C, K, batch, ctl, d, s);
+    };
+    if (full > 0 && (rc = wgrad(0, (int)kWgradChunk, (int)full, partial))) return rc;
+    if (rem > 0 && (rc = wgrad((size_t)full * ck, (int)rem, 1, partial + (size_t)full * pstride))) return rc;
     WgradReduceArgs wr;
     wr.partial = partial;
     wr.slots = (int)wgrad_slots(N);
@@ -844,8 +849,11 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     for (int k = 0; k <= kProjBlocks; ++k) wr.dst[k] = wdst[k];
     if ((rc = cuda_rc(launch_wgrad_reduce(wr, s), "wgrad_reduce launch"))) return rc;
 
-    // dL/dzh = D [W_g; W_a; W_ag; W_b; W_bg] (fp32, over the spent pre-activations).
-    if ((rc = gemm(h, gemm1(false, false, M, C, PB, D, PB, wstack, C, dzh, C)))) return rc;
+    // dL/dzh = D [W_g; W_a; W_ag; W_b; W_bg] (fp32, over the spent pre-activations):
+    // B(n, k) = Wstack[k][n] is MN-major.
+    if ((rc = run_gemm({D, (size_t)PB, 0}, 0, {wstack, (size_t)C, 0}, 1, {dzh, (size_t)C, 0}, 1, M, C, PB, 1, ctl, d,
+                       s)))
+        return rc;
 
     lb.dh = dzh;
     lb.src = static_cast<const bf *>(z);
@@ -1133,10 +1141,7 @@ int trimul_backward(const void *z, const void *mask, const trimul_params *p, int
     if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
         (rc = check_device_ptr(mask, "mask")) || (rc = check_backward_on_device(dout, dz, g)))
         return rc;
-    blas_lock();
-    rc = run_backward(z, mask, p, direction, dout, dz, g, *d, reinterpret_cast<cudaStream_t>(stream));
-    blas_unlock();
-    return rc;
+    return run_backward(z, mask, p, direction, dout, dz, g, *d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t atomattn_workspace_size(void) { return kHeader; }

@@ -5,7 +5,7 @@
 // the final reduction of the weight gradients.
 //
 // These are the elementwise and per-cell steps of the backward; its GEMMs run
-// on cuBLAS (blas.cu). The per-cell kernels walk 64-cell tiles with 8 warps of
+// on the tcgen05 pair kernel (contract_tc.cu). The per-cell kernels walk 64-cell tiles with 8 warps of
 // 8 cells; lane l owns channels l, l + 32, l + 64 and l + 96, so shared-memory
 // tiles are read without bank conflicts. Every kernel issues all global loads
 // for 4 cells (read-only path) before it computes and stores, so each warp

@@ -20,6 +20,10 @@
 // Per SM this moves 32 KB of operands per K block for the same MMA work that
 // a single CTA with a 128 x 256 tile needs 48 KB for.
 //
+// The same kernel serves as the batched GEMM of the backward: M, N and K are
+// separate (ContractArgs), the batch runs where the channel does, and
+// kF32Out stores the accumulator as fp32 (32-column chunks) instead of bf16.
+//
 // Synchronisation (every wait bounded):
 //   full[s]    CTA 0: armed by CTA 0's producer for the pair's 64 KB; CTA 0's
 //              loads and CTA 1's loads (cta_group::2 TMA addressed to CTA 0's
@@ -40,8 +44,8 @@ constexpr int HALF = 128;                         // rows per CTA of A and of B
 constexpr int A_BYTES = HALF * BK * 2;            // 16 KB
 constexpr int B_BYTES = HALF * BK * 2;            // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
-constexpr int OUT_COLS = 64;
-constexpr int OUT_BYTES = HALF * OUT_COLS * 2;    // 16 KB
+constexpr int WBUF_BYTES = 32 * 128;             // 4 KB: a drain warp's 32 rows x 128 bytes (64 bf16 or 32 fp32)
+constexpr int OUT_BYTES = 4 * WBUF_BYTES;         // 16 KB: one such buffer per drain warp
 constexpr int NUM_OUT = 2;
 constexpr int TMEM_COLS = 512;
 constexpr int THREADS = 192;
@@ -50,10 +54,12 @@ constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_OUT * OUT_BYTE
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace con
 
+template <bool kF32Out>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
     contract_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmX, const ContractArgs args) {
     using namespace con;
+    constexpr int OUT_COLS = kF32Out ? 32 : 64;  // accumulator columns per stored chunk
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;
@@ -69,7 +75,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
     uint32_t *peer_phases = reinterpret_cast<uint32_t *>(peer_done + 1);  // [STAGES] (CTA 0) written by CTA 1
     uint32_t *tmem_slot = peer_phases + STAGES;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_go = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -91,7 +96,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
         mbar_init(dead, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *epi_go = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -239,18 +243,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
         }
     } else {
         // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+        // Warp q drains TMEM lanes 32q .. 32q + 31 (accumulator rows r0 ..) and stores them
+        // itself: per chunk a [32 rows][128 bytes] block through its own two 4 KB buffers and
+        // its own TMA store, so the four warps never wait on one another.
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const bool leader = (threadIdx.x == 64);
         const uint32_t tempty0 = map_to_rank(&tempty[0], 0);
         const uint32_t tempty1 = map_to_rank(&tempty[1], 0);
-        // Stores issued so far by this CTA, over all its tiles: store n stages
-        // through buffer n & 1, and before it is written the store that last used
-        // that buffer (n - 2) must have read it, which wait_group.read 1 ensures
-        // only because the count runs on across tiles. A count restarted per tile
-        // would, after a tile with an odd number of stores (one in the ragged last
-        // column of tiles), give the next tile's first chunk the buffer that the
-        // still-pending last store of that tile is reading.
+        uint8_t *wbuf = outbuf + q * 2 * WBUF_BYTES;
+        // Stores issued so far by this warp, over all its tiles: store n stages through
+        // buffer n & 1, and before it is written the store that last used that buffer
+        // (n - 2) must have read it, which wait_group.read 1 ensures only because the
+        // count runs on across tiles. A count restarted per tile would, after a tile with
+        // an odd number of stores (one in the ragged last column of tiles), give the next
+        // tile's first chunk the buffer that the still-pending last store is reading.
         int nst = 0;
         int lt = 0;
         for (int tile = pair; tile < args.total_tiles; tile += npairs, ++lt) {
@@ -260,45 +265,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
             // This CTA's accumulator rows are the A rows it loaded; accumulator columns
             // [0,128) come from CTA 0's B rows and [128,256) from CTA 1's, i.e. tile
             // columns j0 .. j0 + 255 in order.
-            const int i0 = ti * 256 + (int)rank * HALF;
+            const int r0 = ti * 256 + (int)rank * HALF + 32 * q;
             const int j0 = tj * BN;
             const int acc = lt & 1;
             const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
-            if (leader) {
-                const bool got = wait_bounded(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile);
-                if (!got) raise_abort();
-                *epi_go = got ? 1 : 0;
+            if (!warp_wait(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile)) {
+                if (lane == 0) raise_abort();
+                break;
             }
-            named_bar_sync(1, 128);
-            if (!*epi_go) break;
             tc_fence_after();
-            // Chunks whose first column is past N, and whole halves whose first row is past N,
-            // are neither read nor stored.
+            // Chunks whose first column is past the matrix, and rows past it, are neither
+            // read nor stored.
 #pragma unroll 1
             for (int ch = 0; ch < BN / OUT_COLS; ++ch) {
                 const int jst = j0 + ch * OUT_COLS;
-                if (i0 >= args.N || jst >= args.N) continue;
-                uint32_t v[64];
+                if (r0 >= args.M || jst >= args.Ncols) continue;
+                uint32_t p[32];  // the 128-byte row of this thread's accumulator row
                 const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * OUT_COLS);
-                tmem_ld32(taddr, v);
-                tmem_ld32(taddr + 32, v + 32);
-                tmem_ld_wait();
-                uint32_t p[32];
+                if (kF32Out) {
+                    tmem_ld32(taddr, p);
+                    tmem_ld_wait();
+                } else {
+                    uint32_t v[64];
+                    tmem_ld32(taddr, v);
+                    tmem_ld32(taddr + 32, v + 32);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int k = 0; k < 32; ++k) p[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-                uint8_t *ob = outbuf + (nst & 1) * OUT_BYTES;
+                    for (int k = 0; k < 32; ++k)
+                        p[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                }
+                uint8_t *ob = wbuf + (nst & 1) * WBUF_BYTES;
                 ++nst;
-                if (leader) tma_store_wait_read<1>();
-                named_bar_sync(1, 128);
+                if (lane == 0) tma_store_wait_read<1>();
+                __syncwarp();
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
                     uint4 val = make_uint4(p[4 * c16], p[4 * c16 + 1], p[4 * c16 + 2], p[4 * c16 + 3]);
-                    *reinterpret_cast<uint4 *>(ob + row * 128 + ((c16 ^ (row & 7)) << 4)) = val;
+                    *reinterpret_cast<uint4 *>(ob + lane * 128 + ((c16 ^ (lane & 7)) << 4)) = val;
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (leader) {
-                    tma_store_3d(&tmX, ob, jst, i0, c);
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tmX, ob, jst, r0, c);
                     tma_store_commit();
                 }
             }
@@ -307,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
         }
-        if (leader) tma_store_wait_all<0>();
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();
@@ -322,11 +330,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(con::THREADS, 1)
 size_t contract_tc_smem() { return con::SMEM; }
 
 cudaError_t contract_tc_setup() {
-    return cudaFuncSetAttribute(contract_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)con::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(contract_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)con::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(contract_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)con::SMEM);
 }
 
 cudaError_t launch_contract_tc(const ContractMaps &m, const ContractArgs &a, int grid, cudaStream_t s) {
-    contract_tc_kernel<<<grid, con::THREADS, con::SMEM, s>>>(m.a, m.b, m.x, a);
+    if (a.out_f32)
+        contract_tc_kernel<true><<<grid, con::THREADS, con::SMEM, s>>>(m.a, m.b, m.x, a);
+    else
+        contract_tc_kernel<false><<<grid, con::THREADS, con::SMEM, s>>>(m.a, m.b, m.x, a);
     return cudaGetLastError();
 }
 

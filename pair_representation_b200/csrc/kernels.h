@@ -15,35 +15,39 @@ constexpr int kC = 128;  // c_z == c_h in this version
 
 struct PrologueArgs {
     int N;
-    int jt_tiles;     // ceil(N / 64): 64-cell tiles per residue row
-    int total_tiles;  // N * jt_tiles
+    int jt_tiles;     // ceil(N / 128): 128-cell tiles per residue row
+    int total_tiles;  // rows * jt_tiles (rows = N for the whole layer, fewer for a row shard)
     float eps;
     int has_mask;                              // mask rows arrive by TMA (tensor map `mask`)
-    const __nv_bfloat16 *w_a, *w_ag, *w_b, *w_bg;  // [128][128], put into tensor memory by the kernel
     const __nv_bfloat16 *ln_w, *ln_b;          // [128] or null
     const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
     KernelCtl ctl;
 };
 
 struct PrologueMaps {
-    CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 64, 1), swizzle 128B
-    CUtensorMap mask;  // 2-D (j, i) over the [N][pitch] bf16 mask, box (64, 1), no swizzle
-    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][N][ld], box (64, 1, 32), swizzle 128B
+    CUtensorMap w[4];  // W_a, W_ag, W_b, W_bg: 2-D [128 out][128 in], box 64 x 128, swizzle 128B
+    CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 128, 1), swizzle 128B
+    CUtensorMap mask;  // 2-D (j, i) over the [rows][pitch] bf16 mask, box (128, 1), no swizzle
+    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][rows][ld], box (32, 1, 32), swizzle 64B
 };
 
+// X[c][m][n] = sum_k A_c(m, k) B_c(n, k) for m < M, n < Ncols, k < K and every
+// batch index c (a channel of the contraction, or a chunk of the backward's
+// GEMMs): the triangle contraction is M = Ncols = K = N over 128 channels.
 struct ContractArgs {
-    int N;
+    int M, Ncols, K;
     int a_mn, b_mn;   // operand storage: 0 = K-major [rows][k], 1 = MN-major [k][rows]
-    int ti_tiles;     // ceil(N / 256)
-    int tj_tiles;     // ceil(N / 256)
-    int total_tiles;  // 128 * ti_tiles * tj_tiles
-    int kblocks;      // ceil(N / 64)
+    int ti_tiles;     // ceil(M / 256)
+    int tj_tiles;     // ceil(Ncols / 256)
+    int total_tiles;  // batch * ti_tiles * tj_tiles
+    int kblocks;      // ceil(K / 64)
+    int out_f32;      // X is fp32 (else bf16)
     KernelCtl ctl;
 };
 
 struct ContractMaps {
     CUtensorMap a, b;  // K-major: box (64 k, 128 rows, 1); MN-major: box (64 rows, 64 k, 1); swizzle 128B
-    CUtensorMap x;     // 3-D (j, i, c) over x, box (64, 128, 1), swizzle 128B
+    CUtensorMap x;     // 3-D (n, m, c) over X, box (64 bf16 | 32 fp32, 32, 1), swizzle 128B
 };
 
 struct EpilogueArgs {
@@ -111,7 +115,7 @@ struct ContractMxArgs {
 struct ContractMxMaps {
     CUtensorMap a, b;    // 3-D (k, m, c) over q [128][N][ldq] uint8, boxes (128, 128 | 96, 1), swizzle 128B
     CUtensorMap sa, sb;  // 2-D (16 bytes, rows) over the scale arrays, boxes (16, 32 | 64)
-    CUtensorMap x;       // 3-D (j, i, c) over x, box (64, 128, 1), swizzle 128B
+    CUtensorMap x;       // 3-D (j, i, c) over x, box (64, 32, 1), swizzle 128B
 };
 
 cudaError_t launch_mx_quant(const MxQuantArgs &a, int transposed, cudaStream_t s);
@@ -199,36 +203,6 @@ cudaError_t launch_ln_bwd(const LnBwdArgs &a, int sms, cudaStream_t s);
 cudaError_t launch_gate_bwd(const GateBwdArgs &a, int sms, cudaStream_t s);
 cudaError_t launch_proj_bwd(const ProjBwdArgs &a, int sms, cudaStream_t s);
 cudaError_t launch_wgrad_reduce(const WgradReduceArgs &a, cudaStream_t s);
-
-// ---- cuBLAS, loaded on first use (blas.cu) ------------------------------------
-
-// Row-major C = op(A) op(B) (bf16 operands, fp32 accumulation), batched with
-// element strides; op(X) = X^T when tX. C is fp32 when c_f32, else bf16.
-struct Gemm {
-    bool ta, tb;
-    int M, N, K;
-    const void *A;
-    int lda;
-    long long sA;
-    const void *B;
-    int ldb;
-    long long sB;
-    float beta;
-    void *C;
-    bool c_f32;
-    int ldc;
-    long long sC;
-    int batch;
-};
-
-// Serialises use of the per-device handles.
-void blas_lock();
-void blas_unlock();
-// With the lock held: the current device's handle, bound to stream s and the
-// given workspace. Returns 0, or -1 with a message in detail.
-int blas_bind(cudaStream_t s, void *ws, size_t ws_bytes, void **handle, char *detail, size_t detail_n);
-// Returns 0, or the cuBLAS status with a message in detail.
-int blas_gemm(void *handle, const Gemm &g, char *detail, size_t detail_n);
 
 // ---- sequence-local atom attention (atomattn_tc.cu) ---------------------------
 

@@ -157,7 +157,8 @@ constexpr int SFA_BYTES = 512;                  // 128 rows x 4 blocks
 constexpr int SFB_BYTES = 1024;                 // 2 x 128 rows x 4 blocks
 constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int OUT_COLS = 64;
-constexpr int OUT_BYTES = HALF_M * OUT_COLS * 2;  // 16 KB
+constexpr int WBUF_BYTES = 32 * 128;            // 4 KB: a drain warp's 32 rows x 64 bf16
+constexpr int OUT_BYTES = 4 * WBUF_BYTES;       // 16 KB: one such buffer per drain warp
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_SF = 2 * BN;             // 384: scales of stage s at 384 + 12 s
@@ -236,7 +237,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cmx::THREADS, 1)
     uint32_t *peer_phases = reinterpret_cast<uint32_t *>(peer_done + 1);
     uint32_t *tmem_slot = peer_phases + STAGES;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_go = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -257,7 +257,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cmx::THREADS, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *epi_go = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -389,12 +388,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cmx::THREADS, 1)
         }
     } else {
         // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+        // Warp q drains TMEM lanes 32q .. 32q + 31 (accumulator rows r0 ..) and stores them
+        // itself: per chunk a [32 rows][128 bytes] block through its own two 4 KB buffers and
+        // its own TMA store, so the four warps never wait on one another.
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const bool leader = (threadIdx.x == 64);
         const uint32_t tempty0 = map_to_rank(&tempty[0], 0);
         const uint32_t tempty1 = map_to_rank(&tempty[1], 0);
-        int nst = 0;  // stores issued by this CTA over all its tiles (buffer nst & 1)
+        uint8_t *wbuf = outbuf + q * 2 * WBUF_BYTES;
+        // Stores issued so far by this warp, over all its tiles: store n stages through
+        // buffer n & 1, and before it is written the store that last used that buffer
+        // (n - 2) must have read it, which wait_group.read 1 ensures only because the
+        // count runs on across tiles. A count restarted per tile would, after a tile with
+        // an odd number of stores (one in the ragged last column of tiles), give the next
+        // tile's first chunk the buffer that the still-pending last store is reading.
+        int nst = 0;
         int lt = 0;
         for (int tile = pair; tile < args.total_tiles; tile += npairs, ++lt) {
             const int c = tile / tiles_per_c;
@@ -402,52 +409,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cmx::THREADS, 1)
             const int ti = r / args.tj_tiles, tj = r - ti * args.tj_tiles;
             // Accumulator rows: the A rows this CTA loaded; columns [0, 96) from CTA 0's B
             // rows and [96, 192) from CTA 1's, i.e. tile columns j0 .. j0 + 191 in order.
-            const int i0 = ti * BM + (int)rank * HALF_M;
+            const int r0 = ti * BM + (int)rank * HALF_M + 32 * q;
             const int j0 = tj * BN;
             const int acc = lt & 1;
             const uint32_t acc_par = (uint32_t)(lt >> 1) & 1u;
-            if (leader) {
-                const bool got = wait_bounded(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile);
-                if (!got) raise_abort();
-                *epi_go = got ? 1 : 0;
+            if (!warp_wait(&tfull[acc], acc_par, abort_flag, ctl, SITE_CON | 4, tile)) {
+                if (lane == 0) raise_abort();
+                break;
             }
-            named_bar_sync(1, 128);
-            if (!*epi_go) break;
             tc_fence_after();
+            // Chunks whose first column is past the matrix, and rows past it, are neither
+            // read nor stored.
 #pragma unroll 1
             for (int ch = 0; ch < BN / OUT_COLS; ++ch) {
                 const int jst = j0 + ch * OUT_COLS;
-                if (i0 >= args.N || jst >= args.N) continue;
-                uint32_t v[64];
+                if (r0 >= args.N || jst >= args.N) continue;
+                uint32_t p[32];  // the 128-byte row of this thread's accumulator row
                 const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * OUT_COLS);
+                uint32_t v[64];
                 tmem_ld32(taddr, v);
                 tmem_ld32(taddr + 32, v + 32);
                 tmem_ld_wait();
-                uint32_t pk[32];
 #pragma unroll
                 for (int k = 0; k < 32; ++k)
-                    pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-                uint8_t *ob = outbuf + (nst & 1) * OUT_BYTES;
+                    p[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                uint8_t *ob = wbuf + (nst & 1) * WBUF_BYTES;
                 ++nst;
-                if (leader) tma_store_wait_read<1>();
-                named_bar_sync(1, 128);
+                if (lane == 0) tma_store_wait_read<1>();
+                __syncwarp();
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
-                    uint4 val = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-                    *reinterpret_cast<uint4 *>(ob + row * 128 + ((c16 ^ (row & 7)) << 4)) = val;
+                    uint4 val = make_uint4(p[4 * c16], p[4 * c16 + 1], p[4 * c16 + 2], p[4 * c16 + 3]);
+                    *reinterpret_cast<uint4 *>(ob + lane * 128 + ((c16 ^ (lane & 7)) << 4)) = val;
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (leader) {
-                    tma_store_3d(&tmX, ob, jst, i0, c);
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tmX, ob, jst, r0, c);
                     tma_store_commit();
                 }
             }
+            // Every TMEM read of this accumulator is complete: hand it back to the MMA.
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc ? tempty1 : tempty0);
         }
-        if (leader) tma_store_wait_all<0>();
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();

@@ -10,90 +10,78 @@
 // triangle multiplication"), written straight into the channel-major
 // [128][N][ld] bf16 layout the contraction's TMA reads.
 //
-// The LayerNorm is folded into the projections. With the cell's mean mu and
-// rstd r, and W' = W diag(gamma):
-//   W LN(z) + bias = r (W' z - mu s) + t,   s[c] = sum_k W'[c][k],
-//                                            t[c] = sum_k W[c][k] beta[k] + bias[c],
-// so the MMAs read the raw z tile exactly as TMA lands it and no warp ever
-// writes to it. s is summed from the bf16 W' the MMA reads, so the mean term
-// cancels as it would in exact arithmetic.
-//
-// The projection is computed transposed, D[c][cell] = W'[c][:] . z[cell][:]:
-// the four weights live in tensor memory as the MMA's A operand (lane = output
-// channel c, 64 columns of packed bf16 pairs each), z is the K-major B operand
-// in shared memory, and the accumulator has one channel per TMEM lane and one
-// cell per column - already the channel-major order of a and b. The gate
-// weights are halved when they are put in tensor memory (exact in bf16), so the
-// gate accumulator holds g / 2 and sigmoid(g) = (1 + tanh(g / 2)) / 2.
-//
-// Tiles are 64 consecutive cells of one residue row, z[i][j0 .. j0+63][:], one
-// contiguous 16 KB block. Tensor memory: weights in columns 0..255, the
-// accumulators of one tile in 256..511 (a values, a gates, b values, b gates,
-// 64 columns each). Shared memory holds no weights, which leaves room for a
-// ring of 8 z tiles: 128 KB of loads in flight per SM. Roles (448 threads),
-// coupled only through mbarriers:
-//   warp 12 (producer): TMA loads of z and of the tile's mask row segment, up
-//     to 8 tiles ahead.
-//   warp 13 (MMA): per tile the a-half (D_av, D_ag) and the b-half (D_bv, D_bg),
-//     M = 128 channels, N = 64 cells, K = 128, each half issued as soon as its
-//     accumulator columns are free.
-//   warps 8-11 (statistics): mean and rstd of each cell of a landed tile (two
-//     threads per cell, fp32 around the cell's first value) into a per-slot
-//     table.
-//   warps 0-7 (gaters): warp w reads TMEM lanes 32 (w % 4) .. (32 channels) and
-//     columns of cells 32 (w / 4) .. + 31, forms
-//       mask * (1 + tanh(r D_g - mu r s_g + t_g)) / 2 * (r D_v - mu r s_v + t_v)
-//     in packed fp32x2 and writes each channel's 32 results (64 bytes) into a
-//     [32 ch][64 cells] staging buffer shared by the two warps of its lane
-//     quadrant, which one of them stores with TMA: 128-byte rows of a or b.
+// Tiles are 128 consecutive cells of one residue row (z[i][j0 .. j0+127][:],
+// one contiguous 32 KB block). The four weight matrices (128 KB bf16) stay in
+// shared memory for the whole persistent CTA. Roles (416 threads), coupled
+// only through mbarriers:
+//   warp 12 (control): TMA loads of z (two tiles ahead), the two projection
+//     MMAs per tile (a-half D[:, 0:256] = zh [W_a; W_ag]^T, b-half
+//     D[:, 256:512] = zh [W_b; W_bg]^T, M = 128 cells, N = 256, K = 128, all
+//     512 TMEM columns).
+//   warps 8-11 (normalisers): LayerNorm of each landed tile in place (fp32
+//     statistics, two threads per cell), ahead of its MMAs.
+//   warps 0-7 (workers): gating of 32 cells x 32 channels of a and of b: TMEM
+//     is read in the 16-lane fragment layout, m * sigmoid(g) * v is formed in
+//     packed fp32x2, the bf16 results are written channel-major with
+//     stmatrix.trans into a 64-byte-swizzled 2 KB buffer of the warp and
+//     stored by that warp's own TMA store, so no warp waits on global writes.
+// The control warp issues the next tile's a-half MMAs as soon as that tile is
+// normalised and the workers have read the a-half columns, and the b-half as
+// soon as they have read the b-half columns: tensor work, gating,
+// normalisation and the z loads of two tiles ahead overlap. Every wait sleeps
+// in mbarrier.try_wait rather than spinning, which keeps issue slots and the
+// shared-memory pipe free for the warps doing work.
 #include "kernels.h"
 #include "tile_ops.cuh"
 
 namespace trimul {
 namespace pro {
-constexpr int TILE = 64;                        // cells per tile
-constexpr int SLOTS = 8;                        // z ring depth
-constexpr int GATERS = 8;
-constexpr int STATW = 4;
-constexpr int PROD_WARP = GATERS + STATW;       // 12
-constexpr int MMA_WARP = PROD_WARP + 1;         // 13
-constexpr int THREADS = 32 * (MMA_WARP + 1);    // 448
-constexpr int Z_HALF = TILE * 128;              // 8 KB: 64 cells x 64 channels
-constexpr int Z_BYTES = 2 * Z_HALF;             // 16 KB
-constexpr int MASK_BYTES = TILE * 2;            // one bf16 mask row segment per tile
-constexpr int STG_BYTES = 32 * TILE * 2;        // 4 KB: [32 ch][64 cells] bf16, 128-byte rows, 128-byte swizzle
-constexpr int NUM_STG = 8;                      // [lane quadrant][a | b]
-constexpr int STAT_BYTES = TILE * 8;            // per slot: (r, r, -mu r, -mu r) per cell pair
-constexpr int CST_FLOATS = 8 * 128;             // (s, t) of a values, a gates, b values, b gates per channel
-constexpr int BAR_BYTES = 256;
-constexpr uint32_t COL_W = 0;                   // W_a', W_ag'/2, W_b', W_bg'/2: 64 columns each
-constexpr uint32_t COL_D = 256;                 // D_av, D_ag, D_bv, D_bg: 64 columns each
-constexpr size_t SMEM = 1024 + (size_t)SLOTS * Z_BYTES + (size_t)NUM_STG * STG_BYTES + SLOTS * MASK_BYTES +
-                        SLOTS * STAT_BYTES + CST_FLOATS * 4 + BAR_BYTES;
+constexpr int TILE = 128;
+constexpr int WORKERS = 8;
+constexpr int NORMS = 4;
+constexpr int CTRL_WARP = WORKERS + NORMS;
+constexpr int THREADS = 32 * (CTRL_WARP + 1);
+constexpr int W_HALF = 512 * 128;       // one 64-channel K half of the 4 stacked weights: 64 KB
+constexpr int W_BYTES = 2 * W_HALF;     // 128 KB
+constexpr int Z_HALF = TILE * 128;      // 16 KB
+constexpr int Z_BYTES = 2 * Z_HALF;     // 32 KB
+constexpr int ST_BYTES = 32 * 32 * 2;   // 2 KB per warp buffer: [32 ch][32 cells], 64-byte swizzle
+constexpr int ST_PER_WARP = 2;
+constexpr int MASK_SLOTS = 4;           // mask rows of tiles lt .. lt + 3 (indexed lt % 4)
+constexpr int MASK_BYTES = TILE * 2;     // one bf16 mask row segment per tile
+constexpr int BAR_BYTES = 128;
+constexpr size_t SMEM = 1024 + (size_t)W_BYTES + 2 * Z_BYTES + (size_t)WORKERS * ST_PER_WARP * ST_BYTES +
+                        MASK_SLOTS * MASK_BYTES + BAR_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pro
 
+// kVec: some LayerNorm affine or projection bias is present (general path);
+// without them the kernel skips every per-channel vector access.
+template <bool kVec>
 __global__ void __launch_bounds__(pro::THREADS, 1)
-    prologue_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmMask,
-                       const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const PrologueArgs args) {
+    prologue_tc_kernel(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWag,
+                       const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmWbg,
+                       const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmMask,
+                       const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, const PrologueArgs args) {
     using namespace pro;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *zsm = smem;                                     // [SLOTS] z tiles: [2 ch halves][64 cells][64 ch]
-    uint8_t *stg = zsm + SLOTS * Z_BYTES;                    // [4 quadrants][a | b] staging
-    uint8_t *msm = stg + NUM_STG * STG_BYTES;                // [SLOTS] mask rows (bf16)
-    float4 *stats = reinterpret_cast<float4 *>(msm + SLOTS * MASK_BYTES);  // [SLOTS][32 cell pairs]
-    float *cst = reinterpret_cast<float *>(stats + SLOTS * (TILE / 2));    // [8][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(cst + CST_FLOATS);
-    uint64_t *zfull = bars;                   // [SLOTS] z tile (and mask row) landed
-    uint64_t *stat_done = bars + SLOTS;       // [SLOTS] statistics written (4 arrivals)
-    uint64_t *tile_done = bars + 2 * SLOTS;   // [SLOTS] gaters done with the slot's z, mask and statistics (8)
-    uint64_t *mma_h = bars + 3 * SLOTS;       // [2] a-half / b-half MMAs done
-    uint64_t *free_h = mma_h + 2;             // [2] gaters have read the a-half / b-half accumulators (8)
-    uint64_t *wready = free_h + 2;            // weights are in tensor memory (8)
-    uint64_t *drain = wready + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint8_t *wsm = smem;
+    uint8_t *zsm = smem + W_BYTES;                 // [2] z tiles
+    uint8_t *stsm = zsm + 2 * Z_BYTES;             // [8 warps][2] staging buffers
+    uint8_t *msm = stsm + WORKERS * ST_PER_WARP * ST_BYTES;  // [4] mask rows (bf16)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(msm + MASK_SLOTS * MASK_BYTES);
+    uint64_t *wbar = bars;        // weights landed
+    uint64_t *zfull = bars + 1;   // [2] z tile landed
+    uint64_t *mma_a = bars + 3;   // a-half projections done
+    uint64_t *mma_b = bars + 4;   // b-half projections done
+    uint64_t *a_free = bars + 5;  // workers: a-half TMEM columns read (8 arrivals)
+    uint64_t *b_free = bars + 6;  // workers: b-half TMEM columns read (8 arrivals)
+    uint64_t *drain = bars + 7;
+    uint64_t *ln_done = bars + 8; // [2] normalisers: tile in z buffer b normalised (4 arrivals)
+    uint64_t *wprep = bars + 10;  // workers: gate weights halved (8 arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,21 +91,21 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                             : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SLOTS; ++s) {
-            mbar_init(&zfull[s], 1);
-            mbar_init(&stat_done[s], STATW);
-            mbar_init(&tile_done[s], GATERS);
-        }
-        for (int h = 0; h < 2; ++h) {
-            mbar_init(&mma_h[h], 1);
-            mbar_init(&free_h[h], GATERS);
-        }
-        mbar_init(wready, GATERS);
+        mbar_init(wbar, 1);
+        mbar_init(&zfull[0], 1);
+        mbar_init(&zfull[1], 1);
+        mbar_init(mma_a, 1);
+        mbar_init(mma_b, 1);
+        mbar_init(&ln_done[0], NORMS);
+        mbar_init(&ln_done[1], NORMS);
+        mbar_init(a_free, WORKERS);
+        mbar_init(b_free, WORKERS);
         mbar_init(drain, 1);
+        mbar_init(wprep, WORKERS);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == MMA_WARP) {
+    if (warp == CTRL_WARP) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -132,252 +120,253 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         j0 = (tile - i * args.jt_tiles) * TILE;
     };
 
-    if (warp == PROD_WARP) {
-        // ------------------------------ producer ------------------------------
+    if (warp == CTRL_WARP) {
+        // ------------------------------ control warp ------------------------------
         if (lane == 0) {
-            tma_prefetch_desc(&tmZ);
-            if (args.has_mask) tma_prefetch_desc(&tmMask);
-            const uint32_t bytes = Z_BYTES + (args.has_mask ? MASK_BYTES : 0);
-            bool ok = true;
-            int lt = 0;
-            for (; lt < n_local; ++lt) {
-                const int s = lt % SLOTS;
-                // Slot s last held tile lt - SLOTS: its gating (hence its MMAs and statistics) is done.
-                if (lt >= SLOTS &&
-                    !wait_bounded(&tile_done[s], (uint32_t)(lt / SLOTS - 1) & 1u, abort_flag, ctl, SITE_PRO | 1, lt)) {
-                    ok = false;
-                    break;
-                }
+            int last_load0 = -1, last_load1 = -1;
+            auto load_z = [&](int lt) {
                 int i, j0;
                 tile_coords(lt, i, j0);
-                uint8_t *dst = zsm + s * Z_BYTES;
-                mbar_arrive_expect_tx(&zfull[s], bytes);
-                tma_load_3d(dst, &tmZ, &zfull[s], 0, j0, i);
-                tma_load_3d(dst + Z_HALF, &tmZ, &zfull[s], 64, j0, i);
-                if (args.has_mask) tma_load_2d(msm + s * MASK_BYTES, &tmMask, &zfull[s], j0, i);
-            }
-            if (!ok) *abort_flag = 1;
-            // Let the last load into each slot land before shared memory is released (the
-            // consumers may have stopped early).
-            for (int t = lt - 1; t >= 0 && t >= lt - SLOTS; --t)
-                wait_drain(&zfull[t % SLOTS], (uint32_t)(t / SLOTS) & 1u, ctl.timeout_ns);
-        }
-    } else if (warp == MMA_WARP) {
-        // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, TILE, 0, 0);
-            // Accumulators of half h (a or b): values at COL_D + 128 h, gates 64 columns on.
-            auto issue_half = [&](int h, int s) {
-                const uint32_t zb = smem_u32(zsm + s * Z_BYTES);
+                if (lt & 1) last_load1 = lt; else last_load0 = lt;
+                uint8_t *dst = zsm + (lt & 1) * Z_BYTES;
+                mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES + (args.has_mask ? MASK_BYTES : 0));
+                tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
+                tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
+                // Mask slot lt % 4 last served tile lt - 4, whose gating ended before the b-half
+                // MMA of tile lt - 2, which this load waited for.
+                if (args.has_mask) tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
+            };
+            // D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T over K = 128.
+            auto issue_half = [&](int half, int buf) {
+                const uint32_t idesc = idesc_bf16(128, 256, 0, 0);
+                const uint32_t za = smem_u32(zsm + buf * Z_BYTES);
+                const uint32_t wb = smem_u32(wsm) + (uint32_t)(half * 256 * 128);
+                const uint32_t d = tmem_base + (uint32_t)(half * 256);
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const uint32_t d = tmem_base + COL_D + (uint32_t)(h * 128 + p * 64);
-                    const uint32_t wa = tmem_base + COL_W + (uint32_t)((2 * h + p) * 64);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t koff = (uint32_t)((kk >> 2) * Z_HALF + (kk & 3) * 32);
-                        mma_bf16_ts(d, wa + (uint32_t)(kk * 8), sdesc_sw128(zb + koff, 16, 1024), idesc,
-                                    kk ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (uint32_t)((kk >> 2) * Z_HALF + (kk & 3) * 32);
+                    const uint32_t woff = (uint32_t)((kk >> 2) * W_HALF + (kk & 3) * 32);
+                    mma_bf16(d, sdesc_sw128(za + koff, 16, 1024), sdesc_sw128(wb + woff, 16, 1024), idesc,
+                             kk ? 1u : 0u);
                 }
             };
-            bool ok = wait_bounded(wready, 0, abort_flag, ctl, SITE_PRO | 2, 0);
+            mbar_arrive_expect_tx(wbar, W_BYTES);
+            const CUtensorMap *wm[4] = {&tmWa, &tmWag, &tmWb, &tmWbg};
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+                for (int kh = 0; kh < 2; ++kh) tma_load_2d(wsm + kh * W_HALF + w * 128 * 128, wm[w], wbar, kh * 64, 0);
+            if (n_local > 0) load_z(0);
+            if (n_local > 1) load_z(1);
+            bool ok = wait_bounded(wbar, 0, abort_flag, ctl, SITE_PRO | 1, 0) &&
+                      wait_bounded(wprep, 0, abort_flag, ctl, SITE_PRO | 10, 0);
             for (int lt = 0; ok && lt < n_local; ++lt) {
-                const int s = lt % SLOTS;
-                const uint32_t ppar = (uint32_t)(lt - 1) & 1u;
-                if (!wait_bounded(&zfull[s], (uint32_t)(lt / SLOTS) & 1u, abort_flag, ctl, SITE_PRO | 3, lt) ||
-                    (lt > 0 && !wait_bounded(&free_h[0], ppar, abort_flag, ctl, SITE_PRO | 4, lt))) {
+                const uint32_t par = (uint32_t)lt & 1u, ppar = (uint32_t)(lt - 1) & 1u;
+                if (!wait_bounded(&ln_done[lt & 1], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 2, lt) ||
+                    (lt > 0 && !wait_bounded(a_free, ppar, abort_flag, ctl, SITE_PRO | 3, lt))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                issue_half(0, s);
-                mma_commit(&mma_h[0]);
-                if (lt > 0 && !wait_bounded(&free_h[1], ppar, abort_flag, ctl, SITE_PRO | 5, lt)) {
+                issue_half(0, lt & 1);
+                mma_commit(mma_a);
+                if (lt > 0 && !wait_bounded(b_free, ppar, abort_flag, ctl, SITE_PRO | 4, lt)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                issue_half(1, s);
-                mma_commit(&mma_h[1]);
+                issue_half(1, lt & 1);
+                mma_commit(mma_b);
+                if (lt + 2 < n_local) {
+                    // z buffer lt & 1 is free once both projection halves of tile lt have read it.
+                    if (!wait_bounded(mma_b, par, abort_flag, ctl, SITE_PRO | 5, lt)) {
+                        ok = false;
+                        break;
+                    }
+                    load_z(lt + 2);
+                }
             }
-            if (!ok) *abort_flag = 1;
+            if (!ok) {
+                *abort_flag = 1;
+                // Copies that may still be in flight after an abort.
+                wait_drain(wbar, 0, ctl.timeout_ns);
+                if (last_load0 >= 0) wait_drain(&zfull[0], (uint32_t)(last_load0 >> 1) & 1u, ctl.timeout_ns);
+                if (last_load1 >= 0) wait_drain(&zfull[1], (uint32_t)(last_load1 >> 1) & 1u, ctl.timeout_ns);
+            }
             mma_commit(drain);
             wait_drain(drain, 0, ctl.timeout_ns);
         }
-    } else if (warp >= GATERS) {
-        // ------------------------------ statistics ------------------------------
-        // Thread t: cell t / 2 of the tile, channel half t % 2 (its partner is lane ^ 1).
-        const int t = (warp - GATERS) * 32 + lane;
-        const int cell = t >> 1, hh = t & 1;
+    } else if (warp >= WORKERS) {
+        // ------------------------------ normalisers ------------------------------
+        const int t = (warp - WORKERS) * 32 + lane;  // 0..127: cells t/2 and 64 + t/2, channel half t % 2
         bool ok = true;
         for (int lt = 0; lt < n_local; ++lt) {
-            const int s = lt % SLOTS;
-            if (!(ok = warp_wait(&zfull[s], (uint32_t)(lt / SLOTS) & 1u, abort_flag, ctl, SITE_PRO | 6, lt))) break;
-            const uint8_t *zr = zsm + s * Z_BYTES + cell * 128;
-            RowStats st;
-            st.s = st.ss = make_float2(0.f, 0.f);
-            st.k = bf16_bits_to_float(*reinterpret_cast<const uint16_t *>(zr + ((cell & 7) << 4)));
-#pragma unroll
-            for (int kc = 0; kc < 8; ++kc) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(zr + hh * Z_HALF + ((kc ^ (cell & 7)) << 4));
-                stats_add(st, u.x);
-                stats_add(st, u.y);
-                stats_add(st, u.z);
-                stats_add(st, u.w);
-            }
-            const float2 f = stats_finish(st, args.eps);  // (mu, r)
-            if (hh == 0) {
-                float *sp = reinterpret_cast<float *>(&stats[s * (TILE / 2) + (cell >> 1)]);
-                sp[cell & 1] = f.y;
-                sp[2 + (cell & 1)] = -f.x * f.y;
-            }
+            const int b = lt & 1;
+            if (!(ok = warp_wait(&zfull[b], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 6, lt))) break;
+            uint8_t *tile = zsm + b * Z_BYTES;
+            ln_row_sw128<kVec>(tile, Z_HALF, t >> 1, t & 1, args.ln_w, args.ln_b, args.eps);
+            ln_row_sw128<kVec>(tile, Z_HALF, 64 + (t >> 1), t & 1, args.ln_w, args.ln_b, args.eps);
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&stat_done[s]);
+            if (lane == 0) mbar_arrive(&ln_done[b]);
         }
         if (!ok && lane == 0) *abort_flag = 1;
     } else {
-        // ------------------------------ gaters ------------------------------
-        const int q = warp & 3, h = warp >> 2;  // lane quadrant (channels 32q ..), cell half (cells 32h ..)
-        const int c = 32 * q + lane;            // this thread's output channel
-        const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
-
-        // Weights into tensor memory: warp half h writes W_a, W_ag (h = 0) or W_b, W_bg (h = 1),
-        // row c of each, as W' = W gamma rounded to bf16 (the gate weight also halved), and
-        // the per-channel constants s (row sum of the rounded W') and t (W beta + bias; halved
-        // for the gate) into the shared table.
-        {
-            const __nv_bfloat16 *wsrc[2] = {h ? args.w_b : args.w_a, h ? args.w_bg : args.w_ag};
-            const __nv_bfloat16 *bsrc[2] = {h ? args.b_b : args.b_a, h ? args.b_bg : args.b_ag};
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const float scale = p ? 0.5f : 1.f;
-                const uint4 *row = reinterpret_cast<const uint4 *>(wsrc[p] + (size_t)c * 128);
-                uint32_t packed[64];
-                float sum = 0.f, tb = 0.f;
+        // ------------------------------ worker warps ------------------------------
+        const int q = warp & 3, sub = warp >> 2;  // TMEM lane quadrant (cells 32q..32q+31), channel half
+        uint8_t *stw = stsm + warp * ST_PER_WARP * ST_BYTES;
+        int st_round = 0;
+        // Gate 32 cells x 32 channels of a (which = 0) or b (which = 1), channels hh*64 + sub*32 ..,
+        // and store them channel-major.
+        auto slab = [&](int which, int hh, const float (&hm)[4], int i, int j0) {
+            const int ch0 = hh * 64 + sub * 32;
+            uint32_t P[16];  // packed bf16 pairs: [hf][k][e] -> P[hf * 8 + k * 2 + e]
 #pragma unroll
-                for (int k8 = 0; k8 < 16; ++k8) {
-                    const uint4 u = __ldg(row + k8);
-                    const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t V[16], G[16];
+                const uint32_t ta = tmem_base + ((uint32_t)(q * 32 + 16 * hf) << 16) + (uint32_t)(which * 256 + ch0);
+                tmem_ld16x256_x4(ta, V);
+                tmem_ld16x256_x4(ta + 128, G);
+                tmem_ld_wait();
+                const __nv_bfloat16 *bv = which ? args.b_b : args.b_a;
+                const __nv_bfloat16 *bg = which ? args.b_bg : args.b_ag;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = 8 * k8 + 2 * e;
-                        float2 w = unpack_bf16x2(wd[e]);
-                        if (args.ln_b) tb = fmaf(w.x, __bfloat162float(args.ln_b[k]),
-                                                 fmaf(w.y, __bfloat162float(args.ln_b[k + 1]), tb));
-                        if (args.ln_w) w = __fmul2_rn(w, ld_pair_bf16(args.ln_w, k));
-                        w = __fmul2_rn(w, make_float2(scale, scale));
-                        packed[4 * k8 + e] = pack_bf16x2(w.x, w.y);
-                        const float2 wr = unpack_bf16x2(packed[4 * k8 + e]);  // the rounded W' the MMA reads
-                        sum += wr.x + wr.y;
+                for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float2 g = make_float2(__uint_as_float(G[4 * k + 2 * e]), __uint_as_float(G[4 * k + 2 * e + 1]));
+                        float2 v = make_float2(__uint_as_float(V[4 * k + 2 * e]), __uint_as_float(V[4 * k + 2 * e + 1]));
+                        // g holds (W_g zh) / 2: the gate weights were halved in shared memory.
+                        if (kVec) {
+                            const int c = ch0 + 8 * k + 2 * (lane & 3);
+                            if (bg) g = __ffma2_rn(ld_pair_bf16(bg, c), make_float2(0.5f, 0.5f), g);
+                            if (bv) v = __fadd2_rn(v, ld_pair_bf16(bv, c));
+                        }
+                        const float h2 = hm[hf * 2 + e];
+                        const float2 hh2 = make_float2(h2, h2);
+                        const float2 th = tanh2_f16(g);  // two tanh per MUFU instruction
+                        const float2 y = __fmul2_rn(__ffma2_rn(th, hh2, hh2), v);
+                        P[hf * 8 + k * 2 + e] = pack_bf16x2(y.x, y.y);
                     }
                 }
-                tmem_st64(lane_base + COL_W + (uint32_t)((2 * h + p) * 64), packed);
-                if (bsrc[p]) tb += __bfloat162float(bsrc[p][c]);
-                cst[(2 * (2 * h + p)) * 128 + c] = sum;
-                cst[(2 * (2 * h + p) + 1) * 128 + c] = scale * tb;
             }
-            tmem_st_wait();
-            tc_fence_before();
+            uint8_t *buf = stw + (st_round & 1) * ST_BYTES;
+            ++st_round;
+            if (lane == 0) tma_store_wait_read<1>();  // the store that last used `buf` has read it
             __syncwarp();
-            if (lane == 0) mbar_arrive(wready);
-        }
-        named_bar_sync(5, 32 * GATERS);  // the constant table is complete
-        // (s, t) per channel: a values, a gates, b values, b gates.
-        float2 S2[4], T2[4];
+            // Matrix mi of a stmatrix covers channels 8k.. and cells 16hf + 8e..; thread 8mi + j
+            // addresses stored row j = channel 8k + j, whose 8 cells sit in 16-byte chunk 2hf + e
+            // (64-byte swizzle: chunk ^ ((channel >> 1) & 3)).
+            const int mi = lane >> 3, j = lane & 7;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float sv = cst[(2 * m) * 128 + c], tv = cst[(2 * m + 1) * 128 + c];
-            S2[m] = make_float2(sv, sv);
-            T2[m] = make_float2(tv, tv);
-        }
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int kp = 0; kp < 4; kp += 2) {
+                    const int k = kp + (mi >> 1), e = mi & 1;
+                    const int ch = 8 * k + j, chunk = 2 * hf + e;
+                    const uint32_t addr = smem_u32(buf) + (uint32_t)(ch * 64 + ((chunk ^ ((ch >> 1) & 3)) << 4));
+                    stmatrix_x4_trans(addr, P[hf * 8 + kp * 2 + 0], P[hf * 8 + kp * 2 + 1], P[hf * 8 + kp * 2 + 2],
+                                      P[hf * 8 + kp * 2 + 3]);
+                }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(which ? &tmB : &tmA, buf, j0 + 32 * q, i, ch0);
+                tma_store_commit();
+            }
+        };
 
-        bool ok = true;
+        // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4,
+        // from the mask row that landed with the tile (zero past column N).
+        auto read_hm = [&](int lt, int j0, float (&hm)[4]) {
+            const uint16_t *mrow = reinterpret_cast<const uint16_t *>(msm + (lt & 3) * MASK_BYTES);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int jc = 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
+                if (args.has_mask)
+                    hm[c] = 0.5f * bf16_bits_to_float(mrow[jc]);
+                else
+                    hm[c] = j0 + jc < args.N ? 0.5f : 0.f;
+            }
+        };
+
+        // Halve W_ag and W_bg in place (exact in bf16): the MMAs then yield g / 2 for the tanh.
+        bool ok = warp_wait(wbar, 0, abort_flag, ctl, SITE_PRO | 11, 0);
+        if (ok) {
+#pragma unroll 1
+            for (int k = warp * 32 + lane; k < 4 * 1024; k += WORKERS * 32) {  // 4 regions x 1024 uint4
+                const int region = k >> 10;  // (K half, weight) = (0, ag), (0, bg), (1, ag), (1, bg)
+                uint4 *w4 = reinterpret_cast<uint4 *>(wsm + (region >> 1) * W_HALF + (1 + 2 * (region & 1)) * 128 * 128) +
+                            (k & 1023);
+                uint4 u = *w4;
+                const __nv_bfloat162 h = __float2bfloat162_rn(0.5f);
+                uint32_t *pw = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&pw[e]);
+                    x = __hmul2(x, h);
+                    pw[e] = *reinterpret_cast<uint32_t *>(&x);
+                }
+                *w4 = u;
+            }
+            fence_proxy_async_smem();  // read by the tensor core
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wprep);
         for (int lt = 0; ok && lt < n_local; ++lt) {
-            const int s = lt % SLOTS;
             int i, j0;
             tile_coords(lt, i, j0);
-            // The two warps of a lane quadrant share staging buffers and named barriers, so
-            // after every wait they agree (bar.red) on whether to go on.
-            ok = warp_wait(&stat_done[s], (uint32_t)(lt / SLOTS) & 1u, abort_flag, ctl, SITE_PRO | 7, lt);
-            if (!(ok = bar_red_and(6 + q, 64, ok))) break;
-            const float4 *st4 = stats + s * (TILE / 2) + 16 * h;  // this warp's 16 cell pairs
-            const uint32_t *m2 = reinterpret_cast<const uint32_t *>(msm + s * MASK_BYTES) + 16 * h;
-#pragma unroll 1
-            for (int o = 0; o < 2; ++o) {  // a, then b
-                ok = warp_wait(&mma_h[o], (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | (8 + o), lt);
-                if (!(ok = bar_red_and(6 + q, 64, ok))) break;
-                tc_fence_after();
-                uint32_t V[32], G[32];
-                const uint32_t ta = lane_base + COL_D + (uint32_t)(o * 128 + 32 * h);
-                tmem_ld32(ta, V);
-                tmem_ld32(ta + 64, G);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&free_h[o]);
-                const float2 Sv = S2[2 * o], Tv = T2[2 * o], Sg = S2[2 * o + 1], Tg = T2[2 * o + 1];
-                uint32_t P[16];
-#pragma unroll
-                for (int pp = 0; pp < 16; ++pp) {
-                    const float4 sr = st4[pp];  // (r0, r1, -mu0 r0, -mu1 r1)
-                    const float2 R = make_float2(sr.x, sr.y), NMR = make_float2(sr.z, sr.w);
-                    float2 hm;
-                    if (args.has_mask) {
-                        hm = __fmul2_rn(unpack_bf16x2(m2[pp]), make_float2(0.5f, 0.5f));
-                    } else {
-                        const int jc = j0 + 32 * h + 2 * pp;
-                        hm = make_float2(jc < args.N ? 0.5f : 0.f, jc + 1 < args.N ? 0.5f : 0.f);
-                    }
-                    const float2 v = __ffma2_rn(R, make_float2(__uint_as_float(V[2 * pp]), __uint_as_float(V[2 * pp + 1])),
-                                                __ffma2_rn(NMR, Sv, Tv));
-                    const float2 g = __ffma2_rn(R, make_float2(__uint_as_float(G[2 * pp]), __uint_as_float(G[2 * pp + 1])),
-                                                __ffma2_rn(NMR, Sg, Tg));
-                    const float2 th = make_float2(tanh_approx(g.x), tanh_approx(g.y));
-                    const float2 y = __fmul2_rn(__ffma2_rn(th, hm, hm), v);
-                    P[pp] = pack_bf16x2(y.x, y.y);
-                }
-                if (o == 1) {
-                    // Statistics and mask row of slot s are no longer needed.
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tile_done[s]);
-                }
-                // Stage [32 ch][64 cells] (row = lane, 16-byte chunk k at k ^ (row & 7)), then one
-                // TMA store of 32 rows of 128 bytes by warp h = 0 of the quadrant.
-                uint8_t *buf = stg + (2 * q + o) * STG_BYTES;
-                const bool issuer = h == 0 && lane == 0;
-                if (issuer) tma_store_wait_read<1>();  // the store that last used buf (one tile ago) has read it
-                named_bar_sync(1 + q, 64);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    *reinterpret_cast<uint4 *>(buf + lane * 128 + (((4 * h + kk) ^ (lane & 7)) << 4)) =
-                        make_uint4(P[4 * kk], P[4 * kk + 1], P[4 * kk + 2], P[4 * kk + 3]);
-                fence_proxy_async_smem();
-                named_bar_sync(1 + q, 64);
-                if (issuer) {
-                    tma_store_3d(o ? &tmB : &tmA, buf, j0, i, 32 * q);
-                    tma_store_commit();
-                }
+            const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
+            // a-half of tile lt
+            if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
+            tc_fence_after();
+            float hm[4];  // tile lt landed (its a-half MMAs ran after it was normalised)
+            read_hm(lt, j0, hm);
+            if (live) {
+                slab(0, 0, hm, i, j0);
+                slab(0, 1, hm, i, j0);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(a_free);
+            // b-half of tile lt
+            if (!(ok = warp_wait(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 9, lt))) break;
+            tc_fence_after();
+            if (live) {
+                slab(1, 0, hm, i, j0);
+                slab(1, 1, hm, i, j0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_free);
         }
         if (!ok && lane == 0) *abort_flag = 1;
-        if (h == 0 && lane == 0) tma_store_wait_all<0>();
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == MMA_WARP) tmem_dealloc(tmem_base, 512);
+    if (warp == CTRL_WARP) tmem_dealloc(tmem_base, 512);
 }
 
 size_t prologue_tc_smem() { return pro::SMEM; }
 
 cudaError_t prologue_tc_setup() {
-    return cudaFuncSetAttribute(prologue_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pro::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(prologue_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pro::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(prologue_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pro::SMEM);
 }
 
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
-    prologue_tc_kernel<<<grid, pro::THREADS, pro::SMEM, s>>>(m.z, m.mask, m.a, m.b, a);
+    const bool vec = a.ln_w || a.ln_b || a.b_a || a.b_ag || a.b_b || a.b_bg;
+    if (vec)
+        prologue_tc_kernel<true><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
+                                                                        m.a, m.b, a);
+    else
+        prologue_tc_kernel<false><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
+                                                                         m.a, m.b, a);
     return cudaGetLastError();
 }
 

@@ -158,13 +158,13 @@ def test_stage_argument_checks(L):
 # ---- backward ------------------------------------------------------------------
 
 def _bwd_layout_bytes(N):
-    """Backward workspace: cuBLAS slice, sums, weight stack, per-cell sections, then
-    one [768][128] fp32 weight-gradient partial per 4096-cell chunk."""
+    """Backward workspace: sums, weight stack, per-cell sections, then one
+    [768][128] fp32 weight-gradient partial per 4096-cell chunk."""
     r = lambda v: (v + 255) // 256 * 256
     M, C, ld = N * N, 128, (N + 7) // 8 * 8
     cm = C * N * ld
     slots = (M + 4095) // 4096
-    parts = [32 << 20, 10 * C * 4, 5 * C * C * 2, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
+    parts = [10 * C * 4, 5 * C * C * 2, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
              M * C * 4, M * 5 * C * 2, M * C * 2, cm * 2, cm * 2, cm * 2, slots * 768 * C * 4]
     return sum(r(p) for p in parts)
 
