@@ -11,7 +11,8 @@ layer is one pair-cell); algorithmic TFLOP/s is reported beside it.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 With N > 1 (launched by torchrun) every rank runs an independent replica on its
-own GPU (the layer is not sharded); value = cells of all ranks / max time.
+own GPU; value = cells of all ranks / max time. --mode sharded instead splits one
+layer over the ranks (pair_representation_b200.sharded; strong scaling).
 
 Secondary figures on rank 0 at N = 1: every workload per direction
 ("per_config"), one trimul_backward call per direction at N = 768
@@ -481,6 +482,95 @@ def run_backward_only(args):
     print(json.dumps({"backward": res}), flush=True)
 
 
+def run_sharded(args, rank, world, local_rank):
+    """--mode sharded: one layer split over the ranks (row blocks for the prologue and
+    epilogue, channel blocks for the contraction, NCCL send/recv between them;
+    pair_representation_b200.sharded). Total work is fixed as the rank count grows
+    ("scaling": "strong"): value = steps x directions x N^2 / the slowest rank's time."""
+    import torch
+
+    import pair_inputs as pi
+    import pair_representation_b200 as tm
+    from pair_representation_b200 import build as tmbuild
+    from pair_representation_b200.sharded import CudaStages, ShardedTriangleMultiplication, ShardPlan
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        tmbuild.build()
+    if world > 1:
+        dist.barrier()
+    tm.lib()
+    w = pi.WORKLOADS[args.workload]
+    N = w.N
+    plan = ShardPlan(N, world)
+    r0, r1 = plan.rows(rank)
+    z_rows = torch.from_numpy(pi.draw_z(N, 128, w.seed, w.channel_scale, True, rows=range(r0, r1))).to(dev)
+    z_rows = z_rows.to(torch.bfloat16)
+    m = pi.residue_mask(N, w.n_valid)
+    mask_rows = torch.from_numpy(pi.pair_mask(m)[r0:r1].copy()).to(dev).to(torch.bfloat16)
+    case = pi.make_workload(w, with_z=False)
+    sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+    layer = tm.TriangleMultiplicationOutgoing(128, 128).load_state_dict(sd).to(dev, torch.bfloat16)
+    p = layer.params(N)
+    ws = torch.zeros(tm.trimul_shard_workspace_size(N, r1 - r0), dtype=torch.uint8, device=dev)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    code = {"outgoing": tm.OUTGOING, "incoming": tm.INCOMING}
+    layers = {d: ShardedTriangleMultiplication(plan, rank, code[d], CudaStages(tm, p), dev, torch.bfloat16, dist)
+              for d in w.directions}
+    outs = {d: torch.empty_like(z_rows) for d in w.directions}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for d in w.directions:
+            layers[d](z_rows, mask_rows, outs[d])
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    rc, detail = tm.trimul_device_status(p)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} {detail}")
+    total_ms = 0.0
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for _ in range(args.steps):
+        flush.zero_()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total_ms += e0.elapsed_time(e1)
+    sampler.stop()
+    total_ms = max_over_ranks(total_ms, dist if world > 1 else None, dev)
+    value = args.steps * len(w.directions) * N * N / (total_ms / 1e3)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "N": N, "c_z": 128, "c_h": 128, "batch": 1,
+                       "directions": list(w.directions),
+                       "l2": "flushed (512 MB write) before every step, outside the timed events",
+                       "parallelism": f"sharded x{world}: row blocks (prologue, epilogue), channel blocks "
+                                      f"(contraction), NCCL send/recv exchanges"},
+            "gpu_launches": args.steps * len(w.directions) * 3, "clocks": sampler.summary()}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -718,6 +808,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--mode", choices=("replicas", "sharded"), default="replicas",
+                    help="replicas: every rank runs the whole layer (default); sharded: one layer split "
+                         "over the ranks")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=(1, 2, 3, 4, 5))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -749,6 +842,8 @@ def main(argv=None):
         run_attention_only(args)
     elif args.mxfp8_only:
         run_mxfp8_only(args)
+    elif args.mode == "sharded":
+        run_sharded(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -112,3 +112,23 @@ def test_shard_calls_reject_bad_arguments():
     x = torch.zeros((200, N, 64), dtype=torch.bfloat16, device=dc.z.device)
     assert tm.trimul_contract_channels(p, tm.OUTGOING, 129, x, x.clone(), x.clone(), check=False) == \
         tm.ERR["TRIMUL_ERR_INVALID_ARG"]
+
+
+def test_sharded_module_single_rank_equals_layer():
+    """The host-side module on one rank with the CUDA stages (its exchanges reduce to
+    the rank's own copies): bit-identical to trimul_forward."""
+    from pair_representation_b200.sharded import CudaStages, ShardedTriangleMultiplication
+    N = 150
+    case = pi.random_case(N, 81, bf16=True, affine=True, mask="random")
+    dc = DeviceCase(case, "bf16")
+    for d in (tm.OUTGOING, tm.INCOMING):
+        whole = torch.from_numpy(dc.forward(d))
+        p = tm.TrimulParams.from_buffer_copy(dc.p)
+        ws = torch.zeros(tm.trimul_shard_workspace_size(N, N), dtype=torch.uint8, device=dc.z.device)
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+        layer = ShardedTriangleMultiplication(ShardPlan(N, 1), 0, d, CudaStages(tm, p), dc.z.device,
+                                              torch.bfloat16, torch.distributed)
+        got = layer(dc.z, dc.mask).float().cpu()
+        torch.cuda.synchronize()
+        assert tm.trimul_device_status(p)[0] == 0
+        assert torch.equal(got, whole)
