@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(epi::THREADS, 1)
                             hg = __fmul2_rn(__ffma2_rn(nmz, sg, g), hrz);
                             ho = __fmul2_rn(__ffma2_rn(nmx, so, o), hrx);
                         }
-                        const float2 th = tanh2_f16(hg);  // two tanh per MUFU instruction
+                        const float2 th = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
                         const float2 y = __ffma2_rn(th, ho, ho);
                         p[k] = pack_bf16x2(y.x, y.y);
                     }

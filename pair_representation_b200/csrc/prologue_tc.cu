@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                         }
                         const float h2 = hm[hf * 2 + e];
                         const float2 hh2 = make_float2(h2, h2);
-                        const float2 th = tanh2_f16(g);  // two tanh per MUFU instruction
+                        const float2 th = make_float2(tanh_approx(g.x), tanh_approx(g.y));
                         const float2 y = __fmul2_rn(__ffma2_rn(th, hh2, hh2), v);
                         P[hf * 8 + k * 2 + e] = pack_bf16x2(y.x, y.y);
                     }

@@ -2,22 +2,14 @@
 // and epilogue kernels (packed fp32x2 arithmetic, bf16 storage).
 #pragma once
 
-#include <cuda_fp16.h>
-
 #include "common.cuh"
 
 namespace trimul {
 
-// tanh of two values with one hardware instruction at f16 precision
-// (tanh.approx.f16x2: relative error about 2^-11, below the 2^-9 of the bf16
-// results it feeds): the arguments are rounded to f16 (RNE; beyond the f16
-// range they become +-inf, whose tanh is +-1), evaluated, and widened back.
-__device__ __forceinline__ float2 tanh2_f16(float2 x) {
-    uint32_t h;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));  // high half <- x.y
-    asm("tanh.approx.f16x2 %0, %0;" : "+r"(h));
-    __half2 t = *reinterpret_cast<__half2 *>(&h);
-    return __half22float2(t);
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // bf16x2 bits -> (low, high) as float2.
