@@ -300,6 +300,19 @@ def backward_timings(tm, pi, torch, dev, stream, peaks, warmup=3, reps=7):
                   "pair_cells_per_s": round(N * N / (med * 1e-6)),
                   "gemm_tflops": round(N * N * backward_flops_per_cell(N) / (med * 1e-6) / 1e12, 1),
                   "min_bytes_gbs": round(N * N * BACKWARD_BYTES_PER_CELL / (med * 1e-6) / 1e9, 1)}
+        # The same call right after a forward on the same inputs, reusing its a, b and x.
+        layer(z, mask, stream=stream)
+        tr = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer.backward(z, dout, mask, stream=stream, reuse_forward=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tr.append(e0.elapsed_time(e1) * 1e3)
+        tr.sort()
+        res[d]["reuse_forward_median_us"] = round(tr[len(tr) // 2], 1)
         del layer
     res["hbm_peak_gbs"] = peaks["hbm_gbs"]
     del z, mask, dout, flush
@@ -375,7 +388,8 @@ def mxfp8_timings(tm, pi, torch, dev, stream, peaks, wids=(3, 4, 5), warmup=3, r
     """Secondary figure: the MXFP8 contraction (trimul_contract_mxfp8: quantizer and
     block-scaled MMA kernel) beside the bf16 one (trimul_contract) on the same a, b
     (written by the prologue), per workload and direction, CUDA events, L2 flushed
-    before each call; and the whole MXFP8 layer (trimul_forward_mxfp8) at N = 768."""
+    before each call; and the whole MXFP8 layer (trimul_forward_mxfp8, which
+    quantizes inside the prologue) beside the bf16 layer (trimul_forward)."""
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     code = {"outgoing": tm.OUTGOING, "incoming": tm.INCOMING}
 
@@ -416,12 +430,14 @@ def mxfp8_timings(tm, pi, torch, dev, stream, peaks, wids=(3, 4, 5), warmup=3, r
                         "mxfp8_tflops": round(flop / (t_mx * 1e-6) / 1e12, 1),
                         "bf16_tflops": round(flop / (t_bf * 1e-6) / 1e12, 1),
                         "speedup": round(t_bf / t_mx, 3)}
-        if wid == DEFAULT_WORKLOAD:
-            out = torch.empty_like(z)
-            for d in w.directions:
-                t = timed(lambda: tm.trimul_forward_mxfp8(z, mask, p, code[d], out, stream))
-                entry[d]["layer_us"] = round(t, 1)
-                entry[d]["layer_pair_cells_per_s"] = round(w.N * w.N / (t * 1e-6))
+        out = torch.empty_like(z)
+        for d in w.directions:
+            t = timed(lambda: tm.trimul_forward_mxfp8(z, mask, p, code[d], out, stream))
+            t_bf = timed(lambda: tm.trimul_forward(z, mask, p, code[d], out, stream))
+            entry[d]["layer_us"] = round(t, 1)
+            entry[d]["layer_bf16_us"] = round(t_bf, 1)
+            entry[d]["layer_speedup"] = round(t_bf / t, 3)
+            entry[d]["layer_pair_cells_per_s"] = round(w.N * w.N / (t * 1e-6))
         res[w.name] = entry
         rc, detail = tm.trimul_device_status(p, stream)
         if rc != 0:

@@ -236,8 +236,9 @@ int trimul_mxfp8_views(const trimul_params *p, void **aq, void **bq, void **sa, 
  * beta 0) still gets its gradient when its output pointer is set; a NULL output
  * pointer skips that gradient.
  *
- * The forward intermediates are recomputed: the call enqueues the prologue and
- * the contraction into p->workspace, then the backward steps, which keep their
+ * The forward intermediates are recomputed (unless g->flags has
+ * TRIMUL_BWD_REUSE_FORWARD): the call enqueues the prologue and the
+ * contraction into p->workspace, then the backward steps, which keep their
  * intermediates (bf16, with fp32 for the LayerNorm adjoints' inputs) in
  * g->workspace. The contraction's adjoint (per channel dA_c = dX_c B_c and
  * dB_c = dX_c^T A_c outgoing, dA_c = B_c dX_c^T and dB_c = A_c dX_c incoming)
@@ -262,7 +263,15 @@ typedef struct {
     float *d_ln_out_w, *d_ln_out_b;         /* [c_h] */
     void *workspace;                        /* device memory, 256-byte aligned */
     size_t workspace_bytes;                 /* >= trimul_backward_workspace_size */
+    uint32_t flags;                         /* TRIMUL_BWD_*; 0 = recompute the forward */
 } trimul_grads;
+
+/* trimul_grads.flags: p->workspace still holds the a, b and x that the last
+ * trimul_forward(z, mask, p, direction, ...) left there (same z, mask, weights,
+ * direction and workspace, nothing written to the workspace since), so the
+ * backward skips recomputing them. With any of that not true the gradients are
+ * wrong; no check is made. */
+#define TRIMUL_BWD_REUSE_FORWARD 0x1u
 
 /* Bytes of backward workspace (trimul_grads.workspace) for N. */
 size_t trimul_backward_workspace_size(int N, int c_z, int c_h);

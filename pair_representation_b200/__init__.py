@@ -26,6 +26,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libtrimul_b200.so")
 OUTGOING, INCOMING = 0, 1
 DTYPE_F32, DTYPE_BF16 = 0, 1
 DEBUG_STALL_CONTRACT = 0x1
+BWD_REUSE_FORWARD = 0x1
 
 STATUS = {
     0: "TRIMUL_OK", -1: "TRIMUL_ERR_INVALID_ARG", -2: "TRIMUL_ERR_UNSUPPORTED", -3: "TRIMUL_ERR_MISALIGNED",
@@ -80,7 +81,7 @@ class TrimulGrads(ctypes.Structure):
     """Mirror of ``trimul_grads`` in include/trimul.h (fp32 gradient outputs + backward workspace)."""
 
     _fields_ = [(f, ctypes.c_void_p) for f in GRAD_FIELDS] + [
-        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t), ("flags", ctypes.c_uint32)]
 
 
 class AtomAttnParams(ctypes.Structure):
@@ -440,11 +441,14 @@ class _TriangleMultiplication:
         trimul_forward(z, mask, p, self.direction, out, stream)
         return out
 
-    def backward(self, z, dout, mask=None, stream=None):
+    def backward(self, z, dout, mask=None, stream=None, reuse_forward=False):
         """Gradients of sum(layer(z, mask) * dout): (dz, {params field: fp32 gradient}).
 
         Every parameter gets a gradient, including the optional ones the state
-        dict left out (taken as bias 0, gamma 1, beta 0 in the forward)."""
+        dict left out (taken as bias 0, gamma 1, beta 0 in the forward). With
+        reuse_forward the call relies on the layer's last forward call having
+        been ``layer(z, mask)`` with this z and mask (its a, b and x are still in
+        the workspace) and does not recompute them."""
         import torch
         if z.dim() != 3 or z.shape[0] != z.shape[1] or z.shape[2] != self.c_z:
             raise ValueError("z must be [N, N, c_z]")
@@ -460,6 +464,7 @@ class _TriangleMultiplication:
         if getattr(self, "_bws", None) is None or self._bws.numel() < need:
             self._bws = torch.empty(need, dtype=torch.uint8, device=self.device)
         g.workspace, g.workspace_bytes = self._bws.data_ptr(), self._bws.numel()
+        g.flags = BWD_REUSE_FORWARD if reuse_forward else 0
         cz, ch = self.c_z, self.c_h
         shapes = {"w_a": (ch, cz), "w_ag": (ch, cz), "w_b": (ch, cz), "w_bg": (ch, cz), "w_g": (cz, cz),
                   "w_o": (cz, ch), "b_a": (ch,), "b_ag": (ch,), "b_b": (ch,), "b_bg": (ch,), "b_g": (cz,),

@@ -19,7 +19,7 @@ LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtrimul_b200.so")
 SOURCES = ["api.cu", "prologue_tc.cu", "contract_tc.cu", "epilogue_tc.cu", "simt_f32.cu", "noalloc.cu",
            "backward.cu", "atomattn_tc.cu", "mx_tc.cu"]
-HEADERS = ["common.cuh", "kernels.h", "tile_ops.cuh"]
+HEADERS = ["common.cuh", "kernels.h", "tile_ops.cuh", "mx_block.cuh"]
 
 
 def nvcc() -> str:

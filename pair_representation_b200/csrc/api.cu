@@ -349,13 +349,35 @@ int cuda_rc(cudaError_t e, const char *what) {
 // The bf16 prologue over a grid of rows x N cells: z [rows][N][128], mask [rows][N]
 // or null, a and b written as [128][rows][ld]. mask_scratch holds rows * ld bf16
 // for a mask whose rows lack a 16-byte pitch.
+// The launch fields every prologue mode shares (the tiling is set by the caller).
+PrologueArgs prologue_args(const trimul_params *p, bool has_mask, const KernelCtl &ctl) {
+    PrologueArgs a;
+    memset(&a, 0, sizeof a);
+    a.N = p->N;
+    a.eps = p->ln_eps;
+    a.has_mask = has_mask;
+    a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
+    a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
+    a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
+    a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
+    a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
+    a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
+    a.ctl = ctl;
+    return a;
+}
+
+int map_weights(PrologueMaps *m, const trimul_params *p) {
+    const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
+    for (int k = 0; k < 4; ++k)
+        if (int rc = map_weight(&m->w[k], w[k])) return rc;
+    return TRIMUL_OK;
+}
+
 int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int rows, void *a_out, void *b_out,
                     void *mask_scratch, const KernelCtl &ctl, const DevState &d, cudaStream_t s) {
     const size_t ld = ld_of(p->N);
     PrologueMaps m;
-    const void *w[4] = {p->w_a, p->w_ag, p->w_b, p->w_bg};
-    for (int k = 0; k < 4; ++k)
-        if (int rc = map_weight(&m.w[k], w[k])) return rc;
+    if (int rc = map_weights(&m, p)) return rc;
     if (int rc = map_pair(&m.z, z, p->N, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     // The mask rows travel with the z tiles. A tensor map needs a 16-byte row pitch, so a
     // mask whose rows do not have one is first copied into the scratch with pitch ld.
@@ -376,21 +398,11 @@ int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int
     // Each gating warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
     if (int rc = map_cm(&m.a, a_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
     if (int rc = map_cm(&m.b, b_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
-    PrologueArgs a;
-    a.N = p->N;
+    PrologueArgs a = prologue_args(p, mask != nullptr, ctl);
     a.jt_tiles = (p->N + 127) / 128;
     a.total_tiles = rows * a.jt_tiles;
-    a.eps = p->ln_eps;
-    a.has_mask = mask != nullptr;
-    a.ln_w = static_cast<const __nv_bfloat16 *>(p->ln_in_w);
-    a.ln_b = static_cast<const __nv_bfloat16 *>(p->ln_in_b);
-    a.b_a = static_cast<const __nv_bfloat16 *>(p->b_a);
-    a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
-    a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
-    a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
-    a.ctl = ctl;
     const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
-    return cuda_rc(launch_prologue_tc(m, a, grid, s), "prologue_tc launch");
+    return cuda_rc(launch_prologue_tc(m, a, PRO_BF16, grid, s), "prologue_tc launch");
 }
 
 int run_prologue(const void *z, const void *mask, const trimul_params *p, const DevState &d, cudaStream_t s) {
@@ -553,6 +565,8 @@ int check_mx(const trimul_params *p) {
     return TRIMUL_OK;
 }
 
+int run_contract_mx_mma(const trimul_params *p, const DevState &d, cudaStream_t s);
+
 int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cudaStream_t s) {
     const Views v = views_of(p);
     const int N = p->N;
@@ -581,7 +595,15 @@ int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cu
     q.row_tiles = L.tj;
     q.chunks_per_tile = 2;
     if (int rc = cuda_rc(launch_mx_quant(q, tr, s), "mx_quant launch")) return rc;
+    return run_contract_mx_mma(p, d, s);
+}
 
+// The block-scaled contraction of the MXFP8 operands already in the workspace into x.
+int run_contract_mx_mma(const trimul_params *p, const DevState &d, cudaStream_t s) {
+    const Views v = views_of(p);
+    const int N = p->N;
+    const MxLayout L = mx_layout(N);
+    uint8_t *base = static_cast<uint8_t *>(p->workspace);
     ContractMxMaps m;
     const uint64_t qdims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)kC};
     const uint64_t qstr[2] = {L.ldq, (uint64_t)N * L.ldq};
@@ -613,6 +635,87 @@ int run_contract_mx(const trimul_params *p, int direction, const DevState &d, cu
     a.ctl = ctl_of(p, v);
     const int pairs = a.total_tiles < d.sms / 2 ? a.total_tiles : d.sms / 2;
     return cuda_rc(launch_contract_mx(m, a, 2 * pairs, s), "contract_mx launch");
+}
+
+// The prologue writing the MXFP8 operands of `direction`'s contraction (E4M3 codes
+// and scales) straight into the MX sections of the workspace: outgoing on row
+// tiles, incoming on 32 x 4 column tiles (the contracted index of a_ki is the row).
+int run_prologue_mx(const void *z, const void *mask, const trimul_params *p, int direction, const DevState &d,
+                    cudaStream_t s) {
+    const Views v = views_of(p);
+    const int N = p->N;
+    const MxLayout L = mx_layout(N);
+    uint8_t *base = static_cast<uint8_t *>(p->workspace);
+    const bool cols = direction == TRIMUL_INCOMING;
+    // The contraction reads whole 128-wide K chunks: the scales of K blocks past the last
+    // residue (zero codes, no cell writes them) must be finite, so both arrays start at 0.
+    if (int rc = cuda_rc(cudaMemsetAsync(base + L.sa, 0, (size_t)kC * 2 * L.ti * L.kc * 512, s), "mx scale clear"))
+        return rc;
+    if (int rc = cuda_rc(cudaMemsetAsync(base + L.sb, 0, (size_t)kC * L.tj * L.kc * 1024, s), "mx scale clear"))
+        return rc;
+    PrologueMaps m;
+    if (int rc = map_weights(&m, p)) return rc;
+    if (cols) {
+        // (c, j, i) over z, one column's 32 rows per box.
+        const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)N};
+        const uint64_t strides[2] = {128 * 2, (uint64_t)N * 128 * 2};
+        const uint32_t box[3] = {64, 1, 32};
+        if (int rc = encode(&m.z, 3, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    } else if (int rc = map_pair(&m.z, z, N, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) {
+        return rc;
+    }
+    m.mask = m.z;  // unused without a mask
+    if (mask) {
+        // Re-pitched (row tiles) or transposed (column tiles) into plane 0 of x, which
+        // the contraction overwrites later.
+        __nv_bfloat16 *scratch = reinterpret_cast<__nv_bfloat16 *>(v.x);
+        const __nv_bfloat16 *mk = static_cast<const __nv_bfloat16 *>(mask);
+        if (cols) {
+            if (int rc = cuda_rc(launch_mask_transpose(mk, scratch, N, (int)v.ld, s), "mask_transpose launch"))
+                return rc;
+            const uint64_t dims[2] = {(uint64_t)N, (uint64_t)N}, strides[1] = {(uint64_t)v.ld * 2};
+            const uint32_t box[2] = {32, 4};
+            if (int rc = encode(&m.mask, 2, scratch, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+        } else {
+            const void *src = mask;
+            size_t pitch = (size_t)N;
+            if (N % 8 != 0 || !aligned(mask, 16)) {
+                if (int rc = cuda_rc(launch_mask_pad(mk, scratch, N, N, (int)v.ld, s), "mask_pad launch")) return rc;
+                src = scratch;
+                pitch = v.ld;
+            }
+            if (int rc = map_mask(&m.mask, src, N, N, pitch)) return rc;
+        }
+    }
+    // E4M3 operands [c][N][ldq] as (k, row, c); each gating warp stores 32 channels x 32 bytes.
+    const uint64_t qdims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)kC};
+    const uint64_t qstr[2] = {L.ldq, (uint64_t)N * L.ldq};
+    const uint32_t qbox[3] = {32, 1, 32};
+    if (int rc = encode(&m.a, 3, base + L.aq, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    if (int rc = encode(&m.b, 3, base + L.bq, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8))
+        return rc;
+    PrologueArgs a = prologue_args(p, mask != nullptr, ctl_of(p, v));
+    if (cols) {
+        a.jt_tiles = (N + 3) / 4;
+        a.total_tiles = ((N + 31) / 32) * a.jt_tiles;
+    } else {
+        a.jt_tiles = (N + 127) / 128;
+        a.total_tiles = N * a.jt_tiles;
+    }
+    a.sf[0] = base + L.sa;
+    a.sf[1] = base + L.sb;
+    a.sf_rows[0] = 128;
+    a.sf_row_tiles[0] = 2 * L.ti;
+    a.sf_chunks[0] = 1;
+    a.sf_rows[1] = 192;
+    a.sf_row_tiles[1] = L.tj;
+    a.sf_chunks[1] = 2;
+    a.kchunks = L.kc;
+    const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
+    return cuda_rc(launch_prologue_tc(m, a, cols ? PRO_MX_COLS : PRO_MX_ROWS, grid, s), "prologue_tc launch");
 }
 
 // ---- backward ----------------------------------------------------------------------
@@ -721,8 +824,11 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     const bf *x = reinterpret_cast<const bf *>(v.x);
     int rc;
 
-    // Recompute the forward's a, b and x into the forward workspace.
-    if ((rc = clear_status(p, s)) || (rc = run_prologue(z, mask, p, d, s)) || (rc = run_contract(p, direction, d, s)))
+    // Recompute the forward's a, b and x into the forward workspace, unless the caller
+    // states that the last forward call left them there.
+    if ((rc = clear_status(p, s))) return rc;
+    if (!(gr->flags & TRIMUL_BWD_REUSE_FORWARD) &&
+        ((rc = run_prologue(z, mask, p, d, s)) || (rc = run_contract(p, direction, d, s))))
         return rc;
     if ((rc = cuda_rc(cudaMemsetAsync(sums, 0, (size_t)kSumCount * C * 4, s), "backward sums clear"))) return rc;
     const void *wk[kProjBlocks] = {p->w_g, p->w_a, p->w_ag, p->w_b, p->w_bg};
@@ -1002,8 +1108,8 @@ int trimul_forward_mxfp8(const void *z, const void *mask, const trimul_params *p
         return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = clear_status(p, s))) return rc;
-    if ((rc = run_prologue(z, mask, p, *d, s))) return rc;
-    if ((rc = run_contract_mx(p, direction, *d, s))) return rc;
+    if ((rc = run_prologue_mx(z, mask, p, direction, *d, s))) return rc;
+    if ((rc = run_contract_mx_mma(p, *d, s))) return rc;
     return run_epilogue(z, p, out, *d, s);
 }
 

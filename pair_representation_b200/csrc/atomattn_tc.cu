@@ -25,7 +25,8 @@
 // quarter w & 3 and a quarter of their slots. Warp 16, one thread: TMA loads
 // (double-buffered stages) and MMA issue. Barriers, all waits bounded:
 //   full[s]  TMA bytes of stage s landed              (producer -> MMA)
-//   sfull    S of the unit is in TMEM                  (MMA commit -> warps 0-3)
+//   sfull    S of the unit is in TMEM                  (MMA commit -> warps 0-15)
+//   s_read   S of the unit is in the warps' registers  (16 warp arrivals -> MMA issues the next S)
 //   pready   P written, S and the O of two units back read (16 warp arrivals -> MMA)
 //   ofull    O of the unit is in TMEM, stage free      (MMA commit -> warps 0-3, producer)
 #include "kernels.h"
@@ -49,7 +50,7 @@ constexpr int S_COL = 0, O_COL = 256, TMEM_COLS = 512;
 constexpr int WORKER_WARPS = 16;             // 4 per TMEM lane quarter, 32 of a row's 128 slots each
 constexpr int THREADS = (WORKER_WARPS + 1) * 32;
 constexpr int RED_BYTES = 2 * 2 * 4 * ROWS * 4;  // [max, sum][unit parity][key part][row] floats
-constexpr int BAR_BYTES = 128;  // 10 mbarriers, TMEM address, abort flag
+constexpr int BAR_BYTES = 128;  // 11 mbarriers, TMEM address, abort flag
 constexpr size_t SMEM = 1024 + 2 * (size_t)STAGE_BYTES + P_BYTES + RED_BYTES + BAR_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 static_assert(SMEM <= 232448, "shared memory budget");
@@ -124,7 +125,8 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
     uint64_t *ofull = bars + 4;
     uint64_t *drain = bars + 5;
     uint64_t *redbar = bars + 6;  // [4] per lane quarter: its 4 warps published their partials
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    uint64_t *s_read = bars + 10;  // the worker warps have read S of the unit (16 warp arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         mbar_init(ofull, 1);
         mbar_init(drain, 1);
         for (int i = 0; i < 4; ++i) mbar_init(&redbar[i], 4);
+        mbar_init(s_read, WORKER_WARPS);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -200,6 +203,16 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             if (my_units > 1) issue(1);
             if (my_units > 0) ok = mma_s(0);
             for (int lu = 0; ok && lu < my_units; ++lu) {
+                if (lu + 1 < my_units) {
+                    // S of the next unit overwrites S as soon as the worker warps have read it,
+                    // so it is computed while they finish this unit's softmax.
+                    if (!wait_bounded(s_read, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 9, lu)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!(ok = mma_s(lu + 1))) break;
+                }
                 if (!wait_bounded(pready, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 2, lu)) {
                     ok = false;
                     break;
@@ -215,7 +228,6 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                     mma_bf16(od, pdesc + (uint64_t)(((kk >> 2) * P_BLOCK + (kk & 3) * 32) >> 4),
                              vdesc + (uint64_t)((kk * 2048) >> 4), idesc_o, kk ? 1u : 0u);
                 mma_commit(ofull);
-                if (lu + 1 < my_units && !(ok = mma_s(lu + 1))) break;
                 if (lu + 2 < my_units) {
                     // The stage of unit lu is free once its second product has completed.
                     if (!wait_bounded(ofull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 3, lu)) {
@@ -309,6 +321,10 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 uint32_t sv[32];
                 tmem_ld32(lanebase + (uint32_t)(S_COL + 32 * qr + 32 * kp), sv);
                 tmem_ld_wait();
+                // S is in registers: the next unit's S may overwrite it.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_read);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint4 bc = make_uint4(0u, 0u, 0u, 0u);

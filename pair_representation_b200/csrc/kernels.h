@@ -13,22 +13,41 @@ constexpr int kC = 128;  // c_z == c_h in this version
 
 // ---- bf16 tensor-core path (tcgen05 + TMA) --------------------------------
 
+// What the prologue writes:
+//   PRO_BF16     a, b in bf16, channel-major [c][rows][ld]; tiles of 128 cells of one row.
+//   PRO_MX_ROWS  a, b as MXFP8 operands of the outgoing contraction (operand row i,
+//                K = column k): E4M3 [c][N][ldq] and E8M0 scales; same tiles, each
+//                gating warp's 32 cells x 32 channels being 32 whole blocks.
+//   PRO_MX_COLS  the same for the incoming contraction (operand row = column i of
+//                a and b, K = residue row k): tiles of 32 rows x 4 columns, each
+//                gating warp holding one column's 32 rows, again 32 whole blocks.
+enum { PRO_BF16 = 0, PRO_MX_ROWS = 1, PRO_MX_COLS = 2 };
+
 struct PrologueArgs {
     int N;
-    int jt_tiles;     // ceil(N / 128): 128-cell tiles per residue row
-    int total_tiles;  // rows * jt_tiles (rows = N for the whole layer, fewer for a row shard)
+    int jt_tiles;     // PRO_BF16 / PRO_MX_ROWS: ceil(N / 128) tiles per residue row;
+                      // PRO_MX_COLS: ceil(N / 4) groups of 4 columns per block of 32 rows
+    int total_tiles;  // rows * jt_tiles (rows = N for the whole layer, fewer for a row shard);
+                      // PRO_MX_COLS: ceil(N / 32) * jt_tiles
     float eps;
     int has_mask;                              // mask rows arrive by TMA (tensor map `mask`)
     const __nv_bfloat16 *ln_w, *ln_b;          // [128] or null
     const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
+    // MXFP8 modes: the scale arrays of the A (a) and B (b) operands, in the layout the
+    // contraction reads (mx_scale_offset with these row tiles, K chunks and chunks per tile).
+    uint8_t *sf[2];
+    int sf_rows[2], sf_row_tiles[2], sf_chunks[2];
+    int kchunks;
     KernelCtl ctl;
 };
 
 struct PrologueMaps {
     CUtensorMap w[4];  // W_a, W_ag, W_b, W_bg: 2-D [128 out][128 in], box 64 x 128, swizzle 128B
-    CUtensorMap z;     // 3-D (c, j, i) over z, box (64, 128, 1), swizzle 128B
-    CUtensorMap mask;  // 2-D (j, i) over the [rows][pitch] bf16 mask, box (128, 1), no swizzle
-    CUtensorMap a, b;  // 3-D (j, i, c) over a / b [c][rows][ld], box (32, 1, 32), swizzle 64B
+    CUtensorMap z;     // 3-D (c, j, i) over z, swizzle 128B; box (64, 128, 1), PRO_MX_COLS (64, 1, 32)
+    CUtensorMap mask;  // 2-D (j, i) over the [rows][pitch] bf16 mask, box (128, 1), no swizzle;
+                       // PRO_MX_COLS: (k, i) over the transposed mask, box (32, 4)
+    CUtensorMap a, b;  // 3-D (x, row, c): PRO_BF16 over a / b [c][rows][ld], box (32, 1, 32), swizzle 64B;
+                       // MXFP8 over the E4M3 operands [c][N][ldq] (uint8), box (32, 1, 32), no swizzle
 };
 
 // X[c][m][n] = sum_k A_c(m, k) B_c(n, k) for m < M, n < Ncols, k < K and every
@@ -72,9 +91,12 @@ size_t prologue_tc_smem();
 size_t epilogue_tc_smem();
 cudaError_t prologue_tc_setup();
 cudaError_t epilogue_tc_setup();
-cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int mode, int grid, cudaStream_t s);
 // Copies the [rows][N] mask into rows of pitch ld (zero past column N), for a tensor map.
 cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int rows, int ld, cudaStream_t s);
+// dst[i][k] = mask[k][i] for i, k < N, zero for N <= k < ld (the transposed mask the
+// PRO_MX_COLS prologue reads).
+cudaError_t launch_mask_transpose(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int ld, cudaStream_t s);
 size_t contract_tc_smem();
 cudaError_t contract_tc_setup();
 // Clusters of 2 CTAs, one 256 x 256 output tile per pair; grid = 2 x pairs.

@@ -34,25 +34,14 @@
 // per row tile of the contraction (A: 128 rows, one chunk; B: 192 rows, two
 // chunks of which the second is half used) and per 128-wide K chunk, so one
 // TMA box brings a stage's scales.
-#include <cuda_fp8.h>
-
 #include "kernels.h"
+#include "mx_block.cuh"
 
 namespace trimul {
 
 // ---------------------------------------------------------------------------
 // Quantizer
 // ---------------------------------------------------------------------------
-
-// Byte offset of the scale of (row r, K block kb) of channel c in a scale array
-// laid out per row tile (rows_per_tile rows, chunks_per_tile chunks of 128 rows)
-// and per 128-wide K chunk.
-__host__ __device__ __forceinline__ size_t mx_scale_offset(int c, int r, int kb, int rows_per_tile, int row_tiles,
-                                                            int kchunks, int chunks_per_tile) {
-    const int rt = r / rows_per_tile, nl = r - rt * rows_per_tile;
-    const size_t chunk = (((size_t)c * row_tiles + rt) * kchunks + (kb >> 2)) * chunks_per_tile + (nl >> 7);
-    return chunk * 512 + (size_t)(nl & 31) * 16 + ((nl & 127) >> 5) * 4 + (kb & 3);
-}
 
 // One thread per block of 32 values: 64 rows x 4 blocks (one 128-wide K chunk)
 // of one channel per CTA. Rows >= N and columns >= N are zeros (scale byte 0);
@@ -105,25 +94,9 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(MxQuantArgs p) {
         for (int t = 0; t < 32; ++t)
             if (kb0 + t >= p.N) v[t] = 0.f;
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
-    // e = floor(log2 amax) - 8 from the exponent field, clamped to the E8M0 range; a
-    // zero block (or one below the normal range) takes the smallest scale.
-    int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 8;
-    if (amax == 0.f || e < -127) e = -127;
-    if (e > 127) e = 127;
-    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact (e <= 119 for finite bf16)
+    uint32_t q8[8];
+    const int e = mx_quantize32(v, q8);
     if (m < p.N) {
-        uint32_t q8[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const __nv_fp8x2_storage_t lo =
-                __nv_cvt_float2_to_fp8x2(make_float2(v[4 * t] * inv, v[4 * t + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-            const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-                make_float2(v[4 * t + 2] * inv, v[4 * t + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-            q8[t] = (uint32_t)lo | ((uint32_t)hi << 16);
-        }
         if (kb0 < p.ldq) {
             uint8_t *dst = p.q + ((size_t)c * p.N + m) * p.ldq + kb0;  // ldq is a multiple of 16
             *reinterpret_cast<uint4 *>(dst) = make_uint4(q8[0], q8[1], q8[2], q8[3]);

@@ -31,7 +31,19 @@
 // normalisation and the z loads of two tiles ahead overlap. Every wait sleeps
 // in mbarrier.try_wait rather than spinning, which keeps issue slots and the
 // shared-memory pipe free for the warps doing work.
+//
+// MXFP8 modes write a and b directly as the E4M3 operands of the block-scaled
+// contraction (OCP Microscaling v1.0: blocks of 32 along the contracted index,
+// one E8M0 scale each), so no separate pass reads the bf16 values back. A gating
+// warp's 32 cells x 32 channels are 32 whole blocks when its 32 cells run along
+// the contracted index: in PRO_MX_ROWS (outgoing, K = the column k of a_ik) the
+// usual row tiles already do; in PRO_MX_COLS (incoming, K = the row k of a_ki) a
+// tile is 32 rows x 4 columns, loaded column by column, so warp q holds column q.
+// The warp rounds its values to bf16 exactly as the bf16 mode stores them, then
+// each lane quantises one channel's block from the staging buffer and writes its
+// 32 codes back in place for the warp's TMA store; the lane stores the scale byte.
 #include "kernels.h"
+#include "mx_block.cuh"
 #include "tile_ops.cuh"
 
 namespace trimul {
@@ -56,8 +68,9 @@ static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pro
 
 // kVec: some LayerNorm affine or projection bias is present (general path);
-// without them the kernel skips every per-channel vector access.
-template <bool kVec>
+// without them the kernel skips every per-channel vector access. kMode: PRO_BF16,
+// PRO_MX_ROWS or PRO_MX_COLS.
+template <bool kVec, int kMode>
 __global__ void __launch_bounds__(pro::THREADS, 1)
     prologue_tc_kernel(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWag,
                        const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmWbg,
@@ -114,10 +127,18 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // Tile lt of this CTA: z row i, columns j0 .. j0+127; PRO_MX_COLS: rows i .. i+31,
+    // columns j0 .. j0+3.
     auto tile_coords = [&](int lt, int &i, int &j0) {
         const int tile = (int)blockIdx.x + lt * (int)gridDim.x;
-        i = tile / args.jt_tiles;
-        j0 = (tile - i * args.jt_tiles) * TILE;
+        const int r = tile / args.jt_tiles;
+        if (kMode == PRO_MX_COLS) {
+            i = 32 * r;
+            j0 = 4 * (tile - r * args.jt_tiles);
+        } else {
+            i = r;
+            j0 = (tile - r * args.jt_tiles) * TILE;
+        }
     };
 
     if (warp == CTRL_WARP) {
@@ -130,11 +151,26 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                 if (lt & 1) last_load1 = lt; else last_load0 = lt;
                 uint8_t *dst = zsm + (lt & 1) * Z_BYTES;
                 mbar_arrive_expect_tx(&zfull[lt & 1], Z_BYTES + (args.has_mask ? MASK_BYTES : 0));
-                tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
-                tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
+                if (kMode == PRO_MX_COLS) {
+                    // Rows i .. i+31 of column j0 + c land as cells 32c .. 32c+31.
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        tma_load_3d(dst + c * 4096, &tmZ, &zfull[lt & 1], 0, j0 + c, i);
+                        tma_load_3d(dst + Z_HALF + c * 4096, &tmZ, &zfull[lt & 1], 64, j0 + c, i);
+                    }
+                } else {
+                    tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
+                    tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
+                }
                 // Mask slot lt % 4 last served tile lt - 4, whose gating ended before the b-half
-                // MMA of tile lt - 2, which this load waited for.
-                if (args.has_mask) tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
+                // MMA of tile lt - 2, which this load waited for. PRO_MX_COLS reads the
+                // transposed mask: [4 columns][32 rows], the same cell order as z.
+                if (args.has_mask) {
+                    if (kMode == PRO_MX_COLS)
+                        tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], i, j0);
+                    else
+                        tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
+                }
             };
             // D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T over K = 128.
             auto issue_half = [&](int half, int buf) {
@@ -217,8 +253,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         uint8_t *stw = stsm + warp * ST_PER_WARP * ST_BYTES;
         int st_round = 0;
         // Gate 32 cells x 32 channels of a (which = 0) or b (which = 1), channels hh*64 + sub*32 ..,
-        // and store them channel-major.
-        auto slab = [&](int which, int hh, const float (&hm)[4], int i, int j0) {
+        // and store them channel-major at (x = ox .. ox+31, row orow).
+        auto slab = [&](int which, int hh, const float (&hm)[4], int ox, int orow) {
             const int ch0 = hh * 64 + sub * 32;
             uint32_t P[16];  // packed bf16 pairs: [hf][k][e] -> P[hf * 8 + k * 2 + e]
 #pragma unroll
@@ -268,17 +304,44 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                     stmatrix_x4_trans(addr, P[hf * 8 + kp * 2 + 0], P[hf * 8 + kp * 2 + 1], P[hf * 8 + kp * 2 + 2],
                                       P[hf * 8 + kp * 2 + 3]);
                 }
+            if (kMode != PRO_BF16) {
+                // Lane l quantises channel ch0 + l: its 32 bf16 values are buffer row l
+                // (logical 16-byte chunk c at c ^ ((l >> 1) & 3)); its 32 codes go back to
+                // bytes 32 l .. 32 l + 31, a dense [32 ch][32 B] box for the TMA store.
+                __syncwarp();
+                float v[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4));
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        v[8 * c + 2 * t] = __uint_as_float(w[t] << 16);
+                        v[8 * c + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+                    }
+                }
+                __syncwarp();
+                uint32_t q8[8];
+                const int e = mx_quantize32(v, q8);
+                uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * 32);
+                dst[0] = make_uint4(q8[0], q8[1], q8[2], q8[3]);
+                dst[1] = make_uint4(q8[4], q8[5], q8[6], q8[7]);
+                args.sf[which][mx_scale_offset(ch0 + lane, orow, ox >> 5, args.sf_rows[which],
+                                               args.sf_row_tiles[which], args.kchunks, args.sf_chunks[which])] =
+                    (uint8_t)(e + 127);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_store_3d(which ? &tmB : &tmA, buf, j0 + 32 * q, i, ch0);
+                tma_store_3d(which ? &tmB : &tmA, buf, ox, orow, ch0);
                 tma_store_commit();
             }
         };
 
         // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4,
-        // from the mask row that landed with the tile (zero past column N).
-        auto read_hm = [&](int lt, int j0, float (&hm)[4]) {
+        // from the mask that landed with the tile (zero past N). The first cell of the
+        // warp's run of 32 along its row (PRO_MX_COLS: along its column) is `first`.
+        auto read_hm = [&](int lt, int first, float (&hm)[4]) {
             const uint16_t *mrow = reinterpret_cast<const uint16_t *>(msm + (lt & 3) * MASK_BYTES);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -286,7 +349,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                 if (args.has_mask)
                     hm[c] = 0.5f * bf16_bits_to_float(mrow[jc]);
                 else
-                    hm[c] = j0 + jc < args.N ? 0.5f : 0.f;
+                    hm[c] = first + (jc - 32 * q) < args.N ? 0.5f : 0.f;
             }
         };
 
@@ -316,15 +379,19 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         for (int lt = 0; ok && lt < n_local; ++lt) {
             int i, j0;
             tile_coords(lt, i, j0);
-            const bool live = j0 + 32 * q < args.N;  // this warp's 32 cells start inside the row
+            // The warp's 32 cells go to (x = ox .. ox+31, row orow) of the outputs; they
+            // start inside the layer when `live`.
+            const int ox = kMode == PRO_MX_COLS ? i : j0 + 32 * q;
+            const int orow = kMode == PRO_MX_COLS ? j0 + q : i;
+            const bool live = (kMode == PRO_MX_COLS ? orow : ox) < args.N;
             // a-half of tile lt
             if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
             tc_fence_after();
             float hm[4];  // tile lt landed (its a-half MMAs ran after it was normalised)
-            read_hm(lt, j0, hm);
+            read_hm(lt, ox, hm);
             if (live) {
-                slab(0, 0, hm, i, j0);
-                slab(0, 1, hm, i, j0);
+                slab(0, 0, hm, ox, orow);
+                slab(0, 1, hm, ox, orow);
             }
             tc_fence_before();
             __syncwarp();
@@ -333,8 +400,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             if (!(ok = warp_wait(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 9, lt))) break;
             tc_fence_after();
             if (live) {
-                slab(1, 0, hm, i, j0);
-                slab(1, 1, hm, i, j0);
+                slab(1, 0, hm, ox, orow);
+                slab(1, 1, hm, ox, orow);
             }
             tc_fence_before();
             __syncwarp();
@@ -352,21 +419,39 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
 
 size_t prologue_tc_smem() { return pro::SMEM; }
 
-cudaError_t prologue_tc_setup() {
-    cudaError_t e = cudaFuncSetAttribute(prologue_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pro::SMEM);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(prologue_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pro::SMEM);
+template <bool kVec, int kMode>
+static cudaError_t set_smem() {
+    return cudaFuncSetAttribute(prologue_tc_kernel<kVec, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)pro::SMEM);
 }
 
-cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
+cudaError_t prologue_tc_setup() {
+    cudaError_t e;
+    if ((e = set_smem<false, PRO_BF16>()) != cudaSuccess || (e = set_smem<true, PRO_BF16>()) != cudaSuccess ||
+        (e = set_smem<false, PRO_MX_ROWS>()) != cudaSuccess || (e = set_smem<true, PRO_MX_ROWS>()) != cudaSuccess ||
+        (e = set_smem<false, PRO_MX_COLS>()) != cudaSuccess || (e = set_smem<true, PRO_MX_COLS>()) != cudaSuccess)
+        return e;
+    return cudaSuccess;
+}
+
+template <bool kVec, int kMode>
+static void launch_as(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
+    prologue_tc_kernel<kVec, kMode><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z,
+                                                                          m.mask, m.a, m.b, a);
+}
+
+cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int mode, int grid, cudaStream_t s) {
     const bool vec = a.ln_w || a.ln_b || a.b_a || a.b_ag || a.b_b || a.b_bg;
-    if (vec)
-        prologue_tc_kernel<true><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
-                                                                        m.a, m.b, a);
-    else
-        prologue_tc_kernel<false><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z, m.mask,
-                                                                         m.a, m.b, a);
+    switch (mode) {
+        case PRO_BF16: vec ? launch_as<true, PRO_BF16>(m, a, grid, s) : launch_as<false, PRO_BF16>(m, a, grid, s); break;
+        case PRO_MX_ROWS:
+            vec ? launch_as<true, PRO_MX_ROWS>(m, a, grid, s) : launch_as<false, PRO_MX_ROWS>(m, a, grid, s);
+            break;
+        case PRO_MX_COLS:
+            vec ? launch_as<true, PRO_MX_COLS>(m, a, grid, s) : launch_as<false, PRO_MX_COLS>(m, a, grid, s);
+            break;
+        default: return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 
@@ -378,6 +463,28 @@ __global__ void mask_pad_kernel(const __nv_bfloat16 *__restrict__ mask, __nv_bfl
 
 cudaError_t launch_mask_pad(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int rows, int ld, cudaStream_t s) {
     mask_pad_kernel<<<rows, 128, 0, s>>>(mask, dst, N, ld);
+    return cudaGetLastError();
+}
+
+// 32 x 32 tiles through shared memory: reads along mask rows, writes along dst rows.
+__global__ void mask_transpose_kernel(const __nv_bfloat16 *__restrict__ mask, __nv_bfloat16 *__restrict__ dst, int N,
+                                      int ld) {
+    __shared__ __nv_bfloat16 t[32][33];
+    const int k0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 256 threads: 8 rows per pass
+    for (int r = ty; r < 32; r += 8) {
+        const int k = k0 + r, i = i0 + tx;
+        t[r][tx] = (k < N && i < N) ? mask[(size_t)k * N + i] : __float2bfloat16(0.f);
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int i = i0 + r, k = k0 + tx;
+        if (i < N && k < ld) dst[(size_t)i * ld + k] = t[tx][r];
+    }
+}
+
+cudaError_t launch_mask_transpose(const __nv_bfloat16 *mask, __nv_bfloat16 *dst, int N, int ld, cudaStream_t s) {
+    mask_transpose_kernel<<<dim3((ld + 31) / 32, (N + 31) / 32), 256, 0, s>>>(mask, dst, N, ld);
     return cudaGetLastError();
 }
 

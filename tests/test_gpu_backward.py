@@ -152,3 +152,29 @@ def test_backward_layer_api_matches_abi():
     assert rel_l2(dz.double().cpu().numpy(), ref["z"]) <= 1e-6
     for k, v in grads.items():
         assert rel_l2(v.double().cpu().numpy(), ref[k]) <= 1e-6, k
+
+
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_backward_reusing_the_forward_matches_recompute(direction):
+    """With TRIMUL_BWD_REUSE_FORWARD after a forward call on the same inputs, the
+    backward skips recomputing a, b and x and returns what the recomputing call
+    returns (the recompute is deterministic; only the atomically summed bias and
+    LayerNorm gradients may differ in their last bits), and matches the oracle."""
+    N = 129
+    case = pi.random_case(N, 51, bf16=True, affine=True, mask="random")
+    dout = draw_dout(N, 51)
+    ref = run_backward(case, direction, dout)
+    sd = {key: case[field] for field, key, _ in tm.STATE_KEYS if field in case}
+    cls = tm.TriangleMultiplicationOutgoing if direction == "outgoing" else tm.TriangleMultiplicationIncoming
+    layer = cls(128, 128).load_state_dict(sd).to("cuda", torch.bfloat16)
+    z = torch.from_numpy(case["z"]).to("cuda").to(torch.bfloat16)
+    m = torch.from_numpy(case["mask"]).to("cuda")
+    d = torch.from_numpy(dout).to("cuda").to(torch.bfloat16)
+    layer(z, m)
+    dz, grads = layer.backward(z, d, m, reuse_forward=True)
+    torch.cuda.synchronize()
+    assert torch.equal(dz.double().cpu(), torch.from_numpy(ref["z"]))
+    for k, v in grads.items():
+        assert rel_l2(v.double().cpu().numpy(), ref[k]) <= 1e-6, k
+    compare({**{k: v.double().cpu().numpy() for k, v in grads.items()}, "z": dz.double().cpu().numpy()},
+            ob.trimul_backward(case, direction, dout.astype(np.float64)), "reuse")

@@ -12,8 +12,11 @@ Bars:
   * contraction stage: rel-L2 <= 1e-2 and max-abs <= 4 * 2^-9 * max|ref| (the
     bf16 stage bars). The GPU multiplies the same E4M3 elements and scales
     exactly (8-bit significands), accumulates in fp32 and rounds x to bf16 once.
+  * fused prologue (trimul_forward_mxfp8 quantizes inside the prologue): codes
+    and scales bit-exact against the oracle's quantization of the bf16 a, b that
+    the plain prologue stores for the same inputs.
   * whole layer: the oracle contracts, in MXFP8, the very bf16 a and b the GPU's
-    prologue stored (read back from the workspace), so both sides take the same
+    prologue computes (the plain prologue's, read back from the workspace), so both sides take the same
     quantization decisions, then finishes the layer; bars rel-L2 <= 1.5e-2,
     max-abs <= 5e-2 (the bf16 layer bars). (The oracle's own a, b rounded to bf16
     differ from the GPU's by one bf16 ulp in some elements, which flips E4M3
@@ -99,15 +102,10 @@ def _load(dc, a, b):
     return vx
 
 
-@pytest.mark.parametrize("N", [33, 200, 385])
-@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
-def test_mx_quantizer_bit_exact(N, direction):
-    a, b = _operands(N, N)
-    dc = MxCase(pi.random_case(N, 1, bf16=True, mask="ones"))
-    _load(dc, a, b)
-    tm.trimul_contract_mxfp8(dc.p, DIRS[direction])
-    torch.cuda.synchronize()
-    assert tm.trimul_device_status(dc.p)[0] == 0
+def _assert_codes_match(dc, a, b, direction):
+    """The E4M3 codes and scale bytes in dc's MX sections equal the oracle's
+    quantization of the bf16 a, b (cell-major [N][N][128]) along the contracted index."""
+    N = dc.N
     qa, qb, sa, sb, ldq = dc.mx_views()
     ws = dc.ws.cpu().numpy()
     kc, ti, tj = (N + 127) // 128, (N + 255) // 256, (N + 191) // 192
@@ -126,6 +124,38 @@ def test_mx_quantizer_bit_exact(N, direction):
         off = _scale_offset(c_i, r_i, k_i, rpt, rtiles, kc, cpt)
         got_e = ws[soff + off].astype(np.int64) - 127
         assert np.array_equal(got_e, e_op.astype(np.int64)), "scale exponents differ"
+
+
+@pytest.mark.parametrize("N", [33, 200, 385])
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_mx_quantizer_bit_exact(N, direction):
+    a, b = _operands(N, N)
+    dc = MxCase(pi.random_case(N, 1, bf16=True, mask="ones"))
+    _load(dc, a, b)
+    tm.trimul_contract_mxfp8(dc.p, DIRS[direction])
+    torch.cuda.synchronize()
+    assert tm.trimul_device_status(dc.p)[0] == 0
+    _assert_codes_match(dc, a, b, direction)
+
+
+@pytest.mark.parametrize("N", [33, 200, 385])
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+@pytest.mark.parametrize("mask", ["random", None])
+def test_mx_fused_prologue_bit_exact(N, direction, mask):
+    """trimul_forward_mxfp8 quantizes inside the prologue (outgoing on row tiles,
+    incoming on 32 x 4 column tiles). Its codes and scales must equal the oracle's
+    quantization of the bf16 a, b the plain prologue stores for the same inputs (the
+    fused kernel rounds to the same bf16 values before quantizing). Ragged N: partial
+    blocks, partial column groups and partial 128-wide K chunks."""
+    case = pi.random_case(N, 40 + N, bf16=True, affine=True, mask=mask or "ones")
+    dc = MxCase(case, with_mask=mask is not None)
+    tm.trimul_prologue(dc.z, dc.mask, dc.p)
+    torch.cuda.synchronize()
+    a, b = _gpu_ab(dc)
+    tm.trimul_forward_mxfp8(dc.z, dc.mask, dc.p, DIRS[direction], dc.out)
+    torch.cuda.synchronize()
+    assert tm.trimul_device_status(dc.p)[0] == 0
+    _assert_codes_match(dc, a, b, direction)
 
 
 @pytest.mark.parametrize("N", [64, 129, 191, 192, 193, 256, 385, 513, 768])
@@ -159,16 +189,24 @@ def _gpu_ab(dc):
     return DeviceCase.to_cell_major(va, dc.N), DeviceCase.to_cell_major(vb, dc.N)
 
 
+def _prologue_ab(dc):
+    """The bf16 a and b of the plain prologue on dc's inputs: the values the fused
+    MXFP8 prologue rounds to before it quantizes (it stores no bf16 copy)."""
+    tm.trimul_prologue(dc.z, dc.mask, dc.p)
+    torch.cuda.synchronize()
+    return _gpu_ab(dc)
+
+
 @pytest.mark.parametrize("N,seed", [(100, 11), (300, 12)])
 @pytest.mark.parametrize("direction", ["outgoing", "incoming"])
 def test_mx_layer(N, seed, direction):
     case = pi.random_case(N, seed, bf16=True, affine=True, mask="random")
     dc = MxCase(case)
+    a, b = _prologue_ab(dc)
     tm.trimul_forward_mxfp8(dc.z, dc.mask, dc.p, DIRS[direction], dc.out)
     torch.cuda.synchronize()
     assert tm.trimul_device_status(dc.p)[0] == 0
     got = dc.out.double().cpu().numpy()
-    a, b = _gpu_ab(dc)
     ref = oracle.finish(case, mx_contract(a, b, direction))
     assert rel_l2(got, ref) <= 1.5e-2 and max_abs(got, ref) <= 5e-2
     # The prologue's a, b themselves against the oracle (the bf16 stage bar).
@@ -185,12 +223,12 @@ def test_mx_workload3_sampled():
     case = pi.make_workload(w)
     dc = MxCase(case)
     I = pi.sample_grid(w.N, w.seed, n_random=8)
+    a, b = _prologue_ab(dc)
     for direction in w.directions:
         tm.trimul_forward_mxfp8(dc.z, dc.mask, dc.p, DIRS[direction], dc.out)
         torch.cuda.synchronize()
         assert tm.trimul_device_status(dc.p)[0] == 0
         got = dc.out.double().cpu().numpy()[np.ix_(I, I)]
-        a, b = _gpu_ab(dc)
         x = mx_contract_grid(a, b, direction, I)
         sub = {k: v for k, v in case.items() if k not in ("z", "mask", "m")}
         sub["z"] = case["z"][np.ix_(I, I)]
