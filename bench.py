@@ -426,10 +426,17 @@ def mxfp8_timings(tm, pi, torch, dev, stream, peaks, wids=(3, 4, 5), warmup=3, r
         for d in w.directions:
             t_mx = timed(lambda: tm.trimul_contract_mxfp8(p, code[d], stream))
             t_bf = timed(lambda: tm.trimul_contract(p, code[d], stream))
+            # The MMA kernel alone, on the operands the quantizer just wrote.
+            t_mma = timed(lambda: tm.trimul_mma_mxfp8(p, stream))
+            t_pro_mx = timed(lambda: tm.trimul_prologue_mxfp8(z, mask, p, code[d], stream))
+            t_pro = timed(lambda: tm.trimul_prologue(z, mask, p, stream))
             entry[d] = {"mxfp8_us": round(t_mx, 1), "bf16_us": round(t_bf, 1),
                         "mxfp8_tflops": round(flop / (t_mx * 1e-6) / 1e12, 1),
                         "bf16_tflops": round(flop / (t_bf * 1e-6) / 1e12, 1),
-                        "speedup": round(t_bf / t_mx, 3)}
+                        "speedup": round(t_bf / t_mx, 3),
+                        "mma_us": round(t_mma, 1), "mma_tflops": round(flop / (t_mma * 1e-6) / 1e12, 1),
+                        "mma_speedup": round(t_bf / t_mma, 3),
+                        "prologue_mxfp8_us": round(t_pro_mx, 1), "prologue_bf16_us": round(t_pro, 1)}
         out = torch.empty_like(z)
         for d in w.directions:
             t = timed(lambda: tm.trimul_forward_mxfp8(z, mask, p, code[d], out, stream))
@@ -460,7 +467,8 @@ def run_mxfp8_only(args):
     tmbuild.build()
     tm.lib()
     peaks, _ = load_peaks()
-    res = mxfp8_timings(tm, pi, torch, dev, torch.cuda.current_stream(dev), peaks, warmup=args.warmup,
+    wids = tuple(int(x) for x in args.mx_workloads.split(","))
+    res = mxfp8_timings(tm, pi, torch, dev, torch.cuda.current_stream(dev), peaks, wids=wids, warmup=args.warmup,
                         reps=args.steps)
     print(json.dumps({"mxfp8": res}), flush=True)
 
@@ -840,6 +848,8 @@ def main(argv=None):
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8 secondary timing")
     ap.add_argument("--mxfp8-only", action="store_true",
                     help="time only the MXFP8 contraction beside the bf16 one and print that")
+    ap.add_argument("--mx-workloads", default="3,4,5",
+                    help="workload ids --mxfp8-only runs (3: N = 768, 4: N = 2048, 5: N = 3605)")
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget", type=float, default=120.0)
     args = ap.parse_args(argv)

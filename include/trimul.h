@@ -204,7 +204,11 @@ int trimul_epilogue_rows(const void *z_rows, const void *x_rows, const trimul_pa
  * (round to nearest even, saturated at +-448) sharing an E8M0 scale
  * 2^(floor(log2 max|v|) - 8); the contraction then runs on tcgen05
  * block-scaled MMAs (kind::mxf8f6f4) with fp32 accumulation and writes x in
- * bf16. The prologue and epilogue are those of trimul_forward.
+ * bf16. The epilogue is that of trimul_forward. trimul_forward_mxfp8 runs the
+ * prologue in a quantising form (trimul_prologue_mxfp8): it rounds a and b to
+ * bf16 exactly as trimul_prologue stores them and writes their E4M3 codes and
+ * scales straight into the workspace, so no bf16 copy of a and b is stored or
+ * read back.
  *
  * BF16 only (TRIMUL_ERR_UNSUPPORTED otherwise). p->workspace must hold
  * trimul_workspace_size_mxfp8(N, c_z, c_h) bytes: the bf16 sections of
@@ -215,7 +219,19 @@ size_t trimul_workspace_size_mxfp8(int N, int c_z, int c_h);
 int trimul_forward_mxfp8(const void *z, const void *mask, const trimul_params *p, int direction,
                          void *out, trimul_stream_t stream);
 
-/* The MXFP8 contraction stage alone: a, b (bf16, in the workspace) -> x. */
+/* Stage calls of the MXFP8 layer (trimul_forward_mxfp8 = trimul_prologue_mxfp8,
+ * trimul_mma_mxfp8, trimul_epilogue on one stream):
+ *   trimul_prologue_mxfp8  z, mask -> the E4M3 operands and scales of
+ *                          `direction`'s contraction (the bf16 a, b sections
+ *                          are left untouched);
+ *   trimul_mma_mxfp8       the block-scaled contraction of the operands in the
+ *                          workspace -> x (bf16); the operands already encode
+ *                          the direction;
+ *   trimul_contract_mxfp8  a, b (bf16, in the workspace) -> x: quantises them
+ *                          (a separate pass) and runs trimul_mma_mxfp8. */
+int trimul_prologue_mxfp8(const void *z, const void *mask, const trimul_params *p, int direction,
+                          trimul_stream_t stream);
+int trimul_mma_mxfp8(const trimul_params *p, trimul_stream_t stream);
 int trimul_contract_mxfp8(const trimul_params *p, int direction, trimul_stream_t stream);
 
 /* Device pointers of the quantised operands inside p->workspace (host-only):

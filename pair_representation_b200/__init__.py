@@ -41,6 +41,7 @@ EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forwa
            "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
            "trimul_backward", "trimul_backward_workspace_size",
            "trimul_workspace_size_mxfp8", "trimul_forward_mxfp8", "trimul_contract_mxfp8", "trimul_mxfp8_views",
+           "trimul_prologue_mxfp8", "trimul_mma_mxfp8",
            "trimul_shard_workspace_size", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows",
            "atomattn_forward", "atomattn_workspace_size", "atomattn_device_status")
 
@@ -131,6 +132,8 @@ def lib():
         L.trimul_workspace_size_mxfp8.restype = S
         L.trimul_forward_mxfp8.argtypes = [P, P, PP, I, P, P]
         L.trimul_contract_mxfp8.argtypes = [PP, I, P]
+        L.trimul_prologue_mxfp8.argtypes = [P, P, PP, I, P]
+        L.trimul_mma_mxfp8.argtypes = [PP, P]
         L.trimul_mxfp8_views.argtypes = [PP] + [ctypes.POINTER(P)] * 4 + [ctypes.POINTER(S)]
         L.trimul_shard_workspace_size.argtypes = [I, I]
         L.trimul_shard_workspace_size.restype = S
@@ -145,7 +148,7 @@ def lib():
         for f in ("trimul_forward", "trimul_forward_noalloc", "trimul_prologue", "trimul_contract", "trimul_epilogue",
                   "trimul_workspace_views", "trimul_device_status", "trimul_version", "trimul_backward",
                   "atomattn_forward", "atomattn_device_status", "trimul_forward_mxfp8", "trimul_contract_mxfp8",
-                  "trimul_mxfp8_views", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows"):
+                  "trimul_mxfp8_views", "trimul_prologue_mxfp8", "trimul_mma_mxfp8", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -255,6 +258,22 @@ def trimul_contract_mxfp8(params: TrimulParams, direction: int, stream=None, che
     rc = lib().trimul_contract_mxfp8(ctypes.byref(params), direction, _stream(stream))
     if check:
         _check(rc, "trimul_contract_mxfp8")
+    return rc
+
+
+def trimul_prologue_mxfp8(z, mask, params: TrimulParams, direction: int, stream=None, check=True) -> int:
+    """The quantising prologue: z, mask -> E4M3 operands and scales of `direction`'s contraction."""
+    rc = lib().trimul_prologue_mxfp8(_ptr(z), _ptr(mask), ctypes.byref(params), direction, _stream(stream))
+    if check:
+        _check(rc, "trimul_prologue_mxfp8")
+    return rc
+
+
+def trimul_mma_mxfp8(params: TrimulParams, stream=None, check=True) -> int:
+    """The block-scaled contraction of the MXFP8 operands in the workspace -> x."""
+    rc = lib().trimul_mma_mxfp8(ctypes.byref(params), _stream(stream))
+    if check:
+        _check(rc, "trimul_mma_mxfp8")
     return rc
 
 

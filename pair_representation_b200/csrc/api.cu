@@ -350,7 +350,7 @@ int cuda_rc(cudaError_t e, const char *what) {
 // or null, a and b written as [128][rows][ld]. mask_scratch holds rows * ld bf16
 // for a mask whose rows lack a 16-byte pitch.
 // The launch fields every prologue mode shares (the tiling is set by the caller).
-PrologueArgs prologue_args(const trimul_params *p, bool has_mask, const KernelCtl &ctl) {
+PrologueArgs prologue_args(const trimul_params *p, bool has_mask, const KernelCtl &ctl, bool clear) {
     PrologueArgs a;
     memset(&a, 0, sizeof a);
     a.N = p->N;
@@ -362,6 +362,7 @@ PrologueArgs prologue_args(const trimul_params *p, bool has_mask, const KernelCt
     a.b_ag = static_cast<const __nv_bfloat16 *>(p->b_ag);
     a.b_b = static_cast<const __nv_bfloat16 *>(p->b_b);
     a.b_bg = static_cast<const __nv_bfloat16 *>(p->b_bg);
+    a.clear_status = clear ? 1 : 0;
     a.ctl = ctl;
     return a;
 }
@@ -373,8 +374,12 @@ int map_weights(PrologueMaps *m, const trimul_params *p) {
     return TRIMUL_OK;
 }
 
+int clear_status(const trimul_params *p, cudaStream_t s);
+
+// clear: this launch starts the call, so the kernel zeroes the status word (no separate
+// memset in the stream).
 int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int rows, void *a_out, void *b_out,
-                    void *mask_scratch, const KernelCtl &ctl, const DevState &d, cudaStream_t s) {
+                    void *mask_scratch, const KernelCtl &ctl, const DevState &d, cudaStream_t s, bool clear) {
     const size_t ld = ld_of(p->N);
     PrologueMaps m;
     if (int rc = map_weights(&m, p)) return rc;
@@ -398,23 +403,26 @@ int run_prologue_tc(const void *z, const void *mask, const trimul_params *p, int
     // Each gating warp stores 32 cells x 32 channels (64-byte rows, 64-byte swizzle).
     if (int rc = map_cm(&m.a, a_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
     if (int rc = map_cm(&m.b, b_out, p->N, ld, 32, 1, 32, CU_TENSOR_MAP_SWIZZLE_64B, rows)) return rc;
-    PrologueArgs a = prologue_args(p, mask != nullptr, ctl);
+    PrologueArgs a = prologue_args(p, mask != nullptr, ctl, clear);
     a.jt_tiles = (p->N + 127) / 128;
     a.total_tiles = rows * a.jt_tiles;
     const int grid = a.total_tiles < d.sms ? a.total_tiles : d.sms;
     return cuda_rc(launch_prologue_tc(m, a, PRO_BF16, grid, s), "prologue_tc launch");
 }
 
-int run_prologue(const void *z, const void *mask, const trimul_params *p, const DevState &d, cudaStream_t s) {
+int run_prologue(const void *z, const void *mask, const trimul_params *p, const DevState &d, cudaStream_t s,
+                 bool clear) {
     const Views v = views_of(p);
     if (p->dtype == TRIMUL_DTYPE_F32) {
+        if (clear)
+            if (int rc = clear_status(p, s)) return rc;
         const long tiles = (long)p->N * ((p->N + 31) / 32);
         const int grid = (int)(tiles < (long)d.sms * 8 ? tiles : (long)d.sms * 8);
         return cuda_rc(launch_prologue_f32(static_cast<const float *>(z), f32_layer(p, mask, v), grid, s),
                        "prologue_f32 launch");
     }
     // A re-pitched mask goes to plane 0 of x, which the contraction overwrites later.
-    return run_prologue_tc(z, mask, p, p->N, v.a, v.b, v.x, ctl_of(p, v), d, s);
+    return run_prologue_tc(z, mask, p, p->N, v.a, v.b, v.x, ctl_of(p, v), d, s, clear);
 }
 
 // A matrix operand of the pair kernel: element (row, col) of batch b at
@@ -641,7 +649,7 @@ int run_contract_mx_mma(const trimul_params *p, const DevState &d, cudaStream_t 
 // and scales) straight into the MX sections of the workspace: outgoing on row
 // tiles, incoming on 32 x 4 column tiles (the contracted index of a_ki is the row).
 int run_prologue_mx(const void *z, const void *mask, const trimul_params *p, int direction, const DevState &d,
-                    cudaStream_t s) {
+                    cudaStream_t s, bool clear) {
     const Views v = views_of(p);
     const int N = p->N;
     const MxLayout L = mx_layout(N);
@@ -697,7 +705,7 @@ int run_prologue_mx(const void *z, const void *mask, const trimul_params *p, int
     if (int rc = encode(&m.b, 3, base + L.bq, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_DATA_TYPE_UINT8))
         return rc;
-    PrologueArgs a = prologue_args(p, mask != nullptr, ctl_of(p, v));
+    PrologueArgs a = prologue_args(p, mask != nullptr, ctl_of(p, v), clear);
     if (cols) {
         a.jt_tiles = (N + 3) / 4;
         a.total_tiles = ((N + 31) / 32) * a.jt_tiles;
@@ -828,7 +836,7 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     // states that the last forward call left them there.
     if ((rc = clear_status(p, s))) return rc;
     if (!(gr->flags & TRIMUL_BWD_REUSE_FORWARD) &&
-        ((rc = run_prologue(z, mask, p, d, s)) || (rc = run_contract(p, direction, d, s))))
+        ((rc = run_prologue(z, mask, p, d, s, false)) || (rc = run_contract(p, direction, d, s))))
         return rc;
     if ((rc = cuda_rc(cudaMemsetAsync(sums, 0, (size_t)kSumCount * C * 4, s), "backward sums clear"))) return rc;
     const void *wk[kProjBlocks] = {p->w_g, p->w_a, p->w_ag, p->w_b, p->w_bg};
@@ -1040,8 +1048,7 @@ int trimul_prologue(const void *z, const void *mask, const trimul_params *p, tri
         (rc = check_device_ptr(mask, "mask")))
         return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = clear_status(p, s))) return rc;
-    return run_prologue(z, mask, p, *d, s);
+    return run_prologue(z, mask, p, *d, s, true);
 }
 
 int trimul_contract(const trimul_params *p, int direction, trimul_stream_t stream) {
@@ -1075,8 +1082,7 @@ int trimul_forward(const void *z, const void *mask, const trimul_params *p, int 
         (rc = check_device_ptr(mask, "mask")) || (rc = check_device_ptr(out, "out")))
         return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = clear_status(p, s))) return rc;
-    if ((rc = run_prologue(z, mask, p, *d, s))) return rc;
+    if ((rc = run_prologue(z, mask, p, *d, s, true))) return rc;
     if ((rc = run_contract(p, direction, *d, s))) return rc;
     return run_epilogue(z, p, out, *d, s);
 }
@@ -1107,10 +1113,32 @@ int trimul_forward_mxfp8(const void *z, const void *mask, const trimul_params *p
         (rc = check_device_ptr(mask, "mask")) || (rc = check_device_ptr(out, "out")))
         return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = clear_status(p, s))) return rc;
-    if ((rc = run_prologue_mx(z, mask, p, direction, *d, s))) return rc;
+    if ((rc = run_prologue_mx(z, mask, p, direction, *d, s, true))) return rc;
     if ((rc = run_contract_mx_mma(p, *d, s))) return rc;
     return run_epilogue(z, p, out, *d, s);
+}
+
+int trimul_prologue_mxfp8(const void *z, const void *mask, const trimul_params *p, int direction,
+                          trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_direction(direction)) || (rc = check_mx(p)) || (rc = check_z(p, z)) ||
+        (rc = check_mask(p, mask)))
+        return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    if ((rc = check_weights_on_device(p)) || (rc = check_device_ptr(z, "z")) ||
+        (rc = check_device_ptr(mask, "mask")) || (rc = check_device_ptr(p->workspace, "workspace")))
+        return rc;
+    return run_prologue_mx(z, mask, p, direction, *d, reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int trimul_mma_mxfp8(const trimul_params *p, trimul_stream_t stream) {
+    int rc;
+    if ((rc = check_params(p)) || (rc = check_mx(p))) return rc;
+    const DevState *d = nullptr;
+    if ((rc = device_state(&d, true))) return rc;
+    if ((rc = check_device_ptr(p->workspace, "workspace"))) return rc;
+    return run_contract_mx_mma(p, *d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int trimul_mxfp8_views(const trimul_params *p, void **aq, void **bq, void **sa, void **sb, size_t *ldq) {
@@ -1151,10 +1179,9 @@ int trimul_prologue_rows(const void *z_rows, const void *mask_rows, const trimul
         if ((rc = check_device_ptr(v, "shard buffer"))) return rc;
     if ((rc = check_weights_on_device(p))) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = clear_status(p, s))) return rc;
     const Views v = views_of(p);
     return run_prologue_tc(z_rows, mask_rows, p, rows, a, b, static_cast<uint8_t *>(p->workspace) + kHeader,
-                           ctl_of(p, v), *d, s);
+                           ctl_of(p, v), *d, s, true);
 }
 
 int trimul_contract_channels(const trimul_params *p, int direction, int channels, const void *a, const void *b,

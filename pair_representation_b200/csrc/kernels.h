@@ -38,6 +38,10 @@ struct PrologueArgs {
     uint8_t *sf[2];
     int sf_rows[2], sf_row_tiles[2], sf_chunks[2];
     int kchunks;
+    // Nonzero: the call starts here, and CTA 0 zeroes the status word before anything else
+    // (every recorded failure comes from a bounded wait that ran for ctl.timeout_ns, long
+    // after all CTAs of this one-wave grid have started).
+    int clear_status;
     KernelCtl ctl;
 };
 

@@ -32,6 +32,36 @@ __device__ __forceinline__ int mx_quantize32(const float (&v)[32], uint32_t (&q8
     return e;
 }
 
+// The same for 32 bf16 values packed in pairs (w[t] holds values 2t, 2t + 1, the
+// lower index in the low half). Non-negative bf16 bit patterns order like their
+// values, so max|v| is an unsigned 16-bit max over the patterns with the sign
+// cleared, and e comes from its exponent field; the scaling is the fp32 one.
+__device__ __forceinline__ int mx_quantize32_bf16(const uint32_t (&w)[16], uint32_t (&q8)[8]) {
+    uint32_t m[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) m[t] = w[t] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int h = 8; h >= 1; h >>= 1)  // pairwise tree: 4 dependent steps instead of 15
+#pragma unroll
+        for (int t = 0; t < h; ++t) asm("max.u16x2 %0, %0, %1;" : "+r"(m[t]) : "r"(m[t + h]));
+    const uint32_t amax = (m[0] & 0xFFFFu) > (m[0] >> 16) ? (m[0] & 0xFFFFu) : (m[0] >> 16);
+    int e = (int)(amax >> 7) - 127 - 8;
+    if (amax == 0 || e < -127) e = -127;
+    if (e > 127) e = 127;
+    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+    const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        const uint32_t u0 = w[2 * t], u1 = w[2 * t + 1];
+        const float2 x0 = __fmul2_rn(make_float2(__uint_as_float(u0 << 16), __uint_as_float(u0 & 0xFFFF0000u)), inv2);
+        const float2 x1 = __fmul2_rn(make_float2(__uint_as_float(u1 << 16), __uint_as_float(u1 & 0xFFFF0000u)), inv2);
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(x0, __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(x1, __NV_SATFINITE, __NV_E4M3);
+        q8[t] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    return e;
+}
+
 // Byte offset of the scale of (operand row r, K block kb) of channel c in a scale
 // array laid out per row tile of the contraction (rows_per_tile rows in
 // chunks_per_tile chunks of 128 rows) and per 128-wide K chunk: within a

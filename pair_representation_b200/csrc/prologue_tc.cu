@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                        const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const PrologueArgs args) {
     using namespace pro;
+    if (args.clear_status && blockIdx.x == 0 && threadIdx.x == 0) *args.ctl.status = DeviceStatus{0, 0, 0, 0};
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *wsm = smem;
@@ -252,26 +253,107 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         const int q = warp & 3, sub = warp >> 2;  // TMEM lane quadrant (cells 32q..32q+31), channel half
         uint8_t *stw = stsm + warp * ST_PER_WARP * ST_BYTES;
         int st_round = 0;
+        // MXFP8 modes: bytes between the scale arrays of consecutive channels (the scale
+        // offset is linear in the channel; the arrays stay far below 4 GB).
+        auto sf_cstride = [&](int o) {
+            return (uint32_t)args.sf_row_tiles[o] * (uint32_t)args.kchunks * (uint32_t)args.sf_chunks[o] * 512u;
+        };
+
+        // One gated slab waits in its staging buffer while the next slab is gated: the
+        // next slab's tensor-memory loads, its gating and (MXFP8 modes) the pending
+        // slab's quantisation form one straight-line stretch the compiler can
+        // interleave; then the pending slab is stored.
+        struct Pending {
+            uint8_t *buf;
+            int which, ch0, ox, orow;
+            uint32_t sfo;  // scale offset of channel 0 (MXFP8 modes)
+            bool on;
+        } pend;
+        pend.buf = stw;
+        pend.on = false;
+        // Lane l's channel ch0 + l of the pending slab: its 32 bf16 values are buffer row l
+        // (logical 16-byte chunk c at c ^ ((l >> 1) & 3)).
+        auto pending_row = [&](uint32_t (&w)[16]) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(pend.buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4));
+                w[4 * c] = u.x;
+                w[4 * c + 1] = u.y;
+                w[4 * c + 2] = u.z;
+                w[4 * c + 3] = u.w;
+            }
+        };
+        // Store the pending slab; MXFP8 modes first write the quantised codes back in place
+        // (lane l's 32 codes at bytes 32 l .., a dense [32 ch][32 B] box) and the scale byte.
+        // Every lane must have read its row before.
+        auto store_pending = [&](const uint32_t (&q8)[8], int e) {
+            if (kMode != PRO_BF16) {
+                __syncwarp();
+                uint4 *dst = reinterpret_cast<uint4 *>(pend.buf + lane * 32);
+                dst[0] = make_uint4(q8[0], q8[1], q8[2], q8[3]);
+                dst[1] = make_uint4(q8[4], q8[5], q8[6], q8[7]);
+                args.sf[pend.which][pend.sfo + (uint32_t)(pend.ch0 + lane) * sf_cstride(pend.which)] = (uint8_t)(e + 127);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(pend.which ? &tmB : &tmA, pend.buf, pend.ox, pend.orow, pend.ch0);
+                tma_store_commit();
+            }
+            pend.on = false;
+        };
+        auto flush = [&]() {
+            if (!pend.on) return;
+            uint32_t q8[8];
+            int e = 0;
+            if (kMode != PRO_BF16) {
+                uint32_t w[16];
+                __syncwarp();
+                pending_row(w);
+                e = mx_quantize32_bf16(w, q8);
+            }
+            store_pending(q8, e);
+        };
+
         // Gate 32 cells x 32 channels of a (which = 0) or b (which = 1), channels hh*64 + sub*32 ..,
-        // and store them channel-major at (x = ox .. ox+31, row orow).
-        auto slab = [&](int which, int hh, const float (&hm)[4], int ox, int orow) {
+        // for the outputs at (x = ox .. ox+31, row orow). `release` (if set) is signalled
+        // right after the slab's tensor-memory reads, so the next tile's MMAs into these
+        // columns overlap the gating and the stores.
+        auto slab = [&](int which, int hh, const float (&hm)[4], int ox, int orow, uint32_t sfo, uint64_t *release) {
             const int ch0 = hh * 64 + sub * 32;
+            uint32_t V[2][16], G[2][16];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t ta = tmem_base + ((uint32_t)(q * 32 + 16 * hf) << 16) + (uint32_t)(which * 256 + ch0);
+                tmem_ld16x256_x4(ta, V[hf]);
+                tmem_ld16x256_x4(ta + 128, G[hf]);
+            }
+            // The pending slab's row is read (and quantised below) whether or not a slab is
+            // pending: pend.buf always points into this warp's staging buffers.
+            uint32_t w[16];
+            if (kMode != PRO_BF16) {
+                __syncwarp();
+                pending_row(w);
+            }
+            tmem_ld_wait();
+            if (release) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(release);
+            }
             uint32_t P[16];  // packed bf16 pairs: [hf][k][e] -> P[hf * 8 + k * 2 + e]
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                uint32_t V[16], G[16];
-                const uint32_t ta = tmem_base + ((uint32_t)(q * 32 + 16 * hf) << 16) + (uint32_t)(which * 256 + ch0);
-                tmem_ld16x256_x4(ta, V);
-                tmem_ld16x256_x4(ta + 128, G);
-                tmem_ld_wait();
                 const __nv_bfloat16 *bv = which ? args.b_b : args.b_a;
                 const __nv_bfloat16 *bg = which ? args.b_bg : args.b_ag;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        float2 g = make_float2(__uint_as_float(G[4 * k + 2 * e]), __uint_as_float(G[4 * k + 2 * e + 1]));
-                        float2 v = make_float2(__uint_as_float(V[4 * k + 2 * e]), __uint_as_float(V[4 * k + 2 * e + 1]));
+                        float2 g = make_float2(__uint_as_float(G[hf][4 * k + 2 * e]),
+                                               __uint_as_float(G[hf][4 * k + 2 * e + 1]));
+                        float2 v = make_float2(__uint_as_float(V[hf][4 * k + 2 * e]),
+                                               __uint_as_float(V[hf][4 * k + 2 * e + 1]));
                         // g holds (W_g zh) / 2: the gate weights were halved in shared memory.
                         if (kVec) {
                             const int c = ch0 + 8 * k + 2 * (lane & 3);
@@ -286,6 +368,10 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                     }
                 }
             }
+            uint32_t q8[8];
+            int qe = 0;
+            if (kMode != PRO_BF16) qe = mx_quantize32_bf16(w, q8);
+            if (pend.on) store_pending(q8, qe);
             uint8_t *buf = stw + (st_round & 1) * ST_BYTES;
             ++st_round;
             if (lane == 0) tma_store_wait_read<1>();  // the store that last used `buf` has read it
@@ -304,38 +390,13 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                     stmatrix_x4_trans(addr, P[hf * 8 + kp * 2 + 0], P[hf * 8 + kp * 2 + 1], P[hf * 8 + kp * 2 + 2],
                                       P[hf * 8 + kp * 2 + 3]);
                 }
-            if (kMode != PRO_BF16) {
-                // Lane l quantises channel ch0 + l: its 32 bf16 values are buffer row l
-                // (logical 16-byte chunk c at c ^ ((l >> 1) & 3)); its 32 codes go back to
-                // bytes 32 l .. 32 l + 31, a dense [32 ch][32 B] box for the TMA store.
-                __syncwarp();
-                float v[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4));
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        v[8 * c + 2 * t] = __uint_as_float(w[t] << 16);
-                        v[8 * c + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
-                    }
-                }
-                __syncwarp();
-                uint32_t q8[8];
-                const int e = mx_quantize32(v, q8);
-                uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * 32);
-                dst[0] = make_uint4(q8[0], q8[1], q8[2], q8[3]);
-                dst[1] = make_uint4(q8[4], q8[5], q8[6], q8[7]);
-                args.sf[which][mx_scale_offset(ch0 + lane, orow, ox >> 5, args.sf_rows[which],
-                                               args.sf_row_tiles[which], args.kchunks, args.sf_chunks[which])] =
-                    (uint8_t)(e + 127);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_3d(which ? &tmB : &tmA, buf, ox, orow, ch0);
-                tma_store_commit();
-            }
+            pend.buf = buf;
+            pend.which = which;
+            pend.ch0 = ch0;
+            pend.ox = ox;
+            pend.orow = orow;
+            pend.sfo = sfo;
+            pend.on = true;
         };
 
         // hm = mask / 2 for the four cells this thread gates in tile lt: 32q + 16hf + 8e + lane/4,
@@ -384,29 +445,40 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             const int ox = kMode == PRO_MX_COLS ? i : j0 + 32 * q;
             const int orow = kMode == PRO_MX_COLS ? j0 + q : i;
             const bool live = (kMode == PRO_MX_COLS ? orow : ox) < args.N;
+            uint32_t sfo[2] = {0, 0};
+            if (kMode != PRO_BF16 && live) {
+#pragma unroll
+                for (int o = 0; o < 2; ++o)
+                    sfo[o] = (uint32_t)mx_scale_offset(0, orow, ox >> 5, args.sf_rows[o], args.sf_row_tiles[o],
+                                                       args.kchunks, args.sf_chunks[o]);
+            }
+            if (!live) flush();
             // a-half of tile lt
             if (!(ok = warp_wait(mma_a, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 7, lt))) break;
             tc_fence_after();
             float hm[4];  // tile lt landed (its a-half MMAs ran after it was normalised)
             read_hm(lt, ox, hm);
             if (live) {
-                slab(0, 0, hm, ox, orow);
-                slab(0, 1, hm, ox, orow);
+                slab(0, 0, hm, ox, orow, sfo[0], nullptr);
+                slab(0, 1, hm, ox, orow, sfo[0], a_free);
+            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(a_free);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(a_free);
             // b-half of tile lt
             if (!(ok = warp_wait(mma_b, (uint32_t)lt & 1u, abort_flag, ctl, SITE_PRO | 9, lt))) break;
             tc_fence_after();
             if (live) {
-                slab(1, 0, hm, ox, orow);
-                slab(1, 1, hm, ox, orow);
+                slab(1, 0, hm, ox, orow, sfo[1], nullptr);
+                slab(1, 1, hm, ox, orow, sfo[1], b_free);
+            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_free);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_free);
         }
+        if (ok) flush();
         if (!ok && lane == 0) *abort_flag = 1;
         if (lane == 0) tma_store_wait_all<0>();
     }

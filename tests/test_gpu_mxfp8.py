@@ -244,3 +244,22 @@ def test_mx_rejects_small_workspace_and_fp32():
     f = DeviceCase(pi.random_case(64, 3, mask="ones"), "f32")
     rc = tm.trimul_forward_mxfp8(f.z, f.mask, f.p, tm.OUTGOING, f.out, check=False)
     assert rc == tm.ERR["TRIMUL_ERR_UNSUPPORTED"]
+
+
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_mx_stage_calls_compose(direction):
+    """trimul_prologue_mxfp8, trimul_mma_mxfp8 and trimul_epilogue on one stream give
+    bit for bit what trimul_forward_mxfp8 gives."""
+    N = 257
+    case = pi.random_case(N, 77, bf16=True, affine=True, mask="random")
+    dc = MxCase(case)
+    tm.trimul_forward_mxfp8(dc.z, dc.mask, dc.p, DIRS[direction], dc.out)
+    torch.cuda.synchronize()
+    whole = dc.out.clone()
+    dc.out.fill_(float("nan"))
+    tm.trimul_prologue_mxfp8(dc.z, dc.mask, dc.p, DIRS[direction])
+    tm.trimul_mma_mxfp8(dc.p)
+    tm.trimul_epilogue(dc.z, dc.p, dc.out)
+    torch.cuda.synchronize()
+    assert tm.trimul_device_status(dc.p)[0] == 0
+    assert torch.equal(whole, dc.out)
