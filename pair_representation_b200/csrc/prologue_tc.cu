@@ -78,7 +78,6 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                        const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const PrologueArgs args) {
     using namespace pro;
-    if (args.clear_status && blockIdx.x == 0 && threadIdx.x == 0) *args.ctl.status = DeviceStatus{0, 0, 0, 0};
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *wsm = smem;
@@ -127,6 +126,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if (args.clear_status && blockIdx.x == 0 && threadIdx.x == 0) *ctl.status = DeviceStatus{0, 0, 0, 0};
 
     // Tile lt of this CTA: z row i, columns j0 .. j0+127; PRO_MX_COLS: rows i .. i+31,
     // columns j0 .. j0+3.
@@ -507,24 +507,22 @@ cudaError_t prologue_tc_setup() {
 }
 
 template <bool kVec, int kMode>
-static void launch_as(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
+static cudaError_t launch_as(const PrologueMaps &m, const PrologueArgs &a, int grid, cudaStream_t s) {
     prologue_tc_kernel<kVec, kMode><<<grid, pro::THREADS, pro::SMEM, s>>>(m.w[0], m.w[1], m.w[2], m.w[3], m.z,
                                                                           m.mask, m.a, m.b, a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prologue_tc(const PrologueMaps &m, const PrologueArgs &a, int mode, int grid, cudaStream_t s) {
     const bool vec = a.ln_w || a.ln_b || a.b_a || a.b_ag || a.b_b || a.b_bg;
     switch (mode) {
-        case PRO_BF16: vec ? launch_as<true, PRO_BF16>(m, a, grid, s) : launch_as<false, PRO_BF16>(m, a, grid, s); break;
+        case PRO_BF16: return vec ? launch_as<true, PRO_BF16>(m, a, grid, s) : launch_as<false, PRO_BF16>(m, a, grid, s);
         case PRO_MX_ROWS:
-            vec ? launch_as<true, PRO_MX_ROWS>(m, a, grid, s) : launch_as<false, PRO_MX_ROWS>(m, a, grid, s);
-            break;
+            return vec ? launch_as<true, PRO_MX_ROWS>(m, a, grid, s) : launch_as<false, PRO_MX_ROWS>(m, a, grid, s);
         case PRO_MX_COLS:
-            vec ? launch_as<true, PRO_MX_COLS>(m, a, grid, s) : launch_as<false, PRO_MX_COLS>(m, a, grid, s);
-            break;
+            return vec ? launch_as<true, PRO_MX_COLS>(m, a, grid, s) : launch_as<false, PRO_MX_COLS>(m, a, grid, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 __global__ void mask_pad_kernel(const __nv_bfloat16 *__restrict__ mask, __nv_bfloat16 *__restrict__ dst, int N,
