@@ -91,7 +91,8 @@ typedef struct trimul_params {
 
 /* Bytes of workspace that trimul_forward needs for any dtype (sized for the
  * fp32 element). Returns 0 for invalid sizes. The workspace holds a 256-byte
- * status header and a, b, x as [c_h][N][ld] with ld = N rounded up to 8. */
+ * status header and a, b, x as [c_h][N][ld] with ld = N rounded up to 64 for
+ * BF16 (every row starts on a 128-byte boundary) and to 8 for F32. */
 size_t trimul_workspace_size(int N, int c_z, int c_h);
 
 /* Exact bytes of workspace for one dtype (<= trimul_workspace_size). */
@@ -172,7 +173,7 @@ int trimul_forward_noalloc(const void *z, const void *mask, const trimul_params 
  * through torch.distributed in pair_representation_b200.sharded); the
  * prologue and epilogue are per cell, so a row block is just a grid of
  * rows x N cells. All buffers are caller-owned device memory, 16-byte
- * aligned; ld = N rounded up to 8. BF16 only (TRIMUL_ERR_UNSUPPORTED
+ * aligned; ld = N rounded up to 64. BF16 only (TRIMUL_ERR_UNSUPPORTED
  * otherwise); p->N is the full residue count and p->workspace holds the status
  * word and scratch for re-pitching mask rows:
  * trimul_shard_workspace_size(N, rows) bytes. Asynchronous. */

@@ -30,9 +30,17 @@ void set_detail(const char *what, cudaError_t e) {
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-size_t ld_of(int N) { return ((size_t)N + 7) & ~(size_t)7; }
+// Row pitch (elements) of the channel-major a, b, x sections. bf16 rows start on
+// 128-byte boundaries, so every row of a TMA box covers whole 32-byte sectors and
+// 128-byte lines (a pitch of N rounded to 8 leaves half the rows 16 bytes off a
+// sector when N is not a multiple of 16); fp32 rows on 32-byte boundaries.
+size_t ld_of(int N, int dtype = TRIMUL_DTYPE_BF16) {
+    return dtype == TRIMUL_DTYPE_F32 ? round_up((size_t)N, 8) : round_up((size_t)N, 64);
+}
 size_t elem_size(int dtype) { return dtype == TRIMUL_DTYPE_F32 ? 4 : 2; }
-size_t section_bytes(int N, int dtype) { return round_up((size_t)kC * (size_t)N * ld_of(N) * elem_size(dtype), 256); }
+size_t section_bytes(int N, int dtype) {
+    return round_up((size_t)kC * (size_t)N * ld_of(N, dtype) * elem_size(dtype), 256);
+}
 
 bool valid_dtype(int d) { return d == TRIMUL_DTYPE_F32 || d == TRIMUL_DTYPE_BF16; }
 
@@ -243,7 +251,7 @@ Views views_of(const trimul_params *p) {
     v.a = base + kHeader;
     v.b = v.a + sec;
     v.x = v.b + sec;
-    v.ld = ld_of(p->N);
+    v.ld = ld_of(p->N, p->dtype);
     return v;
 }
 

@@ -58,7 +58,8 @@ class ShardPlan:
 
     @property
     def ld(self) -> int:
-        return (self.N + 7) // 8 * 8
+        """Row pitch of the bf16 a, b, x blocks: N rounded up to 64 (the library's rule)."""
+        return (self.N + 63) // 64 * 64
 
     def rows(self, r: int):
         return split(self.N, self.world, r)

@@ -46,10 +46,10 @@ def test_version_and_strings(L):
 
 def test_workspace_size(L):
     for N in (1, 7, 64, 384, 3605):
-        ld = (N + 7) // 8 * 8
-        sec = lambda es: (128 * N * ld * es + 255) // 256 * 256
-        assert tm.trimul_workspace_size(N) == 256 + 3 * sec(4)
-        assert tm.trimul_workspace_size_dtype(N, 128, 128, tm.DTYPE_BF16) == 256 + 3 * sec(2)
+        ld32, ld16 = (N + 7) // 8 * 8, (N + 63) // 64 * 64  # fp32 rows on 32 B, bf16 rows on 128 B
+        sec = lambda es, ld: (128 * N * ld * es + 255) // 256 * 256
+        assert tm.trimul_workspace_size(N) == 256 + 3 * sec(4, ld32)
+        assert tm.trimul_workspace_size_dtype(N, 128, 128, tm.DTYPE_BF16) == 256 + 3 * sec(2, ld16)
         assert tm.trimul_workspace_size_dtype(N, 128, 128, tm.DTYPE_F32) == tm.trimul_workspace_size(N)
     assert tm.trimul_workspace_size(0) == 0
     assert tm.trimul_workspace_size(16385) == 0
@@ -161,7 +161,7 @@ def _bwd_layout_bytes(N):
     """Backward workspace: sums, weight stack, per-cell sections, then one
     [768][128] fp32 weight-gradient partial per 4096-cell chunk."""
     r = lambda v: (v + 255) // 256 * 256
-    M, C, ld = N * N, 128, (N + 7) // 8 * 8
+    M, C, ld = N * N, 128, (N + 63) // 64 * 64
     cm = C * N * ld
     slots = (M + 4095) // 4096
     parts = [10 * C * 4, 5 * C * C * 2, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
