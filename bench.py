@@ -77,7 +77,7 @@ def load_peaks():
 
 
 def source_sha(kernel: str) -> str:
-    files = {"prologue_tc_kernel": ("prologue_tc.cu", "tile_ops.cuh"), "contract_tc_kernel": ("contract_tc.cu",),
+    files = {"prologue_tc_kernel": ("prologue_tc.cu", "tile_ops.cuh", "mx_block.cuh"), "contract_tc_kernel": ("contract_tc.cu",),
              "epilogue_tc_kernel": ("epilogue_tc.cu", "tile_ops.cuh")}[kernel]
     h = hashlib.sha256()
     for f in files + ("common.cuh", "kernels.h"):
