@@ -1023,13 +1023,23 @@ int check_attn(const atomattn_params *p, const void *out) {
     return TRIMUL_OK;
 }
 
-// q, k or v [batch][n][heads][32] as (heads * 32, n, batch): boxes of 64 elements (a head pair) x `rows`.
+// q, k or v [batch][n][heads][32] as (heads * 32, n, batch): boxes of one head's 32 elements x `rows`.
 int map_attn(CUtensorMap *m, const void *t, const atomattn_params *p, uint32_t rows) {
     const uint64_t row = (uint64_t)p->heads * 32;
     const uint64_t dims[3] = {row, (uint64_t)p->n_atoms, (uint64_t)p->batch};
     const uint64_t strides[2] = {row * 2, row * 2 * (uint64_t)p->n_atoms};
-    const uint32_t box[3] = {64, rows, 1};
-    return encode(m, 3, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    const uint32_t box[3] = {32, rows, 1};
+    return encode(m, 3, t, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// bias [batch][n_windows][heads][32][128] as (slot, row, head, window, batch): boxes of one
+// window's 32 rows x 64 slots; windows past n_windows read as 0.
+int map_attn_bias(CUtensorMap *m, const atomattn_params *p) {
+    const uint64_t nw = (uint64_t)attn_windows(p), h = (uint64_t)p->heads;
+    const uint64_t dims[5] = {128, 32, h, nw, (uint64_t)p->batch};
+    const uint64_t strides[4] = {128 * 2, 32 * 128 * 2, h * 32 * 128 * 2, nw * h * 32 * 128 * 2};
+    const uint32_t box[5] = {64, 32, 1, 1, 1};
+    return encode(m, 5, p->bias, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -1296,11 +1306,13 @@ int atomattn_forward(const atomattn_params *p, void *out, trimul_stream_t stream
     for (const void *v : ptrs)
         if ((rc = check_device_ptr(v, "atom attention pointer"))) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = cuda_rc(cudaMemsetAsync(p->workspace, 0, sizeof(DeviceStatus), s), "status clear"))) return rc;
+    // The kernel clears the status word itself (CTA 0, after its setup barrier).
     AttnMaps m;
     if ((rc = map_attn(&m.q, p->q, p, 128)) || (rc = map_attn(&m.k, p->k, p, 224)) ||
         (rc = map_attn(&m.v, p->v, p, 256)))
         return rc;
+    m.bias = m.q;  // unused without a bias
+    if (p->bias && (rc = map_attn_bias(&m.bias, p))) return rc;
     AttnArgs a;
     a.batch = p->batch;
     a.n = p->n_atoms;

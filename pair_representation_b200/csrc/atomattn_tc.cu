@@ -13,13 +13,14 @@
 // [32 (r / 32), 32 (r / 32) + 128) of S; its softmax runs in the thread that
 // owns TMEM lane r, and its probabilities go to shared memory as row r of a
 // [128][256] K-major operand P whose other slots stay 0. Then
-//   O[128][64] = P V               (tcgen05, TMEM columns [256, 320) or [320, 384) by unit parity)
+//   O[128][32] = P V               (tcgen05, TMEM columns [256, 288) or [288, 320) by unit parity)
 // over 256 key rows (slots 224 .. 255 have P = 0).
 //
-// Q, K and V are TMA-loaded as rows of 64 bf16: the head pair (h & ~1, h | 1),
-// so that every operand has 128-byte rows (128-byte swizzle). S contracts the
-// head's 32 of them (the K steps at byte offset 64 (h & 1)), and O's columns
-// [32 (h & 1), 32 (h & 1) + 32) are the head's output.
+// Q, K and V are TMA-loaded as rows of one head's 32 bf16 (64-byte rows, 64-byte
+// swizzle): S contracts them in two K = 16 steps, and O = P V is M = 128, N = 32.
+// The unit's bias (4 windows x 32 rows x 128 slots, 32 KB) is TMA-loaded into the
+// same stage (128-byte swizzle) and read from shared memory by the softmax warps,
+// each lane its own row.
 //
 // Warps 0-15: softmax and epilogue; warp w serves the query rows of TMEM lane
 // quarter w & 3 and a quarter of their slots. Warp 16, one thread: TMA loads
@@ -39,11 +40,15 @@ constexpr int WPG = 4;                       // windows per unit
 constexpr int ROWS = QW * WPG;               // 128 query rows
 constexpr int UNION = QW * (WPG - 1) + KW;   // 224 key rows of S
 constexpr int VROWS = 256;                   // key rows of the second product
-constexpr int ROWB = 128;                    // bytes per operand row (64 bf16)
-constexpr int Q_BYTES = ROWS * ROWB;         // 16 KB
-constexpr int K_BYTES = UNION * ROWB;        // 28 KB
-constexpr int V_BYTES = VROWS * ROWB;        // 32 KB
-constexpr int STAGE_BYTES = Q_BYTES + K_BYTES + V_BYTES;
+constexpr int ROWB = 64;                     // bytes per operand row (one head's 32 bf16)
+constexpr int Q_BYTES = ROWS * ROWB;         // 8 KB
+constexpr int K_BYTES = UNION * ROWB;        // 14 KB
+constexpr int V_BYTES = VROWS * ROWB;        // 16 KB
+constexpr int QKV_BYTES = Q_BYTES + K_BYTES + V_BYTES;
+constexpr int BIAS_HALF = QW * 128;          // one window's 32 rows x 64 slots (4 KB, 128-byte rows)
+constexpr int BIAS_WIN = 2 * BIAS_HALF;      // one window's 32 x 128 slots
+constexpr int BIAS_BYTES = WPG * BIAS_WIN;   // 32 KB
+constexpr int STAGE_BYTES = QKV_BYTES + BIAS_BYTES;
 constexpr int P_BLOCK = ROWS * 128;          // one 64-slot block of P (16 KB)
 constexpr int P_BYTES = 4 * P_BLOCK;
 constexpr int S_COL = 0, O_COL = 256, TMEM_COLS = 512;
@@ -52,7 +57,7 @@ constexpr int THREADS = (WORKER_WARPS + 1) * 32;
 constexpr int RED_BYTES = 2 * 2 * 4 * ROWS * 4;  // [max, sum][unit parity][key part][row] floats
 constexpr int BAR_BYTES = 128;  // 11 mbarriers, TMEM address, abort flag
 constexpr size_t SMEM = 1024 + 2 * (size_t)STAGE_BYTES + P_BYTES + RED_BYTES + BAR_BYTES;
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(STAGE_BYTES % 1024 == 0 && QKV_BYTES % 1024 == 0, "stage alignment");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace aa
 
@@ -67,16 +72,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// 16-byte load on the read-only path, kept where it is written (an early
-// prefetch that the compiler must not sink to the first use).
-__device__ __forceinline__ uint4 ldg_early(const uint4 *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
+// 2-byte load on the read-only path, kept where it is written (an early prefetch
+// that the compiler must not sink to the first use).
 __device__ __forceinline__ uint16_t ldg_early_u16(const uint16_t *p) {
     uint16_t v;
     asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
@@ -111,7 +108,8 @@ __device__ __forceinline__ void unit_step(Unit &x, const AttnArgs &a) {
 
 __global__ void __launch_bounds__(aa::THREADS, 1)
     atomattn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmBias,
+                       const AttnArgs args) {
     using namespace aa;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -148,6 +146,7 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        if (args.bias) tma_prefetch_desc(&tmBias);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -165,22 +164,35 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // The call starts here: CTA 0 clears the status word (every failure is recorded by a
+    // bounded wait after ctl.timeout_ns, long after all CTAs of this one-wave grid started).
+    if (blockIdx.x == 0 && threadIdx.x == 0) *ctl.status = DeviceStatus{0, 0, 0, 0};
 
     if (warp == WORKER_WARPS) {
         if (lane == 0) {
             // ---------------- TMA producer and MMA issuer ----------------
             const uint32_t idesc_s = idesc_bf16(128, UNION, 0, 0);
-            const uint32_t idesc_o = idesc_bf16(128, 64, 0, 1);
+            const uint32_t idesc_o = idesc_bf16(128, 32, 0, 1);
             const uint64_t pdesc = sdesc_sw128(pbase, 16, 1024);
             int issued = 0, landed = 0;
             auto issue = [&](int lu) {
                 const Unit un = unit_of((int)blockIdx.x + lu * (int)gridDim.x, args);
                 uint8_t *st = stage_base + (lu & 1) * STAGE_BYTES;
-                const int x = (un.h & ~1) * 32, a0 = un.g * ROWS;
-                mbar_arrive_expect_tx(&full[lu & 1], STAGE_BYTES);
+                const int x = un.h * 32, a0 = un.g * ROWS;
+                mbar_arrive_expect_tx(&full[lu & 1], args.bias ? STAGE_BYTES : QKV_BYTES);
                 tma_load_3d(st, &tmQ, &full[lu & 1], x, a0, un.b);
                 tma_load_3d(st + Q_BYTES, &tmK, &full[lu & 1], x, a0 + KOFF, un.b);
                 tma_load_3d(st + Q_BYTES + K_BYTES, &tmV, &full[lu & 1], x, a0 + KOFF, un.b);
+                if (args.bias) {
+                    // Windows 4g .. 4g + 3, each as two boxes of 32 rows x 64 slots; windows past
+                    // the last one are out of bounds and read as 0.
+#pragma unroll
+                    for (int w = 0; w < WPG; ++w)
+#pragma unroll
+                        for (int half = 0; half < 2; ++half)
+                            tma_load_5d(st + QKV_BYTES + w * BIAS_WIN + half * BIAS_HALF, &tmBias, &full[lu & 1],
+                                        64 * half, 0, un.h, un.g * WPG + w, un.b);
+                }
                 ++issued;
             };
             auto mma_s = [&](int lu) -> bool {
@@ -188,13 +200,11 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                     return false;
                 ++landed;
                 tc_fence_after();
-                const Unit un = unit_of((int)blockIdx.x + lu * (int)gridDim.x, args);
                 const uint32_t st = smem_u32(stage_base + (lu & 1) * STAGE_BYTES);
-                const uint32_t kofs = (uint32_t)(un.h & 1) * 64;  // the head's 32 elements in the 64-element row
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16(tmem + S_COL, sdesc_sw128(st + kofs + kk * 32, 16, 1024),
-                             sdesc_sw128(st + Q_BYTES + kofs + kk * 32, 16, 1024), idesc_s, kk ? 1u : 0u);
+                    mma_bf16(tmem + S_COL, sdesc_sw64(st + kk * 32, 16, 512), sdesc_sw64(st + Q_BYTES + kk * 32, 16, 512),
+                             idesc_s, kk ? 1u : 0u);
                 mma_commit(sfull);
                 return true;
             };
@@ -220,13 +230,13 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 tc_fence_after();
                 // Descriptor start addresses count 16-byte units in their low bits:
                 // step K by adding to the descriptor.
-                const uint64_t vdesc = sdesc_sw128(smem_u32(stage_base + (lu & 1) * STAGE_BYTES) + Q_BYTES + K_BYTES,
-                                                   V_BYTES, 1024);
-                const uint32_t od = tmem + O_COL + 64 * (lu & 1);
+                const uint64_t vdesc = sdesc_sw64(smem_u32(stage_base + (lu & 1) * STAGE_BYTES) + Q_BYTES + K_BYTES,
+                                                  V_BYTES, 512);
+                const uint32_t od = tmem + O_COL + 32 * (lu & 1);
 #pragma unroll
                 for (int kk = 0; kk < VROWS / 16; ++kk)
                     mma_bf16(od, pdesc + (uint64_t)(((kk >> 2) * P_BLOCK + (kk & 3) * 32) >> 4),
-                             vdesc + (uint64_t)((kk * 2048) >> 4), idesc_o, kk ? 1u : 0u);
+                             vdesc + (uint64_t)((kk * 16 * ROWB) >> 4), idesc_o, kk ? 1u : 0u);
                 mma_commit(ofull);
                 if (lu + 2 < my_units) {
                     // The stage of unit lu is free once its second product has completed.
@@ -247,8 +257,8 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         // ---------------- softmax and epilogue: thread = query row ----------------
         // Warp (qr, kp) = (warp & 3, warp >> 2) owns query rows 32 qr .. 32 qr + 31
         // (TMEM lane quarter qr) and slots 32 kp .. 32 kp + 31 of their window.
-        // Unit lu: its bias slice and key-mask value were loaded during unit lu - 1;
-        // logits stay in registers; partial row maxima and sums are exchanged
+        // Unit lu: its bias rows are in its stage (shared memory), its key-mask value was
+        // loaded during unit lu - 1; logits stay in registers; partial row maxima and sums are exchanged
         // among the quarter's 4 warps through `red` (double-buffered by unit
         // parity) through one mbarrier phase per unit; P is written once the
         // previous unit's second product has finished reading it; then that
@@ -257,22 +267,10 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         const uint32_t lanebase = tmem + ((uint32_t)(qr * 32) << 16);
         const float log2e = 1.4426950408889634f;
         float *red_max = red, *red_sum = red + 2 * 4 * ROWS;
-        uint4 bias[4];
         uint16_t mk_n = 0;
-        bool hb_n = false;
+        const bool hb = args.bias != nullptr;
         auto prefetch = [&](const Unit &un) {
             const int w = un.g * WPG + qr, at = w * QW + KOFF + 32 * kp + lane;
-            hb_n = args.bias != nullptr && w < args.n_windows;
-            if (hb_n) {
-                // Coalesced: instruction i reads rows 8i .. 8i + 7 of the warp's [32 rows][32 slots]
-                // slice, 64 contiguous bytes per row (lane l: row 8i + l / 4, 16-byte chunk l % 4).
-                // The rows reach their owning lanes (row = lane) by shuffles at first use.
-                const __nv_bfloat16 *slice =
-                    args.bias + (((size_t)un.b * args.n_windows + w) * args.heads + un.h) * QW * KW + 32 * kp;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    bias[i] = ldg_early(reinterpret_cast<const uint4 *>(slice + (8 * i + (lane >> 2)) * KW + 8 * (lane & 3)));
-            }
             mk_n = (at < 0 || at >= args.n) ? (uint16_t)0
                    : args.mask ? ldg_early_u16(reinterpret_cast<const uint16_t *>(args.mask) + (size_t)un.b * args.n + at)
                                : (uint16_t)0x3f80u;  // bf16 1.0
@@ -287,7 +285,7 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                          : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]),
                            "=r"(o[7])
-                         : "r"(lanebase + (uint32_t)(O_COL + 64 * (lu & 1) + 32 * (prev.h & 1) + 8 * kp)));
+                         : "r"(lanebase + (uint32_t)(O_COL + 32 * (lu & 1) + 8 * kp)));
             tmem_ld_wait();
             const int atom_q = prev.g * ROWS + row;
             if (atom_q < args.n) {
@@ -308,13 +306,17 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         for (int lu = 0; lu < my_units; ++lu) {
             const Unit un = cur;
             unit_step(cur, args);  // the next unit of this CTA
-            const bool hb = hb_n;
             const uint32_t vb = __ballot_sync(0xffffffffu, (mk_n & 0x7fffu) != 0);  // slot 32 kp + i valid: bit i
             if (!(ok = warp_wait(sfull, (uint32_t)lu & 1u, abort_flag, ctl, SITE_ATT | 4, lu))) break;
+            // The stage's bias (TMA-written) is read below: observe its barrier here too (the
+            // issuing thread waited on it before S, so this only makes the bytes visible).
+            if (hb && !(ok = warp_wait(&full[lu & 1], (uint32_t)(lu >> 1) & 1u, abort_flag, ctl, SITE_ATT | 10, lu)))
+                break;
             tc_fence_after();
-            // Logits of the 32 slots in the log2 domain (invalid: -inf) and their maximum.
-            // Chunk c (slots 8c .. 8c + 7) of this lane's bias row sits in bias[lane / 8] of
-            // lane 4 (lane % 8) + c: fetched by shuffles right before its logits.
+            // Logits of the 32 slots in the log2 domain (invalid: -inf) and their maximum. This
+            // lane's bias row is row `lane` of window qr's tile, slots 32 kp .. 32 kp + 31 in
+            // 16-byte chunks 4 (kp & 1) .. 4 (kp & 1) + 3 of its 64-slot half kp / 2
+            // (128-byte swizzle: chunk ^ (lane & 7)).
             float l[32];
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             {
@@ -325,21 +327,12 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_read);
+                const uint8_t *brow = stage_base + (lu & 1) * STAGE_BYTES + QKV_BYTES + qr * BIAS_WIN +
+                                      (kp >> 1) * BIAS_HALF + lane * 128;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint4 bc = make_uint4(0u, 0u, 0u, 0u);
-                    if (hb) {
-                        const int src = 4 * (lane & 7) + c;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint4 t;
-                            t.x = __shfl_sync(0xffffffffu, bias[i].x, src);
-                            t.y = __shfl_sync(0xffffffffu, bias[i].y, src);
-                            t.z = __shfl_sync(0xffffffffu, bias[i].z, src);
-                            t.w = __shfl_sync(0xffffffffu, bias[i].w, src);
-                            if ((lane >> 3) == i) bc = t;
-                        }
-                    }
+                    if (hb) bc = *reinterpret_cast<const uint4 *>(brow + (((4 * (kp & 1) + c) ^ (lane & 7)) << 4));
                     const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bc);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
@@ -415,7 +408,7 @@ cudaError_t atomattn_tc_setup() {
 }
 
 cudaError_t launch_atomattn_tc(const AttnMaps &m, const AttnArgs &a, int grid, cudaStream_t s) {
-    atomattn_tc_kernel<<<grid, aa::THREADS, aa::SMEM, s>>>(m.q, m.k, m.v, a);
+    atomattn_tc_kernel<<<grid, aa::THREADS, aa::SMEM, s>>>(m.q, m.k, m.v, m.bias, a);
     return cudaGetLastError();
 }
 

@@ -245,7 +245,8 @@ struct AttnArgs {
 };
 
 struct AttnMaps {
-    CUtensorMap q, k, v;  // 3-D (heads * 32, n, batch), boxes (64, 128 | 224 | 256, 1), swizzle 128B
+    CUtensorMap q, k, v;  // 3-D (heads * 32, n, batch), boxes (32, 128 | 224 | 256, 1), swizzle 64B
+    CUtensorMap bias;     // 5-D (128 slots, 32 rows, heads, n_windows, batch), box (64, 32, 1, 1, 1), swizzle 128B
 };
 
 size_t atomattn_tc_smem();
