@@ -68,6 +68,13 @@ __device__ __forceinline__ uint32_t p_chunk_addr(uint32_t pbase, int row, int cu
     return pbase + (uint32_t)((cu >> 3) * aa::P_BLOCK + row * 128 + (((cu & 7) ^ (row & 7)) << 4));
 }
 
+// 2^x on the MUFU (ex2.approx, relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -329,20 +336,31 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 if (lane == 0) mbar_arrive(s_read);
                 const uint8_t *brow = stage_base + (lu & 1) * STAGE_BYTES + QKV_BYTES + qr * BIAS_WIN +
                                       (kp >> 1) * BIAS_HALF + lane * 128;
+                // l = s (scale log2 e) + bias log2 e, two slots at a time (packed fp32x2).
+                const float2 sc2 = make_float2(args.scale * log2e, args.scale * log2e);
+                const float2 l2e = make_float2(log2e, log2e);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint4 bc = make_uint4(0u, 0u, 0u, 0u);
                     if (hb) bc = *reinterpret_cast<const uint4 *>(brow + (((4 * (kp & 1) + c) ^ (lane & 7)) << 4));
-                    const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&bc);
+                    const uint32_t bw[4] = {bc.x, bc.y, bc.z, bc.w};
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int t = 8 * c + u;
-                        const float2 f = __bfloat1622float2(bb[u >> 1]);
-                        const float bj = (u & 1) ? f.y : f.x;
-                        l[t] = ((vb >> t) & 1u) ? (__uint_as_float(sv[t]) * args.scale + bj) * log2e : -INFINITY;
-                        mx4[t & 3] = fmaxf(mx4[t & 3], l[t]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int t = 8 * c + 2 * u;
+                        const float2 b2 = make_float2(__uint_as_float(bw[u] << 16), __uint_as_float(bw[u] & 0xFFFF0000u));
+                        const float2 lv = __ffma2_rn(make_float2(__uint_as_float(sv[t]), __uint_as_float(sv[t + 1])), sc2,
+                                                     __fmul2_rn(b2, l2e));
+                        l[t] = lv.x;
+                        l[t + 1] = lv.y;
                     }
                 }
+                if (vb != 0xFFFFFFFFu) {  // warp-uniform: some of the 32 slots are masked or outside the sequence
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if (!((vb >> t) & 1u)) l[t] = -INFINITY;
+                }
+#pragma unroll
+                for (int t = 0; t < 32; ++t) mx4[t & 3] = fmaxf(mx4[t & 3], l[t]);
             }
             if (lu + 1 < my_units) prefetch(cur);
             float *rm = red_max + (lu & 1) * 4 * ROWS, *rs = red_sum + (lu & 1) * 4 * ROWS;
@@ -360,21 +378,24 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             // P is free once the previous unit's second product has completed.
             if (lu > 0 && !(ok = warp_wait(ofull, (uint32_t)(lu - 1) & 1u, abort_flag, ctl, SITE_ATT | 5, lu))) break;
             // Probabilities (bf16), their partial sum, and this warp's 4 chunks of row `row` of P.
-            float s4[4] = {0.f, 0.f, 0.f, 0.f};
+            // p = 2^(l - m) (hardware ex2; a masked slot's -inf gives 0), rounded to bf16; the
+            // row sum adds the rounded values, the ones the second product uses.
+            float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     const int j = 8 * c + 2 * t;
-                    const __nv_bfloat162 pp = __floats2bfloat162_rn(exp2f(l[j] - m), exp2f(l[j + 1] - m));
-                    const float2 pr = __bfloat1622float2(pp);
-                    s4[t] += pr.x + pr.y;
-                    pk[t] = *reinterpret_cast<const uint32_t *>(&pp);
+                    const float2 d = __fadd2_rn(make_float2(l[j], l[j + 1]), nm2);
+                    pk[t] = pack_bf16x2(ex2_approx(d.x), ex2_approx(d.y));
+                    s2[t & 1] = __fadd2_rn(s2[t & 1], make_float2(__uint_as_float(pk[t] << 16),
+                                                                  __uint_as_float(pk[t] & 0xFFFF0000u)));
                 }
                 st_shared_v4(p_chunk_addr(pbase, row, 4 * qr + 4 * kp + c), pk[0], pk[1], pk[2], pk[3]);
             }
-            rs[kp * ROWS + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            rs[kp * ROWS + row] = (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
