@@ -299,7 +299,9 @@ __device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
 // try_wait); the outcome is made warp-uniform.
 static __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                  const KernelCtl &ctl, int site, int aux) {
-    const int ok = wait_bounded(bar, parity, abort_flag, ctl, site, aux) ? 1 : 0;
+    // The first test is inline: the call (and the register saves it implies) happens only
+    // when the phase is still open.
+    const int ok = (mbar_try_wait(bar, parity) || wait_bounded(bar, parity, abort_flag, ctl, site, aux)) ? 1 : 0;
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
