@@ -118,9 +118,8 @@ constexpr uint32_t kWaitHintNs = 1000000;  // upper bound on one suspension: 1 m
 // raised `abort_flag`, or if this wait ran past ctl.timeout_ns; in the latter
 // case it raises the flag and records DEV_TIMEOUT with `site`. May be called by
 // one thread or by every lane of a warp.
-static __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          const KernelCtl &ctl, int site, int aux) {
-    if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                       const KernelCtl &ctl, int site, int aux) {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
@@ -131,6 +130,13 @@ static __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
             return false;
         }
     }
+}
+
+// The first test is inline: the call (and the register saves of the calling
+// convention) happens only when the phase is still open.
+static __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                    const KernelCtl &ctl, int site, int aux) {
+    return mbar_try_wait(bar, parity) || wait_bounded_slow(bar, parity, abort_flag, ctl, site, aux);
 }
 
 // Like wait_bounded but ignores the abort flag: used on the way out, to let
@@ -299,9 +305,7 @@ __device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
 // try_wait); the outcome is made warp-uniform.
 static __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                  const KernelCtl &ctl, int site, int aux) {
-    // The first test is inline: the call (and the register saves it implies) happens only
-    // when the phase is still open.
-    const int ok = (mbar_try_wait(bar, parity) || wait_bounded(bar, parity, abort_flag, ctl, site, aux)) ? 1 : 0;
+    const int ok = wait_bounded(bar, parity, abort_flag, ctl, site, aux) ? 1 : 0;
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
