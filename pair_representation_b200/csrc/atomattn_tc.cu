@@ -285,15 +285,17 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         Unit prev{0, 0, 0};
         float sum_prev = 0.f;
         bool ok = true;
-        auto epilogue = [&](int lu) {
-            // Output columns 8 kp .. 8 kp + 7 of unit lu (its second product has completed).
+        // Output columns 8 kp .. 8 kp + 7 of unit lu (its second product has completed): the
+        // tensor-memory load is issued first, the normalisation and store after the wait.
+        auto load_o = [&](int lu, uint32_t (&o)[8]) {
             tc_fence_after();
-            uint32_t o[8];
             asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                          : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]),
                            "=r"(o[7])
                          : "r"(lanebase + (uint32_t)(O_COL + 32 * (lu & 1) + 8 * kp)));
-            tmem_ld_wait();
+        };
+        auto store_o = [&](uint32_t (&o)[8]) {
+            tmem_ld_wait_regs(o);
             const int atom_q = prev.g * ROWS + row;
             if (atom_q < args.n) {
                 const float inv = sum_prev > 0.f ? 1.f / sum_prev : 0.f;
@@ -329,20 +331,25 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             {
                 uint32_t sv[32];
                 tmem_ld32(lanebase + (uint32_t)(S_COL + 32 * qr + 32 * kp), sv);
-                tmem_ld_wait();
+                // The bias row is read from shared memory while the S load is in flight.
+                uint4 bcs[4];
+                const uint8_t *brow = stage_base + (lu & 1) * STAGE_BYTES + QKV_BYTES + qr * BIAS_WIN +
+                                      (kp >> 1) * BIAS_HALF + lane * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    bcs[c] = hb ? *reinterpret_cast<const uint4 *>(brow + (((4 * (kp & 1) + c) ^ (lane & 7)) << 4))
+                                : make_uint4(0u, 0u, 0u, 0u);
+                tmem_ld_wait_regs(sv);
                 // S is in registers: the next unit's S may overwrite it.
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_read);
-                const uint8_t *brow = stage_base + (lu & 1) * STAGE_BYTES + QKV_BYTES + qr * BIAS_WIN +
-                                      (kp >> 1) * BIAS_HALF + lane * 128;
                 // l = s (scale log2 e) + bias log2 e, two slots at a time (packed fp32x2).
                 const float2 sc2 = make_float2(args.scale * log2e, args.scale * log2e);
                 const float2 l2e = make_float2(log2e, log2e);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint4 bc = make_uint4(0u, 0u, 0u, 0u);
-                    if (hb) bc = *reinterpret_cast<const uint4 *>(brow + (((4 * (kp & 1) + c) ^ (lane & 7)) << 4));
+                    const uint4 bc = bcs[c];
                     const uint32_t bw[4] = {bc.x, bc.y, bc.z, bc.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -375,8 +382,11 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
                 const float *ps = red_sum + ((lu - 1) & 1) * 4 * ROWS;
                 sum_prev = ps[row] + ps[ROWS + row] + ps[2 * ROWS + row] + ps[3 * ROWS + row];
             }
-            // P is free once the previous unit's second product has completed.
+            // P is free once the previous unit's second product has completed; its output is then
+            // in tensor memory, and its load runs under the exponentials below.
             if (lu > 0 && !(ok = warp_wait(ofull, (uint32_t)(lu - 1) & 1u, abort_flag, ctl, SITE_ATT | 5, lu))) break;
+            uint32_t o_prev[8];
+            if (lu > 0) load_o(lu - 1, o_prev);
             // Probabilities (bf16), their partial sum, and this warp's 4 chunks of row `row` of P.
             // p = 2^(l - m) (hardware ex2; a masked slot's -inf gives 0), rounded to bf16; the
             // row sum adds the rounded values, the ones the second product uses.
@@ -400,7 +410,7 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(pready);
-            if (lu > 0) epilogue(lu - 1);
+            if (lu > 0) store_o(o_prev);
             prev = un;
         }
         if (ok && my_units > 0) {
@@ -412,7 +422,11 @@ __global__ void __launch_bounds__(aa::THREADS, 1)
         if (ok && my_units > 0) {
             const float *ps = red_sum + ((my_units - 1) & 1) * 4 * ROWS;
             sum_prev = ps[row] + ps[ROWS + row] + ps[2 * ROWS + row] + ps[3 * ROWS + row];
-            if (warp_wait(ofull, (uint32_t)(my_units - 1) & 1u, abort_flag, ctl, SITE_ATT | 6, 0)) epilogue(my_units - 1);
+            if (warp_wait(ofull, (uint32_t)(my_units - 1) & 1u, abort_flag, ctl, SITE_ATT | 6, 0)) {
+                uint32_t o_last[8];
+                load_o(my_units - 1, o_last);
+                store_o(o_last);
+            }
         }
     }
 

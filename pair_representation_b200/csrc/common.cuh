@@ -263,6 +263,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// tmem_ld_wait, then tie the loaded registers to a point after it (an empty volatile asm
+// that reads and writes each), so no use of them can be scheduled before the wait even
+// when other work sits between the load and the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 
 // 16 lanes x 256 bits, 4 repetitions along columns (32 columns): thread t gets, for
 // repetition k, r[4k], r[4k+1] = lane (base + t/4), columns 8k + 2(t%4) + {0,1} and
