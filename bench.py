@@ -857,6 +857,24 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_configs:
         del flush
         configs = per_config_timings(tm, pi, torch, dev, stream)
+        if not args.no_cpu_baseline:
+            # The float64 oracle on every workload: the whole layer where it takes seconds
+            # (N <= 384), a sampled grid of about 2 s elsewhere, with the full layer's time
+            # extrapolated from the measured rate (every cell costs the same).
+            for wid, wk in sorted(pi.WORKLOADS.items()):
+                if wk.name not in configs:
+                    continue
+                if wk.N <= 384:
+                    cells, secs = oracle_sample(wk, wk.N)
+                    sample, n_idx = "the whole layer", wk.N
+                else:
+                    cells, secs, n_idx = calibrated_oracle(wk, 2.0)
+                    sample = f"{n_idx} x {n_idx} sampled cells per direction"
+                rate = cells / secs
+                configs[wk.name]["cpu_oracle"] = {
+                    "pair_cells_per_s": round(rate, 1), "sample": sample, "cores": os.cpu_count(),
+                    "full_layer_s": round(wk.N * wk.N * len(wk.directions) / rate, 2),
+                    "full_layer_s_is": "measured" if n_idx == wk.N else "extrapolated"}
     if rank == 0 and world == 1 and not args.no_backward:
         backward = backward_timings(tm, pi, torch, dev, stream, peaks)
     attention = None

@@ -45,7 +45,7 @@ extern "C" {
 typedef struct atomattn_params {
     int batch;        /* >= 1 */
     int n_atoms;      /* >= 1 */
-    int heads;        /* even, 2 .. 64; batch * heads * ceil(n_atoms / 128) < 2^31 */
+    int heads;        /* 1 .. 64; batch * heads * ceil(n_atoms / 128) < 2^31 */
     int head_dim;     /* must be 32 */
     const void *q, *k, *v;
     const void *bias;       /* or NULL */

@@ -1005,7 +1005,7 @@ int check_attn(const atomattn_params *p, const void *out) {
     if (!p || !out || !p->q || !p->k || !p->v) return TRIMUL_ERR_INVALID_ARG;
     if (p->batch < 1 || p->n_atoms < 1 || p->heads < 1) return TRIMUL_ERR_INVALID_ARG;
     if (p->batch > (1 << 20) || p->n_atoms > (1 << 26)) return TRIMUL_ERR_INVALID_ARG;
-    if (p->head_dim != 32 || p->heads > 64 || (p->heads & 1)) return TRIMUL_ERR_UNSUPPORTED;
+    if (p->head_dim != 32 || p->heads > 64) return TRIMUL_ERR_UNSUPPORTED;
     if ((long long)p->batch * p->heads * ((p->n_atoms + 127) / 128) > 0x7fffffffLL) return TRIMUL_ERR_UNSUPPORTED;
     const void *al16[] = {p->q, p->k, p->v, p->bias, out};
     for (const void *v : al16)

@@ -272,7 +272,7 @@ def test_atomattn_argument_checks(L):
     assert tm.lib().atomattn_forward(None, AOUT, None) == E["TRIMUL_ERR_INVALID_ARG"]
     assert f(_attn(), out=None) == E["TRIMUL_ERR_INVALID_ARG"]
     for field, val, code in (("batch", 0, "INVALID_ARG"), ("n_atoms", 0, "INVALID_ARG"), ("heads", 0, "INVALID_ARG"),
-                             ("head_dim", 64, "UNSUPPORTED"), ("heads", 3, "UNSUPPORTED"),
+                             ("head_dim", 64, "UNSUPPORTED"), ("heads", 65, "UNSUPPORTED"),
                              ("heads", 66, "UNSUPPORTED"), ("q", None, "INVALID_ARG"),
                              ("k", BASE + 8, "MISALIGNED"), ("bias", BASE + 0x4000008, "MISALIGNED"),
                              ("atom_mask", BASE + 1, "MISALIGNED"), ("workspace", None, "WORKSPACE"),

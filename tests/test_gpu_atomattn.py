@@ -56,7 +56,7 @@ def run(q, k, v, b, m):
 
 
 @pytest.mark.parametrize("B,n,H", [(1, 1, 2), (1, 32, 2), (2, 100, 4), (1, 128, 4), (1, 129, 2), (2, 257, 4),
-                                   (3, 300, 2), (1, 1000, 6)])
+                                   (3, 300, 2), (1, 1000, 6), (1, 100, 1), (2, 257, 3), (1, 300, 5)])
 def test_atomattn_parity(B, n, H):
     q, k, v, b, m = draw(B, n, H, seed=n + 7 * H)
     got = run(q, k, v, b, m)
