@@ -59,16 +59,20 @@ constexpr int Z_HALF = TILE * 128;      // 16 KB
 constexpr int Z_BYTES = 2 * Z_HALF;     // 32 KB
 constexpr int ST_BYTES = 32 * 32 * 2;   // 2 KB per warp buffer: [32 ch][32 cells], 64-byte swizzle
 constexpr int ST_PER_WARP = 2;
-constexpr int MASK_SLOTS = 4;           // mask rows of tiles lt .. lt + 3 (indexed lt % 4)
+constexpr int MASK_SLOTS = 3;           // mask rows of tiles lt .. lt + 2 (indexed lt % 3)
 constexpr int MASK_BYTES = TILE * 2;     // one bf16 mask row segment per tile
+constexpr int PB_BYTES = 4 * 128 * 2;    // folded projection biases, bf16 [a, ag / 2, b, bg / 2][128]
 constexpr int BAR_BYTES = 128;
 constexpr size_t SMEM = 1024 + (size_t)W_BYTES + 2 * Z_BYTES + (size_t)WORKERS * ST_PER_WARP * ST_BYTES +
-                        MASK_SLOTS * MASK_BYTES + BAR_BYTES;
+                        MASK_SLOTS * MASK_BYTES + PB_BYTES + BAR_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pro
 
-// kVec: some LayerNorm affine or projection bias is present (general path);
-// without them the kernel skips every per-channel vector access. kMode: PRO_BF16,
+// kVec: some LayerNorm affine or projection bias is present (general path). The
+// LayerNorm affine is folded into the projections once per CTA (W' = W diag(gamma) in
+// shared memory, b' = b + W beta), so the normalisers always run the plain
+// LayerNorm and the gating adds b' from shared memory; without them the kernel
+// skips every per-channel vector access. kMode: PRO_BF16,
 // PRO_MX_ROWS or PRO_MX_COLS.
 template <bool kVec, int kMode>
 __global__ void __launch_bounds__(pro::THREADS, 1)
@@ -83,8 +87,9 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
     uint8_t *wsm = smem;
     uint8_t *zsm = smem + W_BYTES;                 // [2] z tiles
     uint8_t *stsm = zsm + 2 * Z_BYTES;             // [8 warps][2] staging buffers
-    uint8_t *msm = stsm + WORKERS * ST_PER_WARP * ST_BYTES;  // [4] mask rows (bf16)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(msm + MASK_SLOTS * MASK_BYTES);
+    uint8_t *msm = stsm + WORKERS * ST_PER_WARP * ST_BYTES;  // [3] mask rows (bf16)
+    __nv_bfloat16 *pbias = reinterpret_cast<__nv_bfloat16 *>(msm + MASK_SLOTS * MASK_BYTES);  // kVec: b'
+    uint64_t *bars = reinterpret_cast<uint64_t *>(msm + MASK_SLOTS * MASK_BYTES + PB_BYTES);
     uint64_t *wbar = bars;        // weights landed
     uint64_t *zfull = bars + 1;   // [2] z tile landed
     uint64_t *mma_a = bars + 3;   // a-half projections done
@@ -163,14 +168,15 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                     tma_load_3d(dst, &tmZ, &zfull[lt & 1], 0, j0, i);
                     tma_load_3d(dst + Z_HALF, &tmZ, &zfull[lt & 1], 64, j0, i);
                 }
-                // Mask slot lt % 4 last served tile lt - 4, whose gating ended before the b-half
-                // MMA of tile lt - 2, which this load waited for. PRO_MX_COLS reads the
+                // Mask slot lt % 3 last served tile lt - 3, whose gating (which reads its mask
+                // first) ended before the b-half MMA of tile lt - 2, which this load waited for.
+                // PRO_MX_COLS reads the
                 // transposed mask: [4 columns][32 rows], the same cell order as z.
                 if (args.has_mask) {
                     if (kMode == PRO_MX_COLS)
-                        tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], i, j0);
+                        tma_load_2d(msm + (lt % MASK_SLOTS) * MASK_BYTES, &tmMask, &zfull[lt & 1], i, j0);
                     else
-                        tma_load_2d(msm + (lt & 3) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
+                        tma_load_2d(msm + (lt % MASK_SLOTS) * MASK_BYTES, &tmMask, &zfull[lt & 1], j0, i);
                 }
             };
             // D[:, half*256 .. +255] = zh * W[half*256 .. +255]^T over K = 128.
@@ -241,8 +247,9 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             const int b = lt & 1;
             if (!(ok = warp_wait(&zfull[b], (uint32_t)(lt >> 1) & 1u, abort_flag, ctl, SITE_PRO | 6, lt))) break;
             uint8_t *tile = zsm + b * Z_BYTES;
-            ln_row_sw128<kVec>(tile, Z_HALF, t >> 1, t & 1, args.ln_w, args.ln_b, args.eps);
-            ln_row_sw128<kVec>(tile, Z_HALF, 64 + (t >> 1), t & 1, args.ln_w, args.ln_b, args.eps);
+            // The affine part is folded into the projections (kVec): plain LayerNorm here.
+            ln_row_sw128<false>(tile, Z_HALF, t >> 1, t & 1, nullptr, nullptr, args.eps);
+            ln_row_sw128<false>(tile, Z_HALF, 64 + (t >> 1), t & 1, nullptr, nullptr, args.eps);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ln_done[b]);
@@ -344,8 +351,6 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
             uint32_t P[16];  // packed bf16 pairs: [hf][k][e] -> P[hf * 8 + k * 2 + e]
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const __nv_bfloat16 *bv = which ? args.b_b : args.b_a;
-                const __nv_bfloat16 *bg = which ? args.b_bg : args.b_ag;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
 #pragma unroll
@@ -357,8 +362,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
                         // g holds (W_g zh) / 2: the gate weights were halved in shared memory.
                         if (kVec) {
                             const int c = ch0 + 8 * k + 2 * (lane & 3);
-                            if (bg) g = __ffma2_rn(ld_pair_bf16(bg, c), make_float2(0.5f, 0.5f), g);
-                            if (bv) v = __fadd2_rn(v, ld_pair_bf16(bv, c));
+                            g = __fadd2_rn(g, ld_pair_bf16(pbias + (2 * which + 1) * 128, c));
+                            v = __fadd2_rn(v, ld_pair_bf16(pbias + 2 * which * 128, c));
                         }
                         const float h2 = hm[hf * 2 + e];
                         const float2 hh2 = make_float2(h2, h2);
@@ -403,7 +408,7 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         // from the mask that landed with the tile (zero past N). The first cell of the
         // warp's run of 32 along its row (PRO_MX_COLS: along its column) is `first`.
         auto read_hm = [&](int lt, int first, float (&hm)[4]) {
-            const uint16_t *mrow = reinterpret_cast<const uint16_t *>(msm + (lt & 3) * MASK_BYTES);
+            const uint16_t *mrow = reinterpret_cast<const uint16_t *>(msm + (lt % MASK_SLOTS) * MASK_BYTES);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int jc = 32 * q + 16 * (c >> 1) + 8 * (c & 1) + (lane >> 2);
@@ -416,7 +421,45 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
 
         // Halve W_ag and W_bg in place (exact in bf16): the MMAs then yield g / 2 for the tanh.
         bool ok = warp_wait(wbar, 0, abort_flag, ctl, SITE_PRO | 11, 0);
-        if (ok) {
+        if (ok && kVec) {
+            // Fold the input LayerNorm's affine into the projections, once per CTA:
+            // W'[n][k] = W[n][k] gamma[k] (bf16, in place; the gate rows also halved) and
+            // b'[n] = b[n] + sum_k W[n][k] beta[k] (halved for the gate rows) into pbias.
+            // Thread T owns stacked rows T and T + 256 (weight w = row / 128); it visits the 16
+            // chunks of a row starting at chunk (lane + j) & 7, so the lanes of a quarter
+            // warp touch different banks.
+#pragma unroll 1
+            for (int rr = 0; rr < 2; ++rr) {
+                const int R = warp * 32 + lane + 256 * rr, w = R >> 7, n = R & 127;
+                const float gscale = (w & 1) ? 0.5f : 1.f;
+                float acc = 0.f;
+#pragma unroll 1
+                for (int kh = 0; kh < 2; ++kh) {
+                    uint8_t *rowp = wsm + kh * W_HALF + w * 128 * 128 + n * 128;
+#pragma unroll 1
+                    for (int j = 0; j < 8; ++j) {
+                        const int pch = (j + lane) & 7, k0 = kh * 64 + 8 * (pch ^ (n & 7));
+                        uint4 *w4 = reinterpret_cast<uint4 *>(rowp + pch * 16);
+                        uint4 u = *w4;
+                        uint32_t *pw = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 wv = unpack_bf16x2(pw[e]);
+                            const int k = k0 + 2 * e;
+                            const float2 gm = args.ln_w ? ld_pair_bf16(args.ln_w, k) : make_float2(1.f, 1.f);
+                            const float2 bt = args.ln_b ? ld_pair_bf16(args.ln_b, k) : make_float2(0.f, 0.f);
+                            acc = fmaf(wv.x, bt.x, fmaf(wv.y, bt.y, acc));
+                            pw[e] = pack_bf16x2(wv.x * gm.x * gscale, wv.y * gm.y * gscale);
+                        }
+                        *w4 = u;
+                    }
+                }
+                const __nv_bfloat16 *bsrc = w == 0 ? args.b_a : w == 1 ? args.b_ag : w == 2 ? args.b_b : args.b_bg;
+                const float bb = (bsrc ? __bfloat162float(bsrc[n]) : 0.f) + acc;
+                pbias[R] = __float2bfloat16_rn(bb * gscale);
+            }
+            fence_proxy_async_smem();  // read by the tensor core
+        } else if (ok) {
 #pragma unroll 1
             for (int k = warp * 32 + lane; k < 4 * 1024; k += WORKERS * 32) {  // 4 regions x 1024 uint4
                 const int region = k >> 10;  // (K half, weight) = (0, ag), (0, bg), (1, ag), (1, bg)
@@ -437,6 +480,8 @@ __global__ void __launch_bounds__(pro::THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(wprep);
+        // Every worker's b' (kVec) is written before its arrival; the gating reads all of it.
+        if (kVec) ok = ok && warp_wait(wprep, 0, abort_flag, ctl, SITE_PRO | 14, 0);
         for (int lt = 0; ok && lt < n_local; ++lt) {
             int i, j0;
             tile_coords(lt, i, j0);
