@@ -5,15 +5,18 @@
 // the final reduction of the weight gradients.
 //
 // These are the elementwise and per-cell steps of the backward; its GEMMs run
-// on the tcgen05 pair kernel (contract_tc.cu). The per-cell kernels walk 64-cell tiles with 8 warps of
-// 8 cells; lane l owns channels l, l + 32, l + 64 and l + 96, so shared-memory
-// tiles are read without bank conflicts. Every kernel issues all global loads
-// for 4 cells (read-only path) before it computes and stores, so each warp
-// keeps several cells' loads in flight. Channel-major operands ([128][N][ld])
-// move as 16-byte vectors of 8 cells and are transposed through a
-// [64 cells][129] fp32 shared tile. Per-channel gradient sums are kept per
-// lane, reduced over the block at the end and added with one atomic per
-// channel and block. Grids are one wave of resident blocks.
+// on the tcgen05 pair kernel (contract_tc.cu). The per-cell kernels walk
+// 64-cell tiles with 8 warps of 8 cells. Half a warp serves one cell: lane q
+// of the half owns channels 8q .. 8q + 7 and moves them as one 16-byte vector,
+// so a warp reads or writes two whole 256-byte cell rows per instruction.
+// Every kernel issues all global loads of its warp's 8 cells (read-only path)
+// before it computes and stores. Channel-major operands ([128][N][ld]) move as
+// 16-byte vectors of 8 cells and are transposed through a [64 cells][128
+// channels] bf16 shared tile whose 16-byte chunks are XOR-swizzled by the
+// cell's group of eight, which keeps both the transposing accesses and the
+// per-cell vector accesses free of bank conflicts. Per-channel gradient sums
+// are kept per lane, reduced over the block at the end and added with one
+// atomic per channel and block. Grids are one wave of resident blocks.
 #include "kernels.h"
 
 namespace trimul {
@@ -24,24 +27,31 @@ typedef __nv_bfloat16 bf;
 constexpr int kTile = 64;               // cells per tile
 constexpr int kWarps = 8;
 constexpr int kCellsPerWarp = kTile / kWarps;
-constexpr int kU = 4;                   // cells whose loads a warp issues together
+constexpr int kPairs = kCellsPerWarp / 2;    // cell pairs per warp and tile (one cell per half warp)
 constexpr int kThreads = kWarps * 32;
-constexpr int kPitch = kC + 1;          // fp32 tile row: 128 channels + 1 pad word
-constexpr int kCPL = kC / 32;           // channels per lane
-constexpr size_t kTileBytes = (size_t)kTile * kPitch * sizeof(float);
+constexpr int kChunks = kC / 8;         // 16-byte chunks of a cell row = lanes per cell
+constexpr size_t kTileBytes = (size_t)kTile * kC * sizeof(bf);
 constexpr size_t kRedBytes = (size_t)kWarps * kC * sizeof(float);
-constexpr int kVecPerTile = kC * (kTile / 8);        // 16-byte vectors of 8 cells in a bf16 tile
+constexpr int kVecPerTile = kC * (kTile / 8);        // 16-byte vectors of 8 cells in a channel-major tile
 constexpr int kVecPerThread = kVecPerTile / kThreads;
 constexpr size_t kP = (size_t)kProjBlocks * kC;      // row length of P and D
 
-__device__ __forceinline__ float ldbf(const bf *p, size_t i, float dflt) {
-    return p ? __bfloat162float(__ldg(p + i)) : dflt;
-}
-__device__ __forceinline__ float ld(const bf *p) { return __bfloat162float(__ldg(p)); }
+static_assert(kChunks == 16 && kCellsPerWarp == 8, "half a warp per 128-channel cell, two cells per warp step");
 
-__device__ __forceinline__ float warp_sum(float v) {
+__device__ __forceinline__ float ld(const bf *p) { return __bfloat162float(__ldg(p)); }
+__device__ __forceinline__ uint4 ldg16(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+__device__ __forceinline__ void st16(void *p, const uint4 &v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+// Eight per-channel parameters c0 .. c0 + 7 (dflt for a null pointer).
+__device__ __forceinline__ void ld8(const bf *p, int c0, float dflt, float f[8]) {
 #pragma unroll
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int t = 0; t < 8; ++t) f[t] = p ? ld(p + c0 + t) : dflt;
+}
+
+// Sum over the 16 lanes of this half warp (one cell).
+__device__ __forceinline__ float half_sum(float v) {
+#pragma unroll
+    for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
@@ -57,13 +67,36 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float f[8]) {
     }
 }
 
+__device__ __forceinline__ float2 bf2f(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
+}
+__device__ __forceinline__ uint32_t f2bf(float x, float y) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint4 pack8(const float f[8]) {
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(f[2 * t], f[2 * t + 1]);
+    return u;
+}
+
+// Index (in 16-byte chunks) of channels 8q .. 8q + 7 of cell jj in a bf16 tile.
+// The XOR with the cell's group of eight spreads a transposing access (8
+// consecutive cells of one channel in a vector, 8 vectors per warp) and a
+// quarter warp's per-cell access (8 chunks of one cell) over all 32 banks.
+__device__ __forceinline__ int chunk_at(int jj, int q) { return jj * kChunks + (q ^ ((jj >> 3) & 7)); }
+
 // Tiles of kA channel-major bf16 arrays, row segment (i, j0 .. j0 + 63), into
-// tile[a][cell][channel]. A vector of 8 cells that starts inside the row ends
-// within the row's pitch (ld is a multiple of 8), so it never leaves the row;
-// cells past N hold whatever the padding holds and are not used.
+// tile[a] (bf16 [cell][channel], swizzled). A vector of 8 cells that starts
+// inside the row ends within the row's pitch (ld is a multiple of 8), so it
+// never leaves the row; cells past N hold whatever the padding holds and are
+// not used.
 template <int kA>
 __device__ __forceinline__ void load_cm(const bf *const (&src)[kA], int N, size_t ld, int i, int j0,
-                                        float *const (&tile)[kA]) {
+                                        uint4 *const (&tile)[kA]) {
     const size_t cs = (size_t)N * ld;
     uint4 v[kA][kVecPerThread];
 #pragma unroll
@@ -71,47 +104,54 @@ __device__ __forceinline__ void load_cm(const bf *const (&src)[kA], int N, size_
 #pragma unroll
         for (int k = 0; k < kVecPerThread; ++k) {
             const int e = threadIdx.x + k * kThreads, c = e >> 3, j = j0 + 8 * (e & 7);
-            v[a][k] = j < N ? __ldg(reinterpret_cast<const uint4 *>(src[a] + c * cs + (size_t)i * ld + j))
-                            : make_uint4(0, 0, 0, 0);
+            v[a][k] = j < N ? ldg16(src[a] + c * cs + (size_t)i * ld + j) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-    for (int a = 0; a < kA; ++a)
+    for (int a = 0; a < kA; ++a) {
+        unsigned short *tb = reinterpret_cast<unsigned short *>(tile[a]);
 #pragma unroll
         for (int k = 0; k < kVecPerThread; ++k) {
             const int e = threadIdx.x + k * kThreads, c = e >> 3, jj = 8 * (e & 7);
-            float f[8];
-            unpack8(v[a][k], f);
+            const uint32_t w[4] = {v[a][k].x, v[a][k].y, v[a][k].z, v[a][k].w};
 #pragma unroll
-            for (int t = 0; t < 8; ++t) tile[a][(jj + t) * kPitch + c] = f[t];
+            for (int t = 0; t < 8; ++t)
+                tb[chunk_at(jj + t, c >> 3) * 8 + (c & 7)] = (unsigned short)(w[t >> 1] >> (16 * (t & 1)));
         }
+    }
 }
 
-// tile[cell][channel] back to a channel-major bf16 row segment in vectors of 8
-// cells; a vector that starts below N also writes the padding cells after N,
-// which the tile holds as 0.
-__device__ __forceinline__ void store_cm(bf *dst, int N, size_t ld, int i, int j0, const float *tile) {
+// A bf16 tile back to a channel-major row segment in vectors of 8 cells; a
+// vector that starts below N also writes the padding cells after N, which the
+// tile holds as 0.
+__device__ __forceinline__ void store_cm(bf *dst, int N, size_t ld, int i, int j0, const uint4 *tile) {
     const size_t cs = (size_t)N * ld;
+    const unsigned short *tb = reinterpret_cast<const unsigned short *>(tile);
 #pragma unroll
     for (int k = 0; k < kVecPerThread; ++k) {
         const int e = threadIdx.x + k * kThreads, c = e >> 3, jj = 8 * (e & 7), j = j0 + jj;
         if (j >= N) continue;
-        uint4 u;
-        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+        uint32_t w[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-            h[t] = __floats2bfloat162_rn(tile[(jj + 2 * t) * kPitch + c], tile[(jj + 2 * t + 1) * kPitch + c]);
-        *reinterpret_cast<uint4 *>(dst + c * cs + (size_t)i * ld + j) = u;
+            w[t] = (uint32_t)tb[chunk_at(jj + 2 * t, c >> 3) * 8 + (c & 7)] |
+                   ((uint32_t)tb[chunk_at(jj + 2 * t + 1, c >> 3) * 8 + (c & 7)] << 16);
+        st16(dst + c * cs + (size_t)i * ld + j, make_uint4(w[0], w[1], w[2], w[3]));
     }
 }
 
-// Adds the block's per-lane channel sums acc[k][r] (channel lane + 32 r) to dst[k][128].
+// Adds the block's per-lane channel sums acc[k][t] (channel 8 (lane % 16) + t)
+// to dst[k][128].
 template <int K>
-__device__ void flush_sums(const float (&acc)[K][kCPL], float *const (&dst)[K], float *red) {
+__device__ void flush_sums(float (&acc)[K][8], float *const (&dst)[K], float *red) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int k = 0; k < K; ++k) {
-        __syncthreads();
 #pragma unroll
-        for (int r = 0; r < kCPL; ++r) red[warp * kC + lane + 32 * r] = acc[k][r];
+    for (int k = 0; k < K; ++k) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[k][t] += __shfl_xor_sync(0xffffffffu, acc[k][t], 16);
+        __syncthreads();
+        if (lane < kChunks)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) red[warp * kC + 8 * lane + t] = acc[k][t];
         __syncthreads();
         if (threadIdx.x < kC && dst[k]) {
             float s = 0.f;
@@ -131,59 +171,57 @@ __device__ __forceinline__ TileIdx tile_of(long long t, int jt) {
     return x;
 }
 
+// The tile cell of pair u for this half warp.
+__device__ __forceinline__ int cell_of(int warp, int u) { return warp * kCellsPerWarp + 2 * u + (threadIdx.x >> 4 & 1); }
+
 // ---- LayerNorm forward (recomputed statistics and normalised operand) ----------
 
 template <bool kCM>
-__global__ void __launch_bounds__(kThreads) ln_fwd_kernel(LnFwdArgs a) {
-    extern __shared__ float tile[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kThreads, 2) ln_fwd_kernel(LnFwdArgs a) {
+    extern __shared__ uint4 tile[];
+    const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kTile - 1) / kTile;
     const long long tiles = (long long)a.N * jt;
-    float gm[kCPL], bt[kCPL];
-#pragma unroll
-    for (int r = 0; r < kCPL; ++r) {
-        gm[r] = ldbf(a.gamma, lane + 32 * r, 1.f);
-        bt[r] = ldbf(a.beta, lane + 32 * r, 0.f);
-    }
+    float gm[8], bt[8];
+    ld8(a.gamma, c0, 1.f, gm);
+    ld8(a.beta, c0, 0.f, bt);
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
         const TileIdx ti = tile_of(t, jt);
         if (kCM) {
             const bf *src[1] = {a.src};
-            float *const tl[1] = {tile};
+            uint4 *const tl[1] = {tile};
             __syncthreads();
             load_cm<1>(src, a.N, a.ld, ti.i, ti.j0, tl);
             __syncthreads();
         }
-        for (int q0 = 0; q0 < kCellsPerWarp; q0 += kU) {
-            float v[kU][kCPL];
+        uint4 raw[kPairs];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = min(ti.j0 + jj, a.N - 1);
-                const size_t m = (size_t)ti.i * a.N + j;
+        for (int u = 0; u < kPairs; ++u) {
+            const int jj = cell_of(warp, u), j = min(ti.j0 + jj, a.N - 1);
+            const size_t m = (size_t)ti.i * a.N + j;
+            raw[u] = kCM ? tile[chunk_at(jj, q)] : ldg16(a.src + m * kC + c0);
+        }
+        // Both halves take every shuffle: a cell past N computes on a clamped copy and stores nothing.
 #pragma unroll
-                for (int r = 0; r < kCPL; ++r)
-                    v[u][r] = kCM ? tile[jj * kPitch + lane + 32 * r] : ld(a.src + m * kC + lane + 32 * r);
+        for (int u = 0; u < kPairs; ++u) {
+            const int j = ti.j0 + cell_of(warp, u);
+            const size_t m = (size_t)ti.i * a.N + j;
+            float v[8], s = 0.f, ss = 0.f;
+            unpack8(raw[u], v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) s += v[k];
+            const float mu = half_sum(s) * (1.f / kC);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                v[k] -= mu;
+                ss += v[k] * v[k];
             }
+            const float rs = rsqrtf(half_sum(ss) * (1.f / kC) + a.eps);
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = ti.j0 + jj;
-                if (j >= a.N) continue;
-                const size_t m = (size_t)ti.i * a.N + j;
-                float s = 0.f;
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r) s += v[u][r];
-                const float mu = warp_sum(s) * (1.f / kC);
-                float ss = 0.f;
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    v[u][r] -= mu;
-                    ss += v[u][r] * v[u][r];
-                }
-                const float rs = rsqrtf(warp_sum(ss) * (1.f / kC) + a.eps);
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r)
-                    a.out[m * kC + lane + 32 * r] = __float2bfloat16_rn(v[u][r] * rs * gm[r] + bt[r]);
-                if (lane == 0) a.stats[m] = make_float2(mu, rs);
+            for (int k = 0; k < 8; ++k) v[k] = v[k] * rs * gm[k] + bt[k];
+            if (j < a.N) {
+                st16(a.out + m * kC + c0, pack8(v));
+                if (q == 0) a.stats[m] = make_float2(mu, rs);
             }
         }
     }
@@ -192,74 +230,65 @@ __global__ void __launch_bounds__(kThreads) ln_fwd_kernel(LnFwdArgs a) {
 // ---- LayerNorm adjoint ------------------------------------------------------------
 
 template <bool kCM>
-__global__ void __launch_bounds__(kThreads) ln_bwd_kernel(LnBwdArgs a) {
-    extern __shared__ float smem[];
-    float *tile = smem;
-    float *red = smem + (kCM ? kTile * kPitch : 0);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kThreads, 2) ln_bwd_kernel(LnBwdArgs a) {
+    extern __shared__ uint4 smem4[];
+    uint4 *tile = smem4;
+    float *red = reinterpret_cast<float *>(smem4 + (kCM ? kTile * kChunks : 0));
+    const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kTile - 1) / kTile;
     const long long tiles = (long long)a.N * jt;
-    float gm[kCPL];
-    float acc[2][kCPL] = {};
-#pragma unroll
-    for (int r = 0; r < kCPL; ++r) gm[r] = ldbf(a.gamma, lane + 32 * r, 1.f);
+    float gm[8];
+    float acc[2][8] = {};
+    ld8(a.gamma, c0, 1.f, gm);
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
         const TileIdx ti = tile_of(t, jt);
         if (kCM) {
             const bf *src[1] = {a.src};
-            float *const tl[1] = {tile};
+            uint4 *const tl[1] = {tile};
             __syncthreads();
             load_cm<1>(src, a.N, a.ld, ti.i, ti.j0, tl);
             __syncthreads();
         }
-        for (int q0 = 0; q0 < kCellsPerWarp; q0 += kU) {
-            float v[kU][kCPL], g[kU][kCPL];
-            float2 st[kU];
+        uint4 raw[kPairs];
+        float4 g[kPairs][2];
+        float2 st[kPairs];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = min(ti.j0 + jj, a.N - 1);
-                const size_t m = (size_t)ti.i * a.N + j;
-                st[u] = __ldg(a.stats + m);
+        for (int u = 0; u < kPairs; ++u) {
+            const int jj = cell_of(warp, u), j = min(ti.j0 + jj, a.N - 1);
+            const size_t m = (size_t)ti.i * a.N + j;
+            st[u] = __ldg(a.stats + m);
+            raw[u] = kCM ? tile[chunk_at(jj, q)] : ldg16(a.src + m * kC + c0);
+            g[u][0] = __ldg(reinterpret_cast<const float4 *>(a.dh + m * kC + c0));
+            g[u][1] = __ldg(reinterpret_cast<const float4 *>(a.dh + m * kC + c0 + 4));
+        }
 #pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    const int c = lane + 32 * r;
-                    v[u][r] = kCM ? tile[jj * kPitch + c] : ld(a.src + m * kC + c);
-                    g[u][r] = __ldg(a.dh + m * kC + c);
+        for (int u = 0; u < kPairs; ++u) {
+            const int jj = cell_of(warp, u), j = ti.j0 + jj;
+            const bool valid = j < a.N;
+            const size_t m = (size_t)ti.i * a.N + j;
+            const float gg[8] = {g[u][0].x, g[u][0].y, g[u][0].z, g[u][0].w,
+                                 g[u][1].x, g[u][1].y, g[u][1].z, g[u][1].w};
+            float v[8], n[8], dn[8], s1 = 0.f, s2 = 0.f;
+            unpack8(raw[u], v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                n[k] = (v[k] - st[u].x) * st[u].y;
+                dn[k] = gg[k] * gm[k];
+                s1 += dn[k];
+                s2 += dn[k] * n[k];
+                if (valid) {
+                    acc[0][k] += gg[k] * n[k];
+                    acc[1][k] += gg[k];
                 }
             }
+            s1 = half_sum(s1) * (1.f / kC);
+            s2 = half_sum(s2) * (1.f / kC);
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = ti.j0 + jj;
-                if (j >= a.N) {
-                    // Padding cell, stored with its vector: zero.
-                    if (kCM)
-#pragma unroll
-                        for (int r = 0; r < kCPL; ++r) tile[jj * kPitch + lane + 32 * r] = 0.f;
-                    continue;
-                }
-                const size_t m = (size_t)ti.i * a.N + j;
-                float n[kCPL], dn[kCPL], s1 = 0.f, s2 = 0.f;
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    n[r] = (v[u][r] - st[u].x) * st[u].y;
-                    dn[r] = g[u][r] * gm[r];
-                    s1 += dn[r];
-                    s2 += dn[r] * n[r];
-                    acc[0][r] += g[u][r] * n[r];
-                    acc[1][r] += g[u][r];
-                }
-                s1 = warp_sum(s1) * (1.f / kC);
-                s2 = warp_sum(s2) * (1.f / kC);
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    const int c = lane + 32 * r;
-                    const float dv = st[u].y * (dn[r] - s1 - n[r] * s2);
-                    if (kCM)
-                        tile[jj * kPitch + c] = dv;  // this warp's own cell row: no other warp touches it
-                    else
-                        a.dsrc[m * kC + c] = __float2bfloat16_rn(dv);
-                }
-            }
+            for (int k = 0; k < 8; ++k) v[k] = st[u].y * (dn[k] - s1 - n[k] * s2);
+            if (kCM)  // this half warp's own cell row: no other thread touches it; padding cells store 0
+                tile[chunk_at(jj, q)] = valid ? pack8(v) : make_uint4(0, 0, 0, 0);
+            else if (valid)
+                st16(a.dsrc + m * kC + c0, pack8(v));
         }
         if (kCM) {
             __syncthreads();
@@ -272,46 +301,41 @@ __global__ void __launch_bounds__(kThreads) ln_bwd_kernel(LnBwdArgs a) {
 
 // ---- output gate adjoint -------------------------------------------------------------
 
-__global__ void __launch_bounds__(kThreads) gate_bwd_kernel(GateBwdArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) gate_bwd_kernel(GateBwdArgs a) {
     __shared__ float red[kWarps * kC];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float bg[kCPL], bo[kCPL];
-    float acc[2][kCPL] = {};
-#pragma unroll
-    for (int r = 0; r < kCPL; ++r) {
-        bg[r] = ldbf(a.b_g, lane + 32 * r, 0.f);
-        bo[r] = ldbf(a.b_o, lane + 32 * r, 0.f);
-    }
+    const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
+    float bg[8], bo[8];
+    float acc[2][8] = {};
+    ld8(a.b_g, c0, 0.f, bg);
+    ld8(a.b_o, c0, 0.f, bo);
     const long long tiles = (a.cells + kTile - 1) / kTile;
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
-        for (int q0 = 0; q0 < kCellsPerWarp; q0 += kU) {
-            float pg[kU][kCPL], y[kU][kCPL], d[kU][kCPL];
+        uint4 pg[kPairs], y[kPairs], d[kPairs];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const long long m = min(t * kTile + warp * kCellsPerWarp + q0 + u, a.cells - 1);
+        for (int u = 0; u < kPairs; ++u) {
+            const long long m = min(t * kTile + cell_of(warp, u), a.cells - 1);
+            pg[u] = ldg16(a.P + m * kP + P_G * kC + c0);
+            y[u] = ldg16(a.Y + m * kC + c0);
+            d[u] = ldg16(a.dout + m * kC + c0);
+        }
 #pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    const int c = lane + 32 * r;
-                    pg[u][r] = ld(a.P + m * kP + P_G * kC + c);
-                    y[u][r] = ld(a.Y + m * kC + c);
-                    d[u][r] = ld(a.dout + m * kC + c);
-                }
+        for (int u = 0; u < kPairs; ++u) {
+            const long long m = t * kTile + cell_of(warp, u);
+            if (m >= a.cells) continue;
+            float fp[8], fy[8], fd[8], dy[8], dpg[8];
+            unpack8(pg[u], fp);
+            unpack8(y[u], fy);
+            unpack8(d[u], fd);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float gt = sigmoid(fp[k] + bg[k]), yy = fy[k] + bo[k];
+                dy[k] = fd[k] * gt;
+                dpg[k] = fd[k] * yy * gt * (1.f - gt);
+                acc[0][k] += dpg[k];
+                acc[1][k] += dy[k];
             }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const long long m = t * kTile + warp * kCellsPerWarp + q0 + u;
-                if (m >= a.cells) continue;
-#pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    const int c = lane + 32 * r;
-                    const float g = sigmoid(pg[u][r] + bg[r]), yy = y[u][r] + bo[r];
-                    const float dy = d[u][r] * g, dpg = d[u][r] * yy * g * (1.f - g);
-                    a.dy[m * kC + c] = __float2bfloat16_rn(dy);
-                    a.D[m * kP + P_G * kC + c] = __float2bfloat16_rn(dpg);
-                    acc[0][r] += dpg;
-                    acc[1][r] += dy;
-                }
-            }
+            st16(a.dy + m * kC + c0, pack8(dy));
+            st16(a.D + m * kP + P_G * kC + c0, pack8(dpg));
         }
     }
     float *const dst[2] = {a.db_g, a.db_o};
@@ -320,63 +344,87 @@ __global__ void __launch_bounds__(kThreads) gate_bwd_kernel(GateBwdArgs a) {
 
 // ---- input gates and mask adjoint --------------------------------------------------------
 
-__global__ void __launch_bounds__(kThreads) proj_bwd_kernel(ProjBwdArgs a) {
-    extern __shared__ float smem[];
-    float *tA = smem, *tB = smem + kTile * kPitch, *red = smem + 2 * kTile * kPitch;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+constexpr int kProjPairs = 1;  // cell pairs whose P loads a warp issues together
+
+__global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
+    extern __shared__ uint4 smem4[];
+    uint4 *tA = smem4, *tB = smem4 + kTile * kChunks;
+    float *red = reinterpret_cast<float *>(smem4 + 2 * kTile * kChunks);
+    const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kTile - 1) / kTile;
     const long long tiles = (long long)a.N * jt;
-    float bias[4][kCPL];
-    float acc[4][kCPL] = {};
+    // The four bias vectors stay bf16 (exact), two channels to a register.
+    __nv_bfloat162 bias[4][4];
+    float acc[4][8] = {};
     const bf *bp[4] = {a.b_a, a.b_ag, a.b_b, a.b_bg};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int r = 0; r < kCPL; ++r) bias[k][r] = ldbf(bp[k], lane + 32 * r, 0.f);
+        for (int t = 0; t < 4; ++t)
+            bias[k][t] = bp[k] ? __halves2bfloat162(bp[k][c0 + 2 * t], bp[k][c0 + 2 * t + 1])
+                               : __floats2bfloat162_rn(0.f, 0.f);
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
         const TileIdx ti = tile_of(t, jt);
         {
             const bf *src[2] = {a.dA, a.dB};
-            float *const tl[2] = {tA, tB};
+            uint4 *const tl[2] = {tA, tB};
             __syncthreads();
             load_cm<2>(src, a.N, a.ld, ti.i, ti.j0, tl);
             __syncthreads();
         }
-        for (int q0 = 0; q0 < kCellsPerWarp; q0 += kU) {
-            float p[kU][4][kCPL], mk[kU];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = min(ti.j0 + jj, a.N - 1);
+        for (int u0 = 0; u0 < kPairs; u0 += kProjPairs) {
+            uint4 p[kProjPairs][4];
+            float mk[kProjPairs];
+#pragma unroll
+            for (int u = 0; u < kProjPairs; ++u) {
+                const int j = min(ti.j0 + cell_of(warp, u0 + u), a.N - 1);
                 const size_t m = (size_t)ti.i * a.N + j;
-                mk[u] = ldbf(a.mask, m, 1.f);
+                mk[u] = a.mask ? ld(a.mask + m) : 1.f;
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-#pragma unroll
-                    for (int r = 0; r < kCPL; ++r) p[u][k][r] = ld(a.P + m * kP + (P_A + k) * kC + lane + 32 * r);
+                for (int k = 0; k < 4; ++k) p[u][k] = ldg16(a.P + m * kP + (P_A + k) * kC + c0);
             }
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int jj = warp * kCellsPerWarp + q0 + u, j = ti.j0 + jj;
+            for (int u = 0; u < kProjPairs; ++u) {
+                const int jj = cell_of(warp, u0 + u), j = ti.j0 + jj;
                 if (j >= a.N) continue;
                 const size_t m = (size_t)ti.i * a.N + j;
-                bf *d = a.D + m * kP;
+                // Two channels at a time: the four outputs of channels c0 + 2t, c0 + 2t + 1
+                // are packed as they are made, which keeps few values live.
+                const uint4 ta = tA[chunk_at(jj, q)], tb = tB[chunk_at(jj, q)];
+                const uint32_t wa[4] = {ta.x, ta.y, ta.z, ta.w}, wb[4] = {tb.x, tb.y, tb.z, tb.w};
+                const uint32_t w0[4] = {p[u][0].x, p[u][0].y, p[u][0].z, p[u][0].w};
+                const uint32_t w1[4] = {p[u][1].x, p[u][1].y, p[u][1].z, p[u][1].w};
+                const uint32_t w2[4] = {p[u][2].x, p[u][2].y, p[u][2].z, p[u][2].w};
+                const uint32_t w3[4] = {p[u][3].x, p[u][3].y, p[u][3].z, p[u][3].w};
+                uint32_t o[4][4];
 #pragma unroll
-                for (int r = 0; r < kCPL; ++r) {
-                    const int c = lane + 32 * r;
-                    const float da = tA[jj * kPitch + c] * mk[u], db = tB[jj * kPitch + c] * mk[u];
-                    const float pa = p[u][0][r] + bias[0][r], pb = p[u][2][r] + bias[2][r];
-                    const float sa = sigmoid(p[u][1][r] + bias[1][r]), sb = sigmoid(p[u][3][r] + bias[3][r]);
-                    const float g0 = da * sa, g1 = da * pa * sa * (1.f - sa);
-                    const float g2 = db * sb, g3 = db * pb * sb * (1.f - sb);
-                    d[P_A * kC + c] = __float2bfloat16_rn(g0);
-                    d[P_AG * kC + c] = __float2bfloat16_rn(g1);
-                    d[P_B * kC + c] = __float2bfloat16_rn(g2);
-                    d[P_BG * kC + c] = __float2bfloat16_rn(g3);
-                    acc[0][r] += g0;
-                    acc[1][r] += g1;
-                    acc[2][r] += g2;
-                    acc[3][r] += g3;
+                for (int t = 0; t < 4; ++t) {
+                    const float2 da = bf2f(wa[t]), db = bf2f(wb[t]);
+                    const float2 b0 = __bfloat1622float2(bias[0][t]), b1 = __bfloat1622float2(bias[1][t]);
+                    const float2 b2 = __bfloat1622float2(bias[2][t]), b3 = __bfloat1622float2(bias[3][t]);
+                    const float2 pa = bf2f(w0[t]), pag = bf2f(w1[t]), pb = bf2f(w2[t]), pbg = bf2f(w3[t]);
+                    float g[4][2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float dah = (h ? da.y : da.x) * mk[u], dbh = (h ? db.y : db.x) * mk[u];
+                        const float sa = sigmoid((h ? pag.y : pag.x) + (h ? b1.y : b1.x));
+                        const float sb = sigmoid((h ? pbg.y : pbg.x) + (h ? b3.y : b3.x));
+                        g[0][h] = dah * sa;
+                        g[1][h] = dah * ((h ? pa.y : pa.x) + (h ? b0.y : b0.x)) * sa * (1.f - sa);
+                        g[2][h] = dbh * sb;
+                        g[3][h] = dbh * ((h ? pb.y : pb.x) + (h ? b2.y : b2.x)) * sb * (1.f - sb);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        acc[k][2 * t] += g[k][0];
+                        acc[k][2 * t + 1] += g[k][1];
+                        o[k][t] = f2bf(g[k][0], g[k][1]);
+                    }
                 }
+                bf *d = a.D + m * kP + c0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) st16(d + (P_A + k) * kC, make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]));
             }
         }
     }
