@@ -18,6 +18,7 @@
 // are kept per lane, reduced over the block at the end and added with one
 // atomic per channel and block. Grids are one wave of resident blocks.
 #include "kernels.h"
+#include "tile_ops.cuh"
 
 namespace trimul {
 namespace {
@@ -55,7 +56,9 @@ __device__ __forceinline__ float half_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ float sigmoid(float t) { return 1.f / (1.f + __expf(-t)); }
+// sigma(t) = (1 + tanh(t / 2)) / 2: one MUFU operation (tanh.approx, relative
+// error about 2^-11, far below the bf16 rounding of every output it feeds).
+__device__ __forceinline__ float sigmoid(float t) { return fmaf(0.5f, tanh_approx(0.5f * t), 0.5f); }
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float f[8]) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -343,15 +346,75 @@ __global__ void __launch_bounds__(kThreads, 2) gate_bwd_kernel(GateBwdArgs a) {
 }
 
 // ---- input gates and mask adjoint --------------------------------------------------------
+//
+// The largest per-cell pass (about 2.5 KB per cell). Its inputs move by
+// asynchronous 16-byte copies (cp.async, no registers held) into a two-stage
+// shared-memory ring, one tile ahead of the compute, on 32-cell tiles: a stage
+// holds P's blocks P_A .. P_BG of the tile's cells ([cell][block][channel],
+// 32 KB) and the channel-major dA and dB row segments as they lie in memory
+// ([array][channel][4 vectors of 8 cells], 16 KB), which are transposed into
+// swizzled cell-major tiles before the compute. Two blocks of 256 threads per
+// SM, so that one block computes while the other waits at its barriers.
 
-constexpr int kProjPairs = 1;  // cell pairs whose P loads a warp issues together
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
+constexpr int kPT = 32;                                  // cells per tile of this pass
+constexpr int kProjPChunks = kPT * 4 * kChunks;          // P_A .. P_BG of one tile, 16-byte chunks
+constexpr int kProjRChunks = 2 * kC * (kPT / 8);         // raw dA, dB row segments
+constexpr int kProjStage = kProjPChunks + kProjRChunks;  // in 16-byte chunks
+constexpr int kProjT = kPT * kChunks;                    // one transposed tile, in chunks
+constexpr size_t kProjSmem = (size_t)(2 * kProjStage + 2 * kProjT) * 16 + 2 * kPT * sizeof(float);
+static_assert(kProjPChunks % kThreads == 0 && kProjRChunks % kThreads == 0, "copies split evenly");
+static_assert(2 * kProjT * 16 >= kRedBytes, "block sums reuse the transposed tiles");
+static_assert(2 * (kProjSmem + 1024) <= 228 * 1024, "two blocks per SM");
+
+struct ProjTile {
+    int i, j0;
+    bool live;
+};
+__device__ __forceinline__ ProjTile proj_tile(long long t, long long tiles, int jt) {
+    ProjTile p;
+    p.live = t < tiles;
+    p.i = p.live ? (int)(t / jt) : 0;
+    p.j0 = p.live ? (int)(t % jt) * kPT : 0;
+    return p;
+}
+
+// Issues the copies of one tile into stage `st` (none for a dead tile; the
+// caller commits a group either way, so that group counting stays uniform).
+// Chunks of cells past N are zero-filled without a read.
+__device__ __forceinline__ void proj_issue(const ProjBwdArgs &a, const ProjTile &ti, uint4 *st) {
+    if (!ti.live) return;
+    const size_t cs = (size_t)a.N * a.ld;
+#pragma unroll
+    for (int r = 0; r < kProjPChunks / kThreads; ++r) {
+        const int x = threadIdx.x + r * kThreads, jj = x >> 6, k = (x >> 4) & 3, q = x & 15;
+        const bool ok = ti.j0 + jj < a.N;
+        const size_t m = (size_t)ti.i * a.N + (ok ? ti.j0 + jj : 0);
+        cp_async16(st + x, a.P + m * kP + (P_A + k) * kC + 8 * q, ok);
+    }
+#pragma unroll
+    for (int r = 0; r < kProjRChunks / kThreads; ++r) {
+        const int y = threadIdx.x + r * kThreads, arr = y / (kC * kPT / 8), c = (y >> 2) & (kC - 1), g = y & 3;
+        const bool ok = ti.j0 + 8 * g < a.N;
+        const bf *src = (arr ? a.dB : a.dA) + c * cs + (size_t)ti.i * a.ld + (ok ? ti.j0 + 8 * g : 0);
+        cp_async16(st + kProjPChunks + y, src, ok);
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
     extern __shared__ uint4 smem4[];
-    uint4 *tA = smem4, *tB = smem4 + kTile * kChunks;
-    float *red = reinterpret_cast<float *>(smem4 + 2 * kTile * kChunks);
+    uint4 *const stage0 = smem4;
+    uint4 *tA = smem4 + 2 * kProjStage, *tB = tA + kProjT;
+    float *msk = reinterpret_cast<float *>(tB + kProjT);  // [2][kPT] mask per stage
+    float *red = reinterpret_cast<float *>(tA);           // after the last tile
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
-    const int jt = (a.N + kTile - 1) / kTile;
+    const int jt = (a.N + kPT - 1) / kPT;
     const long long tiles = (long long)a.N * jt;
     // The four bias vectors stay bf16 (exact), two channels to a register.
     __nv_bfloat162 bias[4][4];
@@ -363,71 +426,89 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
         for (int t = 0; t < 4; ++t)
             bias[k][t] = bp[k] ? __halves2bfloat162(bp[k][c0 + 2 * t], bp[k][c0 + 2 * t + 1])
                                : __floats2bfloat162_rn(0.f, 0.f);
-    for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const TileIdx ti = tile_of(t, jt);
+    const long long t0 = blockIdx.x, dt = gridDim.x;
+    auto mask_of = [&](long long t) -> float {
+        const ProjTile ti = proj_tile(t, tiles, jt);
+        const int j = ti.j0 + (int)threadIdx.x;
+        return a.mask && ti.live && j < a.N ? ld(a.mask + (size_t)ti.i * a.N + j) : 1.f;
+    };
+    proj_issue(a, proj_tile(t0, tiles, jt), stage0);
+    cp_async_commit();
+    proj_issue(a, proj_tile(t0 + dt, tiles, jt), stage0 + kProjStage);
+    cp_async_commit();
+    if (threadIdx.x < kPT) msk[threadIdx.x] = mask_of(t0);
+    int s = 0;
+    for (long long t = t0; t < tiles; t += dt, s ^= 1) {
+        const ProjTile ti = proj_tile(t, tiles, jt);
+        uint4 *const st = stage0 + s * kProjStage;
+        asm volatile("cp.async.wait_group 1;\n" ::: "memory");  // this thread's copies of tile t landed
+        __syncthreads();  // everyone's have; tA, tB and the other mask slot are free
+        const float mnext = threadIdx.x < kPT ? mask_of(t + dt) : 1.f;
         {
-            const bf *src[2] = {a.dA, a.dB};
-            uint4 *const tl[2] = {tA, tB};
-            __syncthreads();
-            load_cm<2>(src, a.N, a.ld, ti.i, ti.j0, tl);
-            __syncthreads();
-        }
+            // Chunk (array, channel c, vector g) holds cells 8g .. 8g + 7 of channel c.
+            const uint4 *raw = st + kProjPChunks;
 #pragma unroll
-        for (int u0 = 0; u0 < kPairs; u0 += kProjPairs) {
-            uint4 p[kProjPairs][4];
-            float mk[kProjPairs];
+            for (int r = 0; r < kProjRChunks / kThreads; ++r) {
+                const int y = threadIdx.x + r * kThreads, arr = y / (kC * kPT / 8), c = (y >> 2) & (kC - 1);
+                const int jj = 8 * (y & 3);
+                const uint4 v = raw[y];
+                unsigned short *tb = reinterpret_cast<unsigned short *>(arr ? tB : tA);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int u = 0; u < kProjPairs; ++u) {
-                const int j = min(ti.j0 + cell_of(warp, u0 + u), a.N - 1);
-                const size_t m = (size_t)ti.i * a.N + j;
-                mk[u] = a.mask ? ld(a.mask + m) : 1.f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) p[u][k] = ldg16(a.P + m * kP + (P_A + k) * kC + c0);
+                for (int e = 0; e < 8; ++e)
+                    tb[chunk_at(jj + e, c >> 3) * 8 + (c & 7)] = (unsigned short)(w[e >> 1] >> (16 * (e & 1)));
             }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int u = 0; u < kPT / kWarps / 2; ++u) {
+            const int jj = warp * (kPT / kWarps) + 2 * u + (int)(threadIdx.x >> 4 & 1), j = ti.j0 + jj;
+            if (j >= a.N) continue;
+            const size_t m = (size_t)ti.i * a.N + j;
+            const float mk = msk[s * kPT + jj];
+            // Two channels at a time: the four outputs of channels c0 + 2e, c0 + 2e + 1
+            // are packed as they are made, which keeps few values live.
+            const uint4 ta = tA[chunk_at(jj, q)], tb = tB[chunk_at(jj, q)];
+            const uint4 p0 = st[(jj * 4 + 0) * kChunks + q], p1 = st[(jj * 4 + 1) * kChunks + q];
+            const uint4 p2 = st[(jj * 4 + 2) * kChunks + q], p3 = st[(jj * 4 + 3) * kChunks + q];
+            const uint32_t wa[4] = {ta.x, ta.y, ta.z, ta.w}, wb[4] = {tb.x, tb.y, tb.z, tb.w};
+            const uint32_t w0[4] = {p0.x, p0.y, p0.z, p0.w}, w1[4] = {p1.x, p1.y, p1.z, p1.w};
+            const uint32_t w2[4] = {p2.x, p2.y, p2.z, p2.w}, w3[4] = {p3.x, p3.y, p3.z, p3.w};
+            uint32_t o[4][4];
 #pragma unroll
-            for (int u = 0; u < kProjPairs; ++u) {
-                const int jj = cell_of(warp, u0 + u), j = ti.j0 + jj;
-                if (j >= a.N) continue;
-                const size_t m = (size_t)ti.i * a.N + j;
-                // Two channels at a time: the four outputs of channels c0 + 2t, c0 + 2t + 1
-                // are packed as they are made, which keeps few values live.
-                const uint4 ta = tA[chunk_at(jj, q)], tb = tB[chunk_at(jj, q)];
-                const uint32_t wa[4] = {ta.x, ta.y, ta.z, ta.w}, wb[4] = {tb.x, tb.y, tb.z, tb.w};
-                const uint32_t w0[4] = {p[u][0].x, p[u][0].y, p[u][0].z, p[u][0].w};
-                const uint32_t w1[4] = {p[u][1].x, p[u][1].y, p[u][1].z, p[u][1].w};
-                const uint32_t w2[4] = {p[u][2].x, p[u][2].y, p[u][2].z, p[u][2].w};
-                const uint32_t w3[4] = {p[u][3].x, p[u][3].y, p[u][3].z, p[u][3].w};
-                uint32_t o[4][4];
+            for (int e = 0; e < 4; ++e) {
+                const float2 da = bf2f(wa[e]), db = bf2f(wb[e]);
+                const float2 b0 = __bfloat1622float2(bias[0][e]), b1 = __bfloat1622float2(bias[1][e]);
+                const float2 b2 = __bfloat1622float2(bias[2][e]), b3 = __bfloat1622float2(bias[3][e]);
+                const float2 pa = bf2f(w0[e]), pag = bf2f(w1[e]), pb = bf2f(w2[e]), pbg = bf2f(w3[e]);
+                float g[4][2];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float2 da = bf2f(wa[t]), db = bf2f(wb[t]);
-                    const float2 b0 = __bfloat1622float2(bias[0][t]), b1 = __bfloat1622float2(bias[1][t]);
-                    const float2 b2 = __bfloat1622float2(bias[2][t]), b3 = __bfloat1622float2(bias[3][t]);
-                    const float2 pa = bf2f(w0[t]), pag = bf2f(w1[t]), pb = bf2f(w2[t]), pbg = bf2f(w3[t]);
-                    float g[4][2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float dah = (h ? da.y : da.x) * mk[u], dbh = (h ? db.y : db.x) * mk[u];
-                        const float sa = sigmoid((h ? pag.y : pag.x) + (h ? b1.y : b1.x));
-                        const float sb = sigmoid((h ? pbg.y : pbg.x) + (h ? b3.y : b3.x));
-                        g[0][h] = dah * sa;
-                        g[1][h] = dah * ((h ? pa.y : pa.x) + (h ? b0.y : b0.x)) * sa * (1.f - sa);
-                        g[2][h] = dbh * sb;
-                        g[3][h] = dbh * ((h ? pb.y : pb.x) + (h ? b2.y : b2.x)) * sb * (1.f - sb);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        acc[k][2 * t] += g[k][0];
-                        acc[k][2 * t + 1] += g[k][1];
-                        o[k][t] = f2bf(g[k][0], g[k][1]);
-                    }
+                for (int h = 0; h < 2; ++h) {
+                    const float dah = (h ? da.y : da.x) * mk, dbh = (h ? db.y : db.x) * mk;
+                    const float sa = sigmoid((h ? pag.y : pag.x) + (h ? b1.y : b1.x));
+                    const float sb = sigmoid((h ? pbg.y : pbg.x) + (h ? b3.y : b3.x));
+                    g[0][h] = dah * sa;
+                    g[1][h] = dah * ((h ? pa.y : pa.x) + (h ? b0.y : b0.x)) * sa * (1.f - sa);
+                    g[2][h] = dbh * sb;
+                    g[3][h] = dbh * ((h ? pb.y : pb.x) + (h ? b2.y : b2.x)) * sb * (1.f - sb);
                 }
-                bf *d = a.D + m * kP + c0;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) st16(d + (P_A + k) * kC, make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]));
+                for (int k = 0; k < 4; ++k) {
+                    acc[k][2 * e] += g[k][0];
+                    acc[k][2 * e + 1] += g[k][1];
+                    o[k][e] = f2bf(g[k][0], g[k][1]);
+                }
             }
+            bf *d = a.D + m * kP + c0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) st16(d + (P_A + k) * kC, make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]));
         }
+        if (threadIdx.x < kPT) msk[(s ^ 1) * kPT + threadIdx.x] = mnext;
+        __syncthreads();  // stage s is read out
+        proj_issue(a, proj_tile(t + 2 * dt, tiles, jt), st);
+        cp_async_commit();
     }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     float *const dst[4] = {a.db, a.db + kC, a.db + 2 * kC, a.db + 3 * kC};
     flush_sums<4>(acc, dst, red);
 }
@@ -449,7 +530,6 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(WgradReduceArgs a) {
 
 size_t ln_fwd_smem(bool cm) { return cm ? kTileBytes : 0; }
 size_t ln_bwd_smem(bool cm) { return (cm ? kTileBytes : 0) + kRedBytes; }
-constexpr size_t kProjSmem = 2 * kTileBytes + kRedBytes;
 
 // One wave: the resident blocks of the kernel on all SMs, at most `work`.
 template <typename K>
@@ -466,6 +546,8 @@ long long tiles_of(int N) { return (long long)N * ((N + kTile - 1) / kTile); }
 
 cudaError_t backward_setup() {
     cudaError_t e = cudaFuncSetAttribute(proj_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kProjSmem);
+    if (e == cudaSuccess)  // all of the unified L1 as shared memory: room for two blocks per SM
+        e = cudaFuncSetAttribute(proj_bwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(ln_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)ln_bwd_smem(true));
@@ -499,7 +581,7 @@ cudaError_t launch_gate_bwd(const GateBwdArgs &a, int sms, cudaStream_t s) {
 }
 
 cudaError_t launch_proj_bwd(const ProjBwdArgs &a, int sms, cudaStream_t s) {
-    proj_bwd_kernel<<<wave(proj_bwd_kernel, kProjSmem, sms, tiles_of(a.N)), kThreads, kProjSmem, s>>>(a);
+    proj_bwd_kernel<<<wave(proj_bwd_kernel, kProjSmem, sms, (long long)a.N * ((a.N + kPT - 1) / kPT)), kThreads, kProjSmem, s>>>(a);
     return cudaGetLastError();
 }
 
