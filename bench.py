@@ -495,6 +495,43 @@ def run_attention_only(args):
     print(json.dumps({"atom_attention": res}), flush=True)
 
 
+def backward_blocked_timing(tm, pi, torch, dev, stream, block_rows=256, warmup=1, reps=2):
+    """The backward of the largest workload (N = 3605, outgoing) in blocks of
+    `block_rows` rows: the workspace that trimul_backward_workspace_size_rows
+    gives for them against the whole-grid size, and the time per call (CUDA
+    events). dout is drawn on the device (values do not change the work)."""
+    w = pi.WORKLOADS[5]
+    N = w.N
+    case = pi.make_workload(w)
+    z = torch.from_numpy(case["z"]).to(dev).to(torch.bfloat16)
+    mask = torch.from_numpy(case["mask"]).to(dev).to(torch.bfloat16)
+    del case["z"]
+    gen = torch.Generator(device=dev).manual_seed(11)
+    dout = torch.randn(z.shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    sd = {key: torch.from_numpy(case[field]) for field, key, _ in tm.STATE_KEYS if field in case}
+    layer = tm.TriangleMultiplicationOutgoing(128, 128).load_state_dict(sd).to(dev, torch.bfloat16)
+    for _ in range(warmup):
+        layer.backward(z, dout, mask, stream=stream, block_rows=block_rows)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer.backward(z, dout, mask, stream=stream, block_rows=block_rows)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    med = ts[len(ts) // 2]
+    res = {"workload": w.name, "N": N, "direction": "outgoing", "block_rows": block_rows,
+           "workspace_gb": round(tm.trimul_backward_workspace_size_rows(N, block_rows) / 1e9, 2),
+           "whole_grid_workspace_gb": round(tm.trimul_backward_workspace_size(N) / 1e9, 2),
+           "median_us": round(med, 1), "pair_cells_per_s": round(N * N / (med * 1e-6)),
+           "gemm_tflops": round(N * N * backward_flops_per_cell(N) / (med * 1e-6) / 1e12, 1)}
+    del layer, z, mask, dout
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_backward_only(args):
     """--backward-only: the backward secondary figure alone, on one GPU."""
     import torch
@@ -509,6 +546,8 @@ def run_backward_only(args):
     tm.lib()
     peaks, _ = load_peaks()
     res = backward_timings(tm, pi, torch, dev, torch.cuda.current_stream(dev), peaks, args.warmup, args.steps)
+    if args.backward_blocked:
+        res["blocked_large"] = backward_blocked_timing(tm, pi, torch, dev, torch.cuda.current_stream(dev))
     print(json.dumps({"backward": res}), flush=True)
 
 
@@ -958,6 +997,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload secondary timings")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward secondary timing")
+    ap.add_argument("--backward-blocked", action="store_true",
+                    help="with --backward-only: also the N = 3605 backward in blocks of 256 rows")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only trimul_backward (W warm-up and K timed calls per direction) and print that")
     ap.add_argument("--no-attention", action="store_true", help="skip the atom-attention secondary timing")

@@ -279,7 +279,7 @@ typedef struct {
     float *d_ln_in_w, *d_ln_in_b;           /* [c_z] */
     float *d_ln_out_w, *d_ln_out_b;         /* [c_h] */
     void *workspace;                        /* device memory, 256-byte aligned */
-    size_t workspace_bytes;                 /* >= trimul_backward_workspace_size */
+    size_t workspace_bytes;                 /* >= trimul_backward_workspace_size_rows(.., 1) */
     uint32_t flags;                         /* TRIMUL_BWD_*; 0 = recompute the forward */
 } trimul_grads;
 
@@ -290,8 +290,22 @@ typedef struct {
  * wrong; no check is made. */
 #define TRIMUL_BWD_REUSE_FORWARD 0x1u
 
-/* Bytes of backward workspace (trimul_grads.workspace) for N. */
+/* Bytes of backward workspace (trimul_grads.workspace) for N: with this much
+ * the per-cell intermediates of the whole grid fit at once (about 6.5 KB per
+ * cell at c_z = c_h = 128). */
 size_t trimul_backward_workspace_size(int N, int c_z, int c_h);
+
+/* Bytes of backward workspace when the per-cell steps run over blocks of
+ * `rows` rows (1 <= rows <= N; 0 for an invalid argument). trimul_backward
+ * takes whatever workspace it is given, at least this for rows = 1, and uses
+ * the largest block of rows that fits: the per-cell intermediates then take
+ * about 4.1 KB per cell of one block, beside about 1 KB per cell of the whole
+ * grid (dL/dx, dL/da and dL/db channel-major, dP_g) and the weight-gradient
+ * partials (96 B per cell). Blocks smaller than the grid cost a second
+ * LayerNorm and projection of each block's z; the result of every cell is
+ * computed the same way, so dz is the same bit for bit and the parameter
+ * gradients differ only in the order of their fp32 sums. */
+size_t trimul_backward_workspace_size_rows(int N, int c_z, int c_h, int rows);
 
 int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,
                     void *dz, const trimul_grads *g, trimul_stream_t stream);

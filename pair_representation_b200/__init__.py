@@ -39,7 +39,7 @@ ERR = {v: k for k, v in STATUS.items()}
 EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forward", "trimul_prologue",
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
            "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
-           "trimul_backward", "trimul_backward_workspace_size",
+           "trimul_backward", "trimul_backward_workspace_size", "trimul_backward_workspace_size_rows",
            "trimul_workspace_size_mxfp8", "trimul_forward_mxfp8", "trimul_contract_mxfp8", "trimul_mxfp8_views",
            "trimul_prologue_mxfp8", "trimul_mma_mxfp8",
            "trimul_shard_workspace_size", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows",
@@ -127,6 +127,8 @@ def lib():
         L.trimul_version.argtypes = []
         L.trimul_backward_workspace_size.argtypes = [I, I, I]
         L.trimul_backward_workspace_size.restype = S
+        L.trimul_backward_workspace_size_rows.argtypes = [I, I, I, I]
+        L.trimul_backward_workspace_size_rows.restype = S
         L.trimul_backward.argtypes = [P, P, PP, I, P, P, ctypes.POINTER(TrimulGrads), P]
         L.trimul_workspace_size_mxfp8.argtypes = [I, I, I]
         L.trimul_workspace_size_mxfp8.restype = S
@@ -230,6 +232,10 @@ def trimul_epilogue(z, params: TrimulParams, out, stream=None, check=True) -> in
 
 def trimul_backward_workspace_size(N: int, c_z: int = 128, c_h: int = 128) -> int:
     return lib().trimul_backward_workspace_size(N, c_z, c_h)
+
+
+def trimul_backward_workspace_size_rows(N: int, rows: int, c_z: int = 128, c_h: int = 128) -> int:
+    return lib().trimul_backward_workspace_size_rows(N, c_z, c_h, rows)
 
 
 def trimul_backward(z, mask, params: TrimulParams, direction: int, dout, dz, grads: TrimulGrads, stream=None,
@@ -460,14 +466,17 @@ class _TriangleMultiplication:
         trimul_forward(z, mask, p, self.direction, out, stream)
         return out
 
-    def backward(self, z, dout, mask=None, stream=None, reuse_forward=False):
+    def backward(self, z, dout, mask=None, stream=None, reuse_forward=False, block_rows=None):
         """Gradients of sum(layer(z, mask) * dout): (dz, {params field: fp32 gradient}).
 
         Every parameter gets a gradient, including the optional ones the state
         dict left out (taken as bias 0, gamma 1, beta 0 in the forward). With
         reuse_forward the call relies on the layer's last forward call having
         been ``layer(z, mask)`` with this z and mask (its a, b and x are still in
-        the workspace) and does not recompute them."""
+        the workspace) and does not recompute them. block_rows gives the call
+        only the workspace for blocks of that many rows
+        (trimul_backward_workspace_size_rows); the library then uses the largest
+        block that fits in it."""
         import torch
         if z.dim() != 3 or z.shape[0] != z.shape[1] or z.shape[2] != self.c_z:
             raise ValueError("z must be [N, N, c_z]")
@@ -479,10 +488,13 @@ class _TriangleMultiplication:
         N = z.shape[0]
         p = self.params(N)
         g = TrimulGrads()
-        need = trimul_backward_workspace_size(N, self.c_z, self.c_h)
+        need = (trimul_backward_workspace_size(N, self.c_z, self.c_h) if block_rows is None
+                else trimul_backward_workspace_size_rows(N, block_rows, self.c_z, self.c_h))
+        if need == 0:
+            raise ValueError("no backward workspace size for these arguments")
         if getattr(self, "_bws", None) is None or self._bws.numel() < need:
             self._bws = torch.empty(need, dtype=torch.uint8, device=self.device)
-        g.workspace, g.workspace_bytes = self._bws.data_ptr(), self._bws.numel()
+        g.workspace, g.workspace_bytes = self._bws.data_ptr(), need
         g.flags = BWD_REUSE_FORWARD if reuse_forward else 0
         cz, ch = self.c_z, self.c_h
         shapes = {"w_a": (ch, cz), "w_ag": (ch, cz), "w_b": (ch, cz), "w_bg": (ch, cz), "w_g": (cz, cz),

@@ -738,15 +738,19 @@ int run_prologue_mx(const void *z, const void *mask, const trimul_params *p, int
 
 constexpr long long kWgradChunk = 4096;  // cells per weight-gradient GEMM partial
 
-long long wgrad_slots(int N) { return ((long long)N * N + kWgradChunk - 1) / kWgradChunk; }
+// Weight-gradient partials of one block of R rows: one per kWgradChunk cells.
+long long wgrad_slots(int N, int R) { return ((long long)R * N + kWgradChunk - 1) / kWgradChunk; }
 
-// Sections of the backward workspace (byte offsets, each 256-byte aligned).
+// Sections of the backward workspace (byte offsets, each 256-byte aligned) for
+// blocks of R rows: the per-cell intermediates and the weight-gradient partials
+// hold one block (R N cells); dX, dA, dB (channel-major) and dP_G (only when
+// R < N) cover the whole grid.
 struct BwdLayout {
-    size_t sums, wstack, st_in, st_out, zh, xh, P, Y, dxh, D, dy, dX, dA, dB, partial, total;
+    size_t sums, wstack, wacc, st_in, st_out, zh, xh, P, Y, dxh, D, dy, dg, dX, dA, dB, partial, total;
 };
 
-BwdLayout bwd_layout(int N) {
-    const size_t M = (size_t)N * N, C = kC, cm = C * (size_t)N * ld_of(N);
+BwdLayout bwd_layout(int N, int R) {
+    const size_t M = (size_t)R * N, C = kC, cm = C * (size_t)N * ld_of(N);
     BwdLayout L;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -756,6 +760,7 @@ BwdLayout bwd_layout(int N) {
     };
     L.sums = take((size_t)kSumCount * C * 4);
     L.wstack = take((size_t)kProjBlocks * C * C * 2);
+    L.wacc = take((size_t)kWgradRows * C * 8);   // weight-gradient sums over the blocks, double
     L.st_in = take(M * 8);
     L.st_out = take(M * 8);
     L.zh = take(M * C * 2);                 // LayerNorm_in(z), bf16 [cells][128]
@@ -765,12 +770,28 @@ BwdLayout bwd_layout(int N) {
     L.dxh = take(M * C * 4);                // dL/dxh, fp32
     L.D = take(M * kProjBlocks * C * 2);    // pre-activation gradients, bf16
     L.dy = take(M * C * 2);                 // dL/dy, bf16
+    L.dg = R < N ? take((size_t)N * N * C * 2) : 0;  // dP_G of every cell, bf16 [cells][128]
     L.dX = take(cm * 2);                    // dL/dx, bf16 [128][N][ld]
     L.dA = take(cm * 2);                    // dL/da, bf16 [128][N][ld]
     L.dB = take(cm * 2);
-    L.partial = take((size_t)wgrad_slots(N) * kWgradRows * C * 4);
+    L.partial = take((size_t)wgrad_slots(N, R) * kWgradRows * C * 4);
     L.total = off;
     return L;
+}
+
+// The largest block of rows whose layout fits `bytes` (0 if none does). Below N
+// the size grows with the rows; the whole grid (R = N) needs no dP_G copy, so
+// it is tried first and can fit where N - 1 rows do not.
+int bwd_rows_for(int N, size_t bytes) {
+    if (bwd_layout(N, N).total <= bytes) return N;
+    if (N == 1 || bwd_layout(N, 1).total > bytes) return 0;
+    int lo = 1, hi = N - 1;  // fits(lo); find the largest fitting R in [lo, hi]
+    if (bwd_layout(N, hi).total <= bytes) return hi;
+    while (hi - lo > 1) {  // fits(lo), !fits(hi)
+        const int mid = lo + (hi - lo) / 2;
+        (bwd_layout(N, mid).total <= bytes ? lo : hi) = mid;
+    }
+    return lo;
 }
 
 int check_backward(const trimul_params *p, const void *z, const void *mask, const void *dout, const void *dz,
@@ -778,7 +799,7 @@ int check_backward(const trimul_params *p, const void *z, const void *mask, cons
     if (!dout || !dz || !g) return TRIMUL_ERR_INVALID_ARG;
     if (p->dtype != TRIMUL_DTYPE_BF16) return TRIMUL_ERR_UNSUPPORTED;
     if (!aligned(dout, 16) || !aligned(dz, 16)) return TRIMUL_ERR_MISALIGNED;
-    if (!g->workspace || g->workspace_bytes < bwd_layout(p->N).total) return TRIMUL_ERR_WORKSPACE;
+    if (!g->workspace || bwd_rows_for(p->N, g->workspace_bytes) < 1) return TRIMUL_ERR_WORKSPACE;
     if (!aligned(g->workspace, 256)) return TRIMUL_ERR_MISALIGNED;
     const size_t n = pair_bytes(p), mb = mask_bytes(p);
     const void *gws = g->workspace;
@@ -818,14 +839,21 @@ int check_backward_on_device(const void *dout, const void *dz, const trimul_grad
     return TRIMUL_OK;
 }
 
-// The backward's launch sequence.
+// The backward's launch sequence. The per-cell steps run over blocks of R rows
+// (R = N when the workspace holds the whole grid, else as many rows as fit): a
+// first pass per block down to dL/dx, the contraction's adjoint over the whole
+// grid, then a second pass per block down to dL/dz. With R < N the second pass
+// recomputes zh and the a/b pre-activations of its block, and takes dP_G from
+// the whole-grid copy the first pass left; with R = N it reuses the first
+// pass's zh and P. The arithmetic of every cell is the same either way.
 int run_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout, void *dz,
                  const trimul_grads *gr, const DevState &d, cudaStream_t s) {
     typedef __nv_bfloat16 bf;
-    const int N = p->N, C = kC;
-    const long long cells = (long long)N * N;
+    const int N = p->N, C = kC, PB = kProjBlocks * kC;
+    const int R = bwd_rows_for(N, gr->workspace_bytes);
+    const bool blocked = R < N;
     const Views v = views_of(p);
-    const BwdLayout L = bwd_layout(N);
+    const BwdLayout L = bwd_layout(N, R);
     uint8_t *base = static_cast<uint8_t *>(gr->workspace);
     float *sums = reinterpret_cast<float *>(base + L.sums);
     bf *wstack = reinterpret_cast<bf *>(base + L.wstack);
@@ -834,10 +862,14 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
     bf *P = reinterpret_cast<bf *>(base + L.P), *Y = reinterpret_cast<bf *>(base + L.Y);
     float *dzh = reinterpret_cast<float *>(base + L.P), *dxh = reinterpret_cast<float *>(base + L.dxh);
     bf *D = reinterpret_cast<bf *>(base + L.D), *dy = reinterpret_cast<bf *>(base + L.dy);
+    bf *dg_all = blocked ? reinterpret_cast<bf *>(base + L.dg) : nullptr;
     bf *dX = reinterpret_cast<bf *>(base + L.dX);
     bf *dA = reinterpret_cast<bf *>(base + L.dA), *dB = reinterpret_cast<bf *>(base + L.dB);
     float *partial = reinterpret_cast<float *>(base + L.partial);
+    double *wacc = reinterpret_cast<double *>(base + L.wacc);
     const bf *x = reinterpret_cast<const bf *>(v.x);
+    const bf *zb = static_cast<const bf *>(z), *doutb = static_cast<const bf *>(dout);
+    bf *dzb = static_cast<bf *>(dz);
     int rc;
 
     // Recompute the forward's a, b and x into the forward workspace, unless the caller
@@ -853,65 +885,112 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
                                           cudaMemcpyDeviceToDevice, s), "weight stack copy")))
             return rc;
 
-    LnFwdArgs lf;
-    lf.src = static_cast<const bf *>(z);
-    lf.channel_major = 0;
-    lf.N = N;
-    lf.ld = v.ld;
-    lf.eps = p->ln_eps;
-    lf.gamma = static_cast<const bf *>(p->ln_in_w);
-    lf.beta = static_cast<const bf *>(p->ln_in_b);
-    lf.out = zh;
-    lf.stats = st_in;
-    if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
-    lf.src = x;
-    lf.channel_major = 1;
-    lf.gamma = static_cast<const bf *>(p->ln_out_w);
-    lf.beta = static_cast<const bf *>(p->ln_out_b);
-    lf.out = xh;
-    lf.stats = st_out;
-    if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
-
     // The plain GEMMs run on the pair kernel (run_gemm): X[m][n] = sum_k A(m, k) B(n, k),
     // each operand K-major or MN-major (mn = 1), bf16 in, fp32 accumulation.
     const KernelCtl ctl = ctl_of(p, v);
-    const int M = (int)cells, PB = kProjBlocks * C;
-    // P = zh [W_g; W_a; W_ag; W_b; W_bg]^T and Y = xh W_o^T (before biases), bf16.
-    if ((rc = run_gemm({zh, (size_t)C, 0}, 0, {wstack, (size_t)C, 0}, 0, {P, (size_t)PB, 0}, 0, M, PB, C, 1, ctl, d,
-                       s)) ||
-        (rc = run_gemm({xh, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 0, {Y, (size_t)C, 0}, 0, M, C, C, 1, ctl, d, s)))
-        return rc;
+    const size_t ck = (size_t)kWgradChunk, pstride = (size_t)kWgradRows * C;
+    float *wdst[kProjBlocks + 1] = {gr->d_w_g, gr->d_w_a, gr->d_w_ag, gr->d_w_b, gr->d_w_bg, gr->d_w_o};
+    // Weight gradients of one block: for each kWgradChunk cells of it, rows row0 ..
+    // row0 + arows of one partial get the sum over the chunk's cells of A[cell][r]
+    // Bm[cell][c] (both operands MN-major: the contracted index is the cell, their row
+    // index; the chunks are the GEMM's batch); then the partials are added, in
+    // double, to the sums over the blocks, which the last block writes out.
+    auto wgrad = [&](const bf *A, int arows, size_t lda, const bf *Bm, long long ncells, int row0, bool first,
+                     bool last) -> int {
+        const long long full = ncells / kWgradChunk, rem = ncells - full * kWgradChunk;
+        float *dst = partial + (size_t)row0 * C;
+        int r;
+        if (full > 0 && (r = run_gemm({A, lda, ck * lda}, 1, {Bm, (size_t)C, ck * C}, 1, {dst, (size_t)C, pstride}, 1,
+                                      arows, C, (int)kWgradChunk, (int)full, ctl, d, s)))
+            return r;
+        if (rem > 0 && (r = run_gemm({A + (size_t)full * ck * lda, lda, ck * lda}, 1, {Bm + (size_t)full * ck * C,
+                                      (size_t)C, ck * C}, 1, {dst + (size_t)full * pstride, (size_t)C, pstride}, 1,
+                                      arows, C, (int)rem, 1, ctl, d, s)))
+            return r;
+        WgradReduceArgs wr;
+        wr.partial = partial;
+        wr.slots = (int)(full + (rem > 0));
+        wr.row0 = row0;
+        wr.rows = arows;
+        wr.acc = wacc;
+        wr.first = first;
+        wr.last = last;
+        for (int k = 0; k <= kProjBlocks; ++k) wr.dst[k] = wdst[k];
+        return cuda_rc(launch_wgrad_reduce(wr, s), "wgrad_reduce launch");
+    };
 
-    GateBwdArgs ga;
-    ga.dout = static_cast<const bf *>(dout);
-    ga.P = P;
-    ga.Y = Y;
-    ga.b_g = static_cast<const bf *>(p->b_g);
-    ga.b_o = static_cast<const bf *>(p->b_o);
-    ga.dy = dy;
-    ga.D = D;
-    ga.db_g = sums + S_B_G * C;
-    ga.db_o = sums + S_B_O * C;
-    ga.cells = cells;
-    if ((rc = cuda_rc(launch_gate_bwd(ga, d.sms, s), "gate_bwd launch"))) return rc;
-
-    // dL/dxh = dy W_o (fp32): B(n, k) = W_o[k][n] is MN-major.
-    if ((rc = run_gemm({dy, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 1, {dxh, (size_t)C, 0}, 1, M, C, C, 1, ctl, d,
-                       s)))
-        return rc;
-
+    LnFwdArgs lf;
+    lf.N = N;
+    lf.ld = v.ld;
+    lf.eps = p->ln_eps;
     LnBwdArgs lb;
-    lb.dh = dxh;
-    lb.src = x;
-    lb.channel_major = 1;
     lb.N = N;
     lb.ld = v.ld;
-    lb.stats = st_out;
-    lb.gamma = static_cast<const bf *>(p->ln_out_w);
-    lb.dsrc = dX;
-    lb.dgamma = sums + S_LN_OUT_W * C;
-    lb.dbeta = sums + S_LN_OUT_B * C;
-    if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+    // LayerNorm_in of the block's z rows into zh (and its statistics).
+    auto ln_in = [&](int r0, int nr) {
+        lf.src = zb + (size_t)r0 * N * C;
+        lf.channel_major = 0;
+        lf.rows = nr;
+        lf.i0 = r0;
+        lf.gamma = static_cast<const bf *>(p->ln_in_w);
+        lf.beta = static_cast<const bf *>(p->ln_in_b);
+        lf.out = zh;
+        lf.stats = st_in;
+        return cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch");
+    };
+
+    // ---- first pass, per block of rows: down to dL/dx ----
+    for (int r0 = 0; r0 < N; r0 += R) {
+        const int nr = N - r0 < R ? N - r0 : R, M = nr * N;
+        if ((rc = ln_in(r0, nr))) return rc;
+        lf.src = x;
+        lf.channel_major = 1;
+        lf.gamma = static_cast<const bf *>(p->ln_out_w);
+        lf.beta = static_cast<const bf *>(p->ln_out_b);
+        lf.out = xh;
+        lf.stats = st_out;
+        if ((rc = cuda_rc(launch_ln_fwd(lf, d.sms, s), "ln_fwd launch"))) return rc;
+        // P = zh [W_g; W_a; W_ag; W_b; W_bg]^T (only its P_G block when the second pass
+        // recomputes the rest) and Y = xh W_o^T, before biases, bf16.
+        if ((rc = run_gemm({zh, (size_t)C, 0}, 0, {wstack, (size_t)C, 0}, 0, {P, (size_t)PB, 0}, 0, M,
+                           blocked ? C : PB, C, 1, ctl, d, s)) ||
+            (rc = run_gemm({xh, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 0, {Y, (size_t)C, 0}, 0, M, C, C, 1, ctl, d,
+                           s)))
+            return rc;
+
+        GateBwdArgs ga;
+        ga.dout = doutb + (size_t)r0 * N * C;
+        ga.P = P;
+        ga.Y = Y;
+        ga.b_g = static_cast<const bf *>(p->b_g);
+        ga.b_o = static_cast<const bf *>(p->b_o);
+        ga.dy = dy;
+        ga.dg = blocked ? dg_all + (size_t)r0 * N * C : D + P_G * C;
+        ga.dg_stride = blocked ? (size_t)C : (size_t)PB;
+        ga.db_g = sums + S_B_G * C;
+        ga.db_o = sums + S_B_O * C;
+        ga.cells = M;
+        if ((rc = cuda_rc(launch_gate_bwd(ga, d.sms, s), "gate_bwd launch"))) return rc;
+
+        // dL/dxh = dy W_o (fp32): B(n, k) = W_o[k][n] is MN-major.
+        if ((rc = run_gemm({dy, (size_t)C, 0}, 0, {p->w_o, (size_t)C, 0}, 1, {dxh, (size_t)C, 0}, 1, M, C, C, 1, ctl,
+                           d, s)))
+            return rc;
+
+        lb.dh = dxh;
+        lb.src = x;
+        lb.channel_major = 1;
+        lb.rows = nr;
+        lb.i0 = r0;
+        lb.stats = st_out;
+        lb.gamma = static_cast<const bf *>(p->ln_out_w);
+        lb.dsrc = dX;
+        lb.dgamma = sums + S_LN_OUT_W * C;
+        lb.dbeta = sums + S_LN_OUT_B * C;
+        if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+        // W_o gradient partials: dy^T xh.
+        if ((rc = wgrad(dy, C, (size_t)C, xh, M, PB, r0 == 0, r0 + nr == N))) return rc;
+    }
 
     // The contraction's adjoint on the forward's contraction kernel, in the
     // form X[m][n] = sum_k A(m, k) B(n, k) with each operand K- or MN-major:
@@ -931,61 +1010,58 @@ int run_backward(const void *z, const void *mask, const trimul_params *p, int di
             return rc;
     }
 
-    ProjBwdArgs pa;
-    pa.dA = dA;
-    pa.dB = dB;
-    pa.P = P;
-    pa.mask = static_cast<const bf *>(mask);
-    pa.b_a = static_cast<const bf *>(p->b_a);
-    pa.b_ag = static_cast<const bf *>(p->b_ag);
-    pa.b_b = static_cast<const bf *>(p->b_b);
-    pa.b_bg = static_cast<const bf *>(p->b_bg);
-    pa.D = D;
-    pa.db = sums + S_B_A * C;
-    pa.N = N;
-    pa.ld = v.ld;
-    if ((rc = cuda_rc(launch_proj_bwd(pa, d.sms, s), "proj_bwd launch"))) return rc;
+    // ---- second pass, per block of rows: down to dL/dz ----
+    for (int r0 = 0; r0 < N; r0 += R) {
+        const int nr = N - r0 < R ? N - r0 : R, M = nr * N;
+        if (blocked) {
+            // zh and P_A .. P_BG of the block again; its dP_G into D's first block.
+            if ((rc = ln_in(r0, nr)) ||
+                (rc = run_gemm({zh, (size_t)C, 0}, 0, {wstack + (size_t)C * C, (size_t)C, 0}, 0, {P + C, (size_t)PB, 0},
+                               0, M, PB - C, C, 1, ctl, d, s)) ||
+                (rc = cuda_rc(cudaMemcpy2DAsync(D, (size_t)PB * 2, dg_all + (size_t)r0 * N * C, (size_t)C * 2,
+                                                (size_t)C * 2, (size_t)M, cudaMemcpyDeviceToDevice, s),
+                              "dP_G copy")))
+                return rc;
+        }
 
-    // Weight gradients, one partial per chunk of kWgradChunk cells:
-    //   rows [0, 640):   D^T zh  ([W_g; W_a; W_ag; W_b; W_bg] gradients)
-    //   rows [640, 768): dy^T xh (W_o gradient)
-    // then summed over the chunks in double. Both operands are MN-major here (the
-    // contracted index is the cell, the row index of D, dy, zh and xh); the chunks
-    // are the GEMM's batch.
-    const long long full = cells / kWgradChunk, rem = cells - full * kWgradChunk;
-    const size_t ck = (size_t)kWgradChunk, pstride = (size_t)kWgradRows * C;
-    auto wgrad = [&](size_t r0, int K, int batch, float *dst) {
-        int r;
-        if ((r = run_gemm({D + r0 * PB, (size_t)PB, ck * PB}, 1, {zh + r0 * C, (size_t)C, ck * C}, 1,
-                          {dst, (size_t)C, pstride}, 1, PB, C, K, batch, ctl, d, s)))
-            return r;
-        return run_gemm({dy + r0 * C, (size_t)C, ck * C}, 1, {xh + r0 * C, (size_t)C, ck * C}, 1,
-                        {dst + (size_t)PB * C, (size_t)C, pstride}, 1, C, C, K, batch, ctl, d, s);
-    };
-    if (full > 0 && (rc = wgrad(0, (int)kWgradChunk, (int)full, partial))) return rc;
-    if (rem > 0 && (rc = wgrad((size_t)full * ck, (int)rem, 1, partial + (size_t)full * pstride))) return rc;
-    WgradReduceArgs wr;
-    wr.partial = partial;
-    wr.slots = (int)wgrad_slots(N);
-    float *wdst[kProjBlocks + 1] = {gr->d_w_g, gr->d_w_a, gr->d_w_ag, gr->d_w_b, gr->d_w_bg, gr->d_w_o};
-    for (int k = 0; k <= kProjBlocks; ++k) wr.dst[k] = wdst[k];
-    if ((rc = cuda_rc(launch_wgrad_reduce(wr, s), "wgrad_reduce launch"))) return rc;
+        ProjBwdArgs pa;
+        pa.dA = dA;
+        pa.dB = dB;
+        pa.P = P;
+        pa.mask = static_cast<const bf *>(mask);
+        pa.b_a = static_cast<const bf *>(p->b_a);
+        pa.b_ag = static_cast<const bf *>(p->b_ag);
+        pa.b_b = static_cast<const bf *>(p->b_b);
+        pa.b_bg = static_cast<const bf *>(p->b_bg);
+        pa.D = D;
+        pa.db = sums + S_B_A * C;
+        pa.N = N;
+        pa.rows = nr;
+        pa.i0 = r0;
+        pa.ld = v.ld;
+        if ((rc = cuda_rc(launch_proj_bwd(pa, d.sms, s), "proj_bwd launch"))) return rc;
 
-    // dL/dzh = D [W_g; W_a; W_ag; W_b; W_bg] (fp32, over the spent pre-activations):
-    // B(n, k) = Wstack[k][n] is MN-major.
-    if ((rc = run_gemm({D, (size_t)PB, 0}, 0, {wstack, (size_t)C, 0}, 1, {dzh, (size_t)C, 0}, 1, M, C, PB, 1, ctl, d,
-                       s)))
-        return rc;
+        // [W_g; W_a; W_ag; W_b; W_bg] gradient partials: D^T zh.
+        if ((rc = wgrad(D, PB, (size_t)PB, zh, M, 0, r0 == 0, r0 + nr == N))) return rc;
 
-    lb.dh = dzh;
-    lb.src = static_cast<const bf *>(z);
-    lb.channel_major = 0;
-    lb.stats = st_in;
-    lb.gamma = static_cast<const bf *>(p->ln_in_w);
-    lb.dsrc = static_cast<bf *>(dz);
-    lb.dgamma = sums + S_LN_IN_W * C;
-    lb.dbeta = sums + S_LN_IN_B * C;
-    if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+        // dL/dzh = D [W_g; W_a; W_ag; W_b; W_bg] (fp32, over the spent pre-activations):
+        // B(n, k) = Wstack[k][n] is MN-major.
+        if ((rc = run_gemm({D, (size_t)PB, 0}, 0, {wstack, (size_t)C, 0}, 1, {dzh, (size_t)C, 0}, 1, M, C, PB, 1, ctl,
+                           d, s)))
+            return rc;
+
+        lb.dh = dzh;
+        lb.src = zb + (size_t)r0 * N * C;
+        lb.channel_major = 0;
+        lb.rows = nr;
+        lb.i0 = r0;
+        lb.stats = st_in;
+        lb.gamma = static_cast<const bf *>(p->ln_in_w);
+        lb.dsrc = dzb + (size_t)r0 * N * C;
+        lb.dgamma = sums + S_LN_IN_W * C;
+        lb.dbeta = sums + S_LN_IN_B * C;
+        if ((rc = cuda_rc(launch_ln_bwd(lb, d.sms, s), "ln_bwd launch"))) return rc;
+    }
 
     float *vec[kSumCount] = {gr->d_b_g, gr->d_b_o, gr->d_b_a, gr->d_b_ag, gr->d_b_b, gr->d_b_bg,
                              gr->d_ln_out_w, gr->d_ln_out_b, gr->d_ln_in_w, gr->d_ln_in_b};
@@ -1278,7 +1354,12 @@ int trimul_device_status(const trimul_params *p, trimul_stream_t stream, int *de
 
 size_t trimul_backward_workspace_size(int N, int c_z, int c_h) {
     if (N < 1 || N > kMaxN || c_z != kC || c_h != kC) return 0;
-    return bwd_layout(N).total;
+    return bwd_layout(N, N).total;
+}
+
+size_t trimul_backward_workspace_size_rows(int N, int c_z, int c_h, int rows) {
+    if (N < 1 || N > kMaxN || c_z != kC || c_h != kC || rows < 1 || rows > N) return 0;
+    return bwd_layout(N, rows).total;
 }
 
 int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,

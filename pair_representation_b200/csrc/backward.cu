@@ -159,17 +159,18 @@ constexpr int kTChunks = kPT * kChunks;      // one cell-major tile
 static_assert(kRawChunks % kThreads == 0 && kTChunks * 16 >= (int)kRedBytes, "tile sizes");
 
 struct PTile {
-    int i, j0;
-    bool live;  // false past the last tile: nothing is copied
+    int li, i, j0;  // row within the block, global row (i0 + li), first cell
+    bool live;      // false past the last tile: nothing is copied
 };
-__device__ __forceinline__ PTile ptile(long long t, long long tiles, int jt) {
+__device__ __forceinline__ PTile ptile(long long t, long long tiles, int jt, int i0) {
     PTile p;
     p.live = t < tiles;
-    p.i = p.live ? (int)(t / jt) : 0;
+    p.li = p.live ? (int)(t / jt) : 0;
+    p.i = i0 + p.li;
     p.j0 = p.live ? (int)(t % jt) * kPT : 0;
     return p;
 }
-long long ptiles_of(int N) { return (long long)N * ((N + kPT - 1) / kPT); }
+long long ptiles_of(int rows, int N) { return (long long)rows * ((N + kPT - 1) / kPT); }
 
 // The tile cell of pair u (0 or 1) for this half warp.
 __device__ __forceinline__ int pcell_of(int warp, int u) {
@@ -253,7 +254,7 @@ __device__ __forceinline__ void ln_fwd_cell(const uint4 &raw, const float (&gm)[
 __global__ void __launch_bounds__(kThreads, 2) ln_fwd_kernel(LnFwdArgs a) {
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kTile - 1) / kTile;
-    const long long tiles = (long long)a.N * jt;
+    const long long tiles = (long long)a.rows * jt;
     float gm[8], bt[8];
     ld8(a.gamma, c0, 1.f, gm);
     ld8(a.beta, c0, 0.f, bt);
@@ -283,29 +284,29 @@ __global__ void __launch_bounds__(kThreads, 2) ln_fwd_cm_kernel(LnFwdArgs a) {
     uint4 *tile = smem4 + kLnFwdStages * kRawChunks;
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kPT - 1) / kPT;
-    const long long tiles = (long long)a.N * jt, t0 = blockIdx.x, dt = gridDim.x;
+    const long long tiles = (long long)a.rows * jt, t0 = blockIdx.x, dt = gridDim.x;
     float gm[8], bt[8];
     ld8(a.gamma, c0, 1.f, gm);
     ld8(a.beta, c0, 0.f, bt);
 #pragma unroll
     for (int p = 0; p < kLnFwdStages - 1; ++p) {
-        issue_raw(a.src, a.N, a.ld, ptile(t0 + p * dt, tiles, jt), smem4 + p * kRawChunks);
+        issue_raw(a.src, a.N, a.ld, ptile(t0 + p * dt, tiles, jt, a.i0), smem4 + p * kRawChunks);
         cp_async_commit();
     }
     int s = 0;
     for (long long t = t0; t < tiles; t += dt) {
-        const PTile ti = ptile(t, tiles, jt);
+        const PTile ti = ptile(t, tiles, jt, a.i0);
         cp_async_wait<kLnFwdStages - 2>();  // this thread's copies of tile t have landed
         __syncthreads();  // everyone's have; the previous tile's stage and the cell-major tile are free
         const int sn = s == 0 ? kLnFwdStages - 1 : s - 1;
-        issue_raw(a.src, a.N, a.ld, ptile(t + (kLnFwdStages - 1) * dt, tiles, jt), smem4 + sn * kRawChunks);
+        issue_raw(a.src, a.N, a.ld, ptile(t + (kLnFwdStages - 1) * dt, tiles, jt, a.i0), smem4 + sn * kRawChunks);
         cp_async_commit();
         transpose_raw(smem4 + s * kRawChunks, tile);
         __syncthreads();
 #pragma unroll
         for (int u = 0; u < kPT / kWarps / 2; ++u) {
             const int jj = pcell_of(warp, u), j = ti.j0 + jj;
-            const size_t m = (size_t)ti.i * a.N + j;
+            const size_t m = (size_t)ti.li * a.N + j;
             ln_fwd_cell(tile[chunk_at(jj, q)], gm, bt, a.eps, j < a.N, a.out + m * kC + c0, a.stats + m);
         }
         s = s + 1 == kLnFwdStages ? 0 : s + 1;
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2) ln_bwd_kernel(LnBwdArgs a) {
     __shared__ float red[kWarps * kC];
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kTile - 1) / kTile;
-    const long long tiles = (long long)a.N * jt;
+    const long long tiles = (long long)a.rows * jt;
     float gm[8];
     float acc[2][8] = {};
     ld8(a.gamma, c0, 1.f, gm);
@@ -395,12 +396,12 @@ __device__ __forceinline__ void ln_bwd_issue(const LnBwdArgs &a, const PTile &ti
     for (int r = 0; r < kDhChunks / kThreads; ++r) {
         const int z = threadIdx.x + r * kThreads, jj = z >> 5, p = z & 31;
         const bool ok = ti.j0 + jj < a.N;
-        const size_t m = (size_t)ti.i * a.N + (ok ? ti.j0 + jj : 0);
+        const size_t m = (size_t)ti.li * a.N + (ok ? ti.j0 + jj : 0);
         cp_async16(st + kRawChunks + jj * 32 + dh_pos(p), a.dh + m * kC + 4 * p, ok);
     }
     if (threadIdx.x < kPT) {
         const bool ok = ti.j0 + (int)threadIdx.x < a.N;
-        const size_t m = (size_t)ti.i * a.N + (ok ? ti.j0 + threadIdx.x : 0);
+        const size_t m = (size_t)ti.li * a.N + (ok ? ti.j0 + threadIdx.x : 0);
         cp_async8(reinterpret_cast<float2 *>(st + kRawChunks + kDhChunks) + threadIdx.x, a.stats + m, ok);
     }
 }
@@ -411,23 +412,23 @@ __global__ void __launch_bounds__(kThreads, 2) ln_bwd_cm_kernel(LnBwdArgs a) {
     float *red = reinterpret_cast<float *>(tile);  // after the last tile
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kPT - 1) / kPT;
-    const long long tiles = (long long)a.N * jt, t0 = blockIdx.x, dt = gridDim.x;
+    const long long tiles = (long long)a.rows * jt, t0 = blockIdx.x, dt = gridDim.x;
     float gm[8];
     float acc[2][8] = {};
     ld8(a.gamma, c0, 1.f, gm);
 #pragma unroll
     for (int p = 0; p < kLnBwdStages - 1; ++p) {
-        ln_bwd_issue(a, ptile(t0 + p * dt, tiles, jt), smem4 + p * kLnBwdStage);
+        ln_bwd_issue(a, ptile(t0 + p * dt, tiles, jt, a.i0), smem4 + p * kLnBwdStage);
         cp_async_commit();
     }
     int s = 0;
     for (long long t = t0; t < tiles; t += dt) {
-        const PTile ti = ptile(t, tiles, jt);
+        const PTile ti = ptile(t, tiles, jt, a.i0);
         const uint4 *st = smem4 + s * kLnBwdStage;
         cp_async_wait<kLnBwdStages - 2>();  // this thread's copies of tile t have landed
         __syncthreads();  // everyone's have; the previous tile's stage and the cell-major tile are free
         const int sn = s == 0 ? kLnBwdStages - 1 : s - 1;
-        ln_bwd_issue(a, ptile(t + (kLnBwdStages - 1) * dt, tiles, jt), smem4 + sn * kLnBwdStage);
+        ln_bwd_issue(a, ptile(t + (kLnBwdStages - 1) * dt, tiles, jt, a.i0), smem4 + sn * kLnBwdStage);
         cp_async_commit();
         transpose_raw(st, tile);
         __syncthreads();
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2) gate_bwd_kernel(GateBwdArgs a) {
                 acc[1][k] += dy[k];
             }
             st16(a.dy + m * kC + c0, pack8(dy));
-            st16(a.D + m * kP + P_G * kC + c0, pack8(dpg));
+            st16(a.dg + m * a.dg_stride + c0, pack8(dpg));
         }
     }
     float *const dst[2] = {a.db_g, a.db_o};
@@ -514,7 +515,7 @@ __device__ __forceinline__ void proj_issue(const ProjBwdArgs &a, const PTile &ti
     for (int r = 0; r < kProjPChunks / kThreads; ++r) {
         const int x = threadIdx.x + r * kThreads, jj = x >> 6, k = (x >> 4) & 3, q = x & 15;
         const bool ok = ti.j0 + jj < a.N;
-        const size_t m = (size_t)ti.i * a.N + (ok ? ti.j0 + jj : 0);
+        const size_t m = (size_t)ti.li * a.N + (ok ? ti.j0 + jj : 0);
         cp_async16(st + x, a.P + m * kP + (P_A + k) * kC + 8 * q, ok);
     }
     issue_raw(a.dA, a.N, a.ld, ti, st + kProjPChunks);
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
     float *red = reinterpret_cast<float *>(tA);             // after the last tile
     const int warp = threadIdx.x >> 5, q = threadIdx.x & 15, c0 = 8 * q;
     const int jt = (a.N + kPT - 1) / kPT;
-    const long long tiles = (long long)a.N * jt, t0 = blockIdx.x, dt = gridDim.x;
+    const long long tiles = (long long)a.rows * jt, t0 = blockIdx.x, dt = gridDim.x;
     // The four bias vectors stay bf16 (exact), two channels to a register.
     __nv_bfloat162 bias[4][4];
     float acc[4][8] = {};
@@ -540,18 +541,18 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
             bias[k][t] = bp[k] ? __halves2bfloat162(bp[k][c0 + 2 * t], bp[k][c0 + 2 * t + 1])
                                : __floats2bfloat162_rn(0.f, 0.f);
     auto mask_of = [&](long long t) -> float {
-        const PTile ti = ptile(t, tiles, jt);
+        const PTile ti = ptile(t, tiles, jt, a.i0);
         const int j = ti.j0 + (int)threadIdx.x;
         return a.mask && ti.live && j < a.N ? ld(a.mask + (size_t)ti.i * a.N + j) : 1.f;
     };
-    proj_issue(a, ptile(t0, tiles, jt), smem4);
+    proj_issue(a, ptile(t0, tiles, jt, a.i0), smem4);
     cp_async_commit();
-    proj_issue(a, ptile(t0 + dt, tiles, jt), smem4 + kProjStage);
+    proj_issue(a, ptile(t0 + dt, tiles, jt, a.i0), smem4 + kProjStage);
     cp_async_commit();
     if (threadIdx.x < kPT) msk[threadIdx.x] = mask_of(t0);
     int s = 0;
     for (long long t = t0; t < tiles; t += dt, s ^= 1) {
-        const PTile ti = ptile(t, tiles, jt);
+        const PTile ti = ptile(t, tiles, jt, a.i0);
         uint4 *const st = smem4 + s * kProjStage;
         cp_async_wait<1>();  // this thread's copies of tile t have landed
         __syncthreads();     // everyone's have; tA, tB and the other mask slot are free
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
         for (int u = 0; u < kPT / kWarps / 2; ++u) {
             const int jj = pcell_of(warp, u), j = ti.j0 + jj;
             if (j >= a.N) continue;
-            const size_t m = (size_t)ti.i * a.N + j;
+            const size_t m = (size_t)ti.li * a.N + j;
             const float mk = msk[s * kPT + jj];
             // Two channels at a time: the four outputs of channels c0 + 2e, c0 + 2e + 1
             // are packed as they are made, which keeps few values live.
@@ -604,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
         }
         if (threadIdx.x < kPT) msk[(s ^ 1) * kPT + threadIdx.x] = mnext;
         __syncthreads();  // stage s is read out
-        proj_issue(a, ptile(t + 2 * dt, tiles, jt), st);
+        proj_issue(a, ptile(t + 2 * dt, tiles, jt, a.i0), st);
         cp_async_commit();
     }
     cp_async_wait<0>();
@@ -616,10 +617,12 @@ __global__ void __launch_bounds__(kThreads, 2) proj_bwd_kernel(ProjBwdArgs a) {
 
 __global__ void __launch_bounds__(256) wgrad_reduce_kernel(WgradReduceArgs a) {
     constexpr int kPer = kC * kC;
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= kWgradRows * kC) return;
-    double s = 0.0;
+    const int e = a.row0 * kC + blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (a.row0 + a.rows) * kC) return;
+    double s = a.first ? 0.0 : a.acc[e];
     for (int k = 0; k < a.slots; ++k) s += (double)__ldg(a.partial + (size_t)k * kWgradRows * kC + e);
+    a.acc[e] = s;
+    if (!a.last) return;
     float *dst = nullptr;
 #pragma unroll
     for (int k = 0; k <= kProjBlocks; ++k)
@@ -636,7 +639,7 @@ int wave(K kernel, size_t smem, int sms, long long work) {
     return (int)(work < g ? work : g);
 }
 
-long long tiles_of(int N) { return (long long)N * ((N + kTile - 1) / kTile); }
+long long tiles_of(int rows, int N) { return (long long)rows * ((N + kTile - 1) / kTile); }
 
 }  // namespace
 
@@ -654,17 +657,17 @@ cudaError_t backward_setup() {
 
 cudaError_t launch_ln_fwd(const LnFwdArgs &a, int sms, cudaStream_t s) {
     if (a.channel_major)
-        ln_fwd_cm_kernel<<<wave(ln_fwd_cm_kernel, kLnFwdCmSmem, sms, ptiles_of(a.N)), kThreads, kLnFwdCmSmem, s>>>(a);
+        ln_fwd_cm_kernel<<<wave(ln_fwd_cm_kernel, kLnFwdCmSmem, sms, ptiles_of(a.rows, a.N)), kThreads, kLnFwdCmSmem, s>>>(a);
     else
-        ln_fwd_kernel<<<wave(ln_fwd_kernel, 0, sms, tiles_of(a.N)), kThreads, 0, s>>>(a);
+        ln_fwd_kernel<<<wave(ln_fwd_kernel, 0, sms, tiles_of(a.rows, a.N)), kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_ln_bwd(const LnBwdArgs &a, int sms, cudaStream_t s) {
     if (a.channel_major)
-        ln_bwd_cm_kernel<<<wave(ln_bwd_cm_kernel, kLnBwdCmSmem, sms, ptiles_of(a.N)), kThreads, kLnBwdCmSmem, s>>>(a);
+        ln_bwd_cm_kernel<<<wave(ln_bwd_cm_kernel, kLnBwdCmSmem, sms, ptiles_of(a.rows, a.N)), kThreads, kLnBwdCmSmem, s>>>(a);
     else
-        ln_bwd_kernel<<<wave(ln_bwd_kernel, 0, sms, tiles_of(a.N)), kThreads, 0, s>>>(a);
+        ln_bwd_kernel<<<wave(ln_bwd_kernel, 0, sms, tiles_of(a.rows, a.N)), kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -674,12 +677,12 @@ cudaError_t launch_gate_bwd(const GateBwdArgs &a, int sms, cudaStream_t s) {
 }
 
 cudaError_t launch_proj_bwd(const ProjBwdArgs &a, int sms, cudaStream_t s) {
-    proj_bwd_kernel<<<wave(proj_bwd_kernel, kProjSmem, sms, ptiles_of(a.N)), kThreads, kProjSmem, s>>>(a);
+    proj_bwd_kernel<<<wave(proj_bwd_kernel, kProjSmem, sms, ptiles_of(a.rows, a.N)), kThreads, kProjSmem, s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_wgrad_reduce(const WgradReduceArgs &a, cudaStream_t s) {
-    wgrad_reduce_kernel<<<(kWgradRows * kC + 255) / 256, 256, 0, s>>>(a);
+    wgrad_reduce_kernel<<<(a.rows * kC + 255) / 256, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

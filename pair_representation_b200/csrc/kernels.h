@@ -158,13 +158,19 @@ enum BwdSum { S_B_G, S_B_O, S_B_A, S_B_AG, S_B_B, S_B_BG, S_LN_OUT_W, S_LN_OUT_B
 // (their gradients), and of the stacked weight [5 * 128][128].
 enum ProjBlock { P_G, P_A, P_AG, P_B, P_BG, kProjBlocks };
 
+// The per-cell backward kernels work on a block of `rows` rows of the N x N
+// grid, rows i0 .. i0 + rows - 1: cell-major arrays ([cells][...]) are passed
+// already offset to the block's first cell (cell (i0 + r, j) at index r N + j);
+// channel-major arrays ([128][N][ld]) and the mask are passed whole and indexed
+// by the global row.
+
 // LayerNorm of each cell: out = (v - mean) * rstd * gamma + beta as bf16
-// [cells][128], and (mean, rstd) per cell. src is cell-major [N][N][128] or,
+// [cells][128], and (mean, rstd) per cell. src is cell-major [cells][128] or,
 // when channel_major, [128][N][ld].
 struct LnFwdArgs {
     const __nv_bfloat16 *src;
     int channel_major;
-    int N;
+    int N, rows, i0;
     size_t ld;
     float eps;
     const __nv_bfloat16 *gamma, *beta;  // or null
@@ -179,7 +185,7 @@ struct LnBwdArgs {
     const float *dh;  // [cells][128]
     const __nv_bfloat16 *src;
     int channel_major;
-    int N;
+    int N, rows, i0;
     size_t ld;
     const float2 *stats;
     const __nv_bfloat16 *gamma;  // or null
@@ -195,8 +201,9 @@ struct GateBwdArgs {
     const __nv_bfloat16 *Y;     // [cells][128]
     const __nv_bfloat16 *b_g, *b_o;
     __nv_bfloat16 *dy;  // [cells][128]
-    __nv_bfloat16 *D;   // [cells][5 * 128], block P_G written
-    float *db_g, *db_o;
+    __nv_bfloat16 *dg;  // dP_G of cell m at dg + m * dg_stride (128 channels)
+    size_t dg_stride;
+    float *db_g, *db_o;  // or null: no sums
     long long cells;
 };
 
@@ -209,16 +216,22 @@ struct ProjBwdArgs {
     const __nv_bfloat16 *b_a, *b_ag, *b_b, *b_bg;
     __nv_bfloat16 *D;
     float *db;  // [4][128]: b_a, b_ag, b_b, b_bg
-    int N;
+    int N, rows, i0;
     size_t ld;
 };
 
 // Weight gradients: the rows of [W_g; W_a; W_ag; W_b; W_bg; W_o] gradients,
 // each GEMM partial (one per chunk of cells) being [kWgradRows][128] fp32.
 constexpr int kWgradRows = (kProjBlocks + 1) * kC;
+// One reduction adds the partials of one block of rows to a running sum in
+// double (rows row0 .. row0 + rows of the stacked gradient), and the last block
+// writes the sums out.
 struct WgradReduceArgs {
     const float *partial;  // [slots][kWgradRows][128]
     int slots;
+    int row0, rows;
+    double *acc;  // [kWgradRows][128]
+    int first, last;
     float *dst[kProjBlocks + 1];  // [128][128] each (block order above), or null
 };
 

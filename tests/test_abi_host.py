@@ -157,24 +157,38 @@ def test_stage_argument_checks(L):
 
 # ---- backward ------------------------------------------------------------------
 
-def _bwd_layout_bytes(N):
-    """Backward workspace: sums, weight stack, per-cell sections, then one
-    [768][128] fp32 weight-gradient partial per 4096-cell chunk."""
+def _bwd_layout_bytes(N, R=None):
+    """Backward workspace for blocks of R rows (default: the whole grid): sums,
+    weight stack, the double weight-gradient sums, the per-cell sections of one
+    block, dP_G of the whole grid when R < N, dX, dA, dB channel-major, then one
+    [768][128] fp32 weight-gradient partial per 4096 cells of a block."""
+    R = N if R is None else R
     r = lambda v: (v + 255) // 256 * 256
-    M, C, ld = N * N, 128, (N + 63) // 64 * 64
+    M, C, ld = R * N, 128, (N + 63) // 64 * 64
     cm = C * N * ld
-    slots = (M + 4095) // 4096
-    parts = [10 * C * 4, 5 * C * C * 2, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
-             M * C * 4, M * 5 * C * 2, M * C * 2, cm * 2, cm * 2, cm * 2, slots * 768 * C * 4]
+    parts = [10 * C * 4, 5 * C * C * 2, 768 * C * 8, M * 8, M * 8, M * C * 2, M * C * 2, M * 5 * C * 2, M * C * 2,
+             M * C * 4, M * 5 * C * 2, M * C * 2] + ([N * N * C * 2] if R < N else []) + \
+            [cm * 2, cm * 2, cm * 2, (M + 4095) // 4096 * 768 * C * 4]
     return sum(r(p) for p in parts)
 
 
 def test_backward_workspace_size(L):
     for N in (1, 7, 64, 129, 768):
         assert tm.trimul_backward_workspace_size(N) == _bwd_layout_bytes(N), N
+        assert tm.trimul_backward_workspace_size_rows(N, N) == _bwd_layout_bytes(N), N
+    for N, R in ((7, 1), (64, 5), (129, 64), (200, 37), (768, 100), (3605, 256)):
+        assert tm.trimul_backward_workspace_size_rows(N, R) == _bwd_layout_bytes(N, R), (N, R)
     assert tm.trimul_backward_workspace_size(0) == 0
     assert tm.trimul_backward_workspace_size(16385) == 0
     assert tm.trimul_backward_workspace_size(64, 64, 128) == 0
+    assert tm.trimul_backward_workspace_size_rows(64, 0) == 0
+    assert tm.trimul_backward_workspace_size_rows(64, 65) == 0
+    # The largest workload's backward: about 65 GB for the whole grid, under 18 GB in blocks of 256 rows.
+    assert tm.trimul_backward_workspace_size(3605) > 60e9
+    assert tm.trimul_backward_workspace_size_rows(3605, 256) < 18e9
+    # Below the whole grid the size grows with the rows.
+    sizes = [tm.trimul_backward_workspace_size_rows(200, R) for R in range(1, 200)]
+    assert all(a < b for a, b in zip(sizes, sizes[1:]))
 
 
 DOUT = BASE + 0x100000000
@@ -207,7 +221,7 @@ def test_backward_argument_checks(L):
     assert _bwd(p, g, dz=DZ + 2) == E["TRIMUL_ERR_MISALIGNED"]
     q = _grads(); q.workspace = None
     assert _bwd(p, q) == E["TRIMUL_ERR_WORKSPACE"]
-    q = _grads(); q.workspace_bytes -= 1
+    q = _grads(); q.workspace_bytes = tm.trimul_backward_workspace_size_rows(64, 1) - 1
     assert _bwd(p, q) == E["TRIMUL_ERR_WORKSPACE"]
     q = _grads(); q.workspace += 128
     assert _bwd(p, q) == E["TRIMUL_ERR_MISALIGNED"]

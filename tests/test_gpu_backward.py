@@ -39,12 +39,14 @@ def _gpu():
     tm.lib()
 
 
-def run_backward(case, direction, dout, with_mask=True):
-    """dz and the 16 parameter gradients from the library, as float64 numpy."""
+def run_backward(case, direction, dout, with_mask=True, rows=None):
+    """dz and the 16 parameter gradients from the library, as float64 numpy;
+    with `rows`, given only the workspace for blocks of that many rows."""
     dc = DeviceCase(case, "bf16", with_mask=with_mask)
     N = dc.N
     g = tm.TrimulGrads()
-    bws = torch.empty(tm.trimul_backward_workspace_size(N), dtype=torch.uint8, device="cuda")
+    need = tm.trimul_backward_workspace_size(N) if rows is None else tm.trimul_backward_workspace_size_rows(N, rows)
+    bws = torch.empty(need, dtype=torch.uint8, device="cuda")
     g.workspace, g.workspace_bytes = bws.data_ptr(), bws.numel()
     out = {}
     for f in tm.GRAD_FIELDS:
@@ -178,3 +180,39 @@ def test_backward_reusing_the_forward_matches_recompute(direction):
         assert rel_l2(v.double().cpu().numpy(), ref[k]) <= 1e-6, k
     compare({**{k: v.double().cpu().numpy() for k, v in grads.items()}, "z": dz.double().cpu().numpy()},
             ob.trimul_backward(case, direction, dout.astype(np.float64)), "reuse")
+
+
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_backward_in_row_blocks(direction):
+    """Given the workspace for blocks of 37 rows, the N = 200 backward runs in
+    five blocks of 37 rows and one of 15. Every cell is computed as in the
+    whole-grid call, so dz is the same bit for bit; the parameter gradients
+    differ only in the order of their fp32 sums. Both match the oracle."""
+    N = 200
+    case = pi.random_case(N, 53, bf16=True, affine=True, mask="random")
+    dout = draw_dout(N, 53)
+    whole = run_backward(case, direction, dout)
+    blocks = run_backward(case, direction, dout, rows=37)
+    assert np.array_equal(blocks["z"], whole["z"])
+    for k in ob.WEIGHTS + ob.BIASES + ob.AFFINES:
+        assert rel_l2(blocks[k], whole[k]) <= 1e-5, k
+    compare(blocks, ob.trimul_backward(case, direction, dout), f"blocks of 37 rows {direction}")
+
+
+def test_backward_single_row_blocks_through_the_layer():
+    """The smallest workspace (blocks of one row) through the layer API: the
+    same dz as the whole-grid call, the same gradients up to summation order."""
+    N = 64
+    case = pi.random_case(N, 55, bf16=True, affine=True, mask="random")
+    dout = draw_dout(N, 55)
+    ref = run_backward(case, "incoming", dout)
+    sd = {key: case[field] for field, key, _ in tm.STATE_KEYS if field in case}
+    layer = tm.TriangleMultiplicationIncoming(128, 128).load_state_dict(sd).to("cuda", torch.bfloat16)
+    z = torch.from_numpy(case["z"]).to("cuda").to(torch.bfloat16)
+    m = torch.from_numpy(case["mask"]).to("cuda")
+    d = torch.from_numpy(dout).to("cuda").to(torch.bfloat16)
+    dz, grads = layer.backward(z, d, m, block_rows=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(dz.double().cpu().numpy(), ref["z"])
+    for k, v in grads.items():
+        assert rel_l2(v.double().cpu().numpy(), ref[k]) <= 1e-5, k
