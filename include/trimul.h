@@ -291,7 +291,7 @@ typedef struct {
 #define TRIMUL_BWD_REUSE_FORWARD 0x1u
 
 /* Bytes of backward workspace (trimul_grads.workspace) for N: with this much
- * the per-cell intermediates of the whole grid fit at once (about 6.5 KB per
+ * the per-cell intermediates of the whole grid fit at once (about 5 KB per
  * cell at c_z = c_h = 128). */
 size_t trimul_backward_workspace_size(int N, int c_z, int c_h);
 
