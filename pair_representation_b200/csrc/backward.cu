@@ -2,7 +2,9 @@
 // triangle multiplicative update ("Scaling biomolecular modeling with context
 // parallelism in NVIDIA BioNeMo", section "Context-parallel implementation of
 // triangle multiplication": the layer's forward, differentiated by hand), and
-// the final reduction of the weight gradients.
+// the reduction of the weight-gradient partials into sums in double. Each
+// kernel works on one block of rows of the N x N grid (all of it, or as many
+// rows as the caller's workspace holds).
 //
 // These are the elementwise and per-cell steps of the backward; its GEMMs run
 // on the tcgen05 pair kernel (contract_tc.cu). Half a warp serves one cell:
