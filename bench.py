@@ -52,6 +52,8 @@ UNIT = "pair-cells/s"
 DEFAULT_WORKLOAD = 3
 FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (HGX HBM3e bandwidth, dense bf16 tensor rate), reported beside the measured ones.
+NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 KERNELS = ("prologue_tc_kernel", "contract_tc_kernel", "epilogue_tc_kernel")
 
 
@@ -865,9 +867,11 @@ def run_ours(args, rank, world, local_rank):
             if u == "bytes":
                 entry["achieved_gbs"] = round(q / avg / 1e9, 1)
                 entry["frac_hbm"] = round(q / avg / 1e9 / peaks["hbm_gbs"], 4)
+                entry["frac_hbm_nominal"] = round(q / avg / 1e9 / NOMINAL_PEAKS["hbm_gbs"], 4)
             else:
                 entry["achieved_tflops"] = round(q / avg / 1e12, 1)
                 entry["frac_tensor"] = round(q / avg / 1e12 / peaks["bf16_tflops"], 4)
+                entry["frac_tensor_nominal"] = round(q / avg / 1e12 / NOMINAL_PEAKS["bf16_tflops"], 4)
         breakdown[n] = entry
     roofline = None
     if dom in alg:
@@ -935,6 +939,8 @@ def run_ours(args, rank, world, local_rank):
         "tflops_frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
         "roofline": roofline,
         "kernels": breakdown,
+        "peaks": {"frac_hbm and frac_tensor against": dict(peaks, source=peak_src),
+                  "frac_*_nominal against (datasheet)": NOMINAL_PEAKS},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": sum(launches.values()),
