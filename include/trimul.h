@@ -307,6 +307,12 @@ size_t trimul_backward_workspace_size(int N, int c_z, int c_h);
  * gradients differ only in the order of their fp32 sums. */
 size_t trimul_backward_workspace_size_rows(int N, int c_z, int c_h, int rows);
 
+/* The block of rows trimul_backward uses with a workspace of workspace_bytes:
+ * N when the whole grid fits, else the largest block that fits, 0 when none
+ * does (the call then returns TRIMUL_ERR_WORKSPACE) or for an invalid size.
+ * Host only. */
+int trimul_backward_block_rows(int N, int c_z, int c_h, size_t workspace_bytes);
+
 int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,
                     void *dz, const trimul_grads *g, trimul_stream_t stream);
 

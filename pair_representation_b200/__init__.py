@@ -40,6 +40,7 @@ EXPORTS = ("trimul_workspace_size", "trimul_workspace_size_dtype", "trimul_forwa
            "trimul_contract", "trimul_epilogue", "trimul_workspace_views", "trimul_device_status",
            "trimul_error_string", "trimul_last_error_detail", "trimul_version", "trimul_forward_noalloc",
            "trimul_backward", "trimul_backward_workspace_size", "trimul_backward_workspace_size_rows",
+           "trimul_backward_block_rows",
            "trimul_workspace_size_mxfp8", "trimul_forward_mxfp8", "trimul_contract_mxfp8", "trimul_mxfp8_views",
            "trimul_prologue_mxfp8", "trimul_mma_mxfp8",
            "trimul_shard_workspace_size", "trimul_prologue_rows", "trimul_contract_channels", "trimul_epilogue_rows",
@@ -129,6 +130,7 @@ def lib():
         L.trimul_backward_workspace_size.restype = S
         L.trimul_backward_workspace_size_rows.argtypes = [I, I, I, I]
         L.trimul_backward_workspace_size_rows.restype = S
+        L.trimul_backward_block_rows.argtypes = [I, I, I, S]
         L.trimul_backward.argtypes = [P, P, PP, I, P, P, ctypes.POINTER(TrimulGrads), P]
         L.trimul_workspace_size_mxfp8.argtypes = [I, I, I]
         L.trimul_workspace_size_mxfp8.restype = S
@@ -236,6 +238,10 @@ def trimul_backward_workspace_size(N: int, c_z: int = 128, c_h: int = 128) -> in
 
 def trimul_backward_workspace_size_rows(N: int, rows: int, c_z: int = 128, c_h: int = 128) -> int:
     return lib().trimul_backward_workspace_size_rows(N, c_z, c_h, rows)
+
+
+def trimul_backward_block_rows(N: int, workspace_bytes: int, c_z: int = 128, c_h: int = 128) -> int:
+    return lib().trimul_backward_block_rows(N, c_z, c_h, workspace_bytes)
 
 
 def trimul_backward(z, mask, params: TrimulParams, direction: int, dout, dz, grads: TrimulGrads, stream=None,

@@ -1362,6 +1362,11 @@ size_t trimul_backward_workspace_size_rows(int N, int c_z, int c_h, int rows) {
     return bwd_layout(N, rows).total;
 }
 
+int trimul_backward_block_rows(int N, int c_z, int c_h, size_t workspace_bytes) {
+    if (N < 1 || N > kMaxN || c_z != kC || c_h != kC) return 0;
+    return bwd_rows_for(N, workspace_bytes);
+}
+
 int trimul_backward(const void *z, const void *mask, const trimul_params *p, int direction, const void *dout,
                     void *dz, const trimul_grads *g, trimul_stream_t stream) {
     int rc;

@@ -191,6 +191,27 @@ def test_backward_workspace_size(L):
     assert all(a < b for a, b in zip(sizes, sizes[1:]))
 
 
+def test_backward_block_rows(L):
+    """The block the call uses for a given workspace: the whole grid when it fits,
+    else the largest block whose size fits, none below one row."""
+    for N in (1, 7, 200, 768, 3605):
+        full = tm.trimul_backward_workspace_size(N)
+        assert tm.trimul_backward_block_rows(N, full) == N
+        assert tm.trimul_backward_block_rows(N, 10 * full) == N
+        one = tm.trimul_backward_workspace_size_rows(N, 1)
+        assert tm.trimul_backward_block_rows(N, one - 1) == 0
+        if N > 1:
+            for R in sorted({1, 2, N // 3, N // 2, N - 1} - {0}):
+                size = tm.trimul_backward_workspace_size_rows(N, R)
+                got = tm.trimul_backward_block_rows(N, size)
+                assert got >= R, (N, R, got)
+                if got < N:  # the largest block that fits
+                    assert tm.trimul_backward_workspace_size_rows(N, got) <= size
+                    assert got == N - 1 or tm.trimul_backward_workspace_size_rows(N, got + 1) > size
+    assert tm.trimul_backward_block_rows(0, 1 << 40) == 0
+    assert tm.trimul_backward_block_rows(64, 1 << 40, 64, 128) == 0
+
+
 DOUT = BASE + 0x100000000
 DZ = BASE + 0x140000000
 GWS = BASE + 0x200000000
